@@ -1,0 +1,93 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
+
+This module holds no attention arithmetic: it only draws random tensors and names
+the workload shapes, so both the CUDA library's callers and the fp64 oracle can be
+fed identical inputs.
+
+Recipe: a CPU ``torch.Generator`` seeded per call; ``torch.randn`` in fp32, then a
+cast to bf16 (so every value is exactly representable in both the bf16 kernel
+inputs and the fp64 oracle).  Tensors are drawn in the order Q, K, V (then dO)
+with shape ``[B, N, H, d]`` (dense) or ``[T, H, d]`` (packed variable length).
+Variable-length batches draw their lengths uniformly from ``[lo, hi]`` with their
+own generator (seed 1).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One attention forward problem: dense ``[B,N,H,d]`` or packed varlen."""
+    name: str
+    B: int
+    H: int
+    N: int              # dense sequence length, or the maximum length when varlen
+    d: int
+    causal: bool
+    q_mult: float = 1.0  # exact power-of-two multiplier applied to the bf16 Q
+    lengths: Optional[List[int]] = field(default=None)  # varlen sequence lengths
+
+    @property
+    def varlen(self) -> bool:
+        return self.lengths is not None
+
+    @property
+    def total_tokens(self) -> int:
+        return sum(self.lengths) if self.varlen else self.B * self.N
+
+    def seq_lengths(self) -> List[int]:
+        return list(self.lengths) if self.varlen else [self.N] * self.B
+
+    def cu_seqlens(self) -> List[int]:
+        cu = [0]
+        for L in self.seq_lengths():
+            cu.append(cu[-1] + L)
+        return cu
+
+
+def varlen_lengths(n: int = 16, lo: int = 512, hi: int = 16384, seed: int = 1) -> List[int]:
+    """Sequence lengths uniform in [lo, hi] from their own seeded generator."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return [int(x) for x in torch.randint(lo, hi + 1, (n,), generator=g)]
+
+
+# The five benchmark problems: tiny latency case, dense non-causal (and a variant
+# with Q scaled by 4 so the running maximum moves often), long causal, packed
+# causal varlen, and the causal backward problem.
+TINY = Workload("B1-H1-N256-d64", 1, 1, 256, 64, False)
+DENSE = Workload("B4-H16-N2048-d128", 4, 16, 2048, 128, False)
+DENSE_X4 = Workload("B4-H16-N2048-d128-qx4", 4, 16, 2048, 128, False, q_mult=4.0)
+CAUSAL = Workload("B2-H16-N8192-d128-causal", 2, 16, 8192, 128, True)
+_VL = varlen_lengths()
+VARLEN = Workload("varlen16-H16-d128-causal", len(_VL), 16, max(_VL), 128, True, lengths=_VL)
+BWD_CAUSAL = CAUSAL  # the backward problem uses the causal forward's shapes
+
+ALL = {w.name: w for w in (TINY, DENSE, DENSE_X4, CAUSAL, VARLEN)}
+
+
+def make_qkv(w: Workload, seed: int = 0, with_dout: bool = False):
+    """bf16 CPU tensors (q, k, v[, dout]) for workload ``w``.
+
+    Dense: ``[B, N, H, d]``.  Varlen: ``[T, H, d]``.
+    """
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    shape = (w.total_tokens, w.H, w.d) if w.varlen else (w.B, w.N, w.H, w.d)
+    out = []
+    for _ in range(4 if with_dout else 3):
+        out.append(torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16))
+    if w.q_mult != 1.0:
+        out[0] = (out[0].float() * w.q_mult).to(torch.bfloat16)
+    return tuple(out)
+
+
+def make_custom(B: int, N: int, H: int, d: int, seed: int = 0, lengths=None, n: int = 3,
+                std: float = 1.0):
+    """Generic seeded bf16 tensors for test shapes (dense when ``lengths`` is None)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    shape = (sum(lengths), H, d) if lengths is not None else (B, N, H, d)
+    return tuple((torch.randn(shape, generator=g, dtype=torch.float32) * std).to(torch.bfloat16)
+                 for _ in range(n))

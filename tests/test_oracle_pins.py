@@ -1,0 +1,286 @@
+"""Pins for the fp64 oracle: what fixes it to something other than itself.
+
+Each test checks the oracle against a closed form, a mathematical invariant, a
+special case that reduces to a library routine (PyTorch's fp64 CPU
+scaled_dot_product_attention / logsumexp / autograd), or finite differences.
+A plausible mistake in the oracle -- a dropped scale, a wrong sign, a transposed
+operand, an off-by-one causal mask, a missing max subtraction that overflows,
+mixed-up heads or sequences -- fails at least one of them.
+Definitions pinned: "FlashAttention 1-4 详解", section 原算法 (softmax(QK^T/sqrt(d))V),
+Online Softmax 数学推导 (two-pass softmax and the online recurrences), and the
+causal lower-triangle rule of section 其他优化.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attn_inputs import make_custom
+
+
+def _packed(t):
+    """[B,N,H,d] or [T,H,d] tensor -> fp64 numpy [T,H,d]."""
+    a = t.double().numpy()
+    return a.reshape(-1, a.shape[-2], a.shape[-1])
+
+
+def _sdpa_ref(q, k, v, causal, scale):
+    """PyTorch fp64 CPU SDPA per sequence: q/k/v [B,N,H,d] fp64 -> O [B,N,H,d]."""
+    qt, kt, vt = (x.double().permute(0, 2, 1, 3) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=causal, scale=scale)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+# ---------------------------------------------------------------- closed forms
+
+def test_two_key_closed_form():
+    """One query, keys 0 and 1, values 0 and 1, scale 1: s = (0, x),
+    O = e^x/(1+e^x) (the logistic function), LSE = ln(1+e^x).  With x = ln 3:
+    O = 3/4 and LSE = ln 4 exactly."""
+    x = math.log(3.0)
+    q = np.array([[[x]], [[0.0]]])  # token 1 is a second query we ignore
+    k = np.array([[[0.0]], [[1.0]]])
+    v = np.array([[[0.0]], [[1.0]]])
+    o, lse, _ = oracle.fwd(q, k, v, [0, 2], causal=False, scale=1.0)
+    assert abs(o[0, 0, 0] - 0.75) < 1e-15
+    assert abs(lse[0, 0] - math.log(4.0)) < 1e-15
+    # query 1 has q = 0: uniform weights -> mean of values, LSE = ln 2.
+    assert abs(o[1, 0, 0] - 0.5) < 1e-15
+    assert abs(lse[0, 1] - math.log(2.0)) < 1e-15
+
+
+def test_scale_is_applied_inside_softmax():
+    """Same two keys, scale 1/2 and q = 2 ln 3: the scaled score is ln 3 again,
+    so O = 3/4 -- a dropped or squared scale gives 9/10 or 0.63..."""
+    x = 2.0 * math.log(3.0)
+    q = np.array([[[x]], [[0.0]]])
+    k = np.array([[[0.0]], [[1.0]]])
+    v = np.array([[[0.0]], [[1.0]]])
+    o, lse, _ = oracle.fwd(q, k, v, [0, 2], causal=False, scale=0.5)
+    assert abs(o[0, 0, 0] - 0.75) < 1e-15
+    assert abs(lse[0, 0] - math.log(4.0)) < 1e-15
+
+
+def test_causal_three_token_closed_form():
+    """Causal, d=1, q = k = 1, v = (1, 2, 4), scale ln 2: every visible score is ln 2,
+    so row i averages v_0..v_i: O = (1, 1.5, 7/3); LSE_i = ln((i+1) * 2)."""
+    q = np.ones((3, 1, 1))
+    k = np.ones((3, 1, 1))
+    v = np.array([1.0, 2.0, 4.0]).reshape(3, 1, 1)
+    o, lse, _ = oracle.fwd(q, k, v, [0, 3], causal=True, scale=math.log(2.0))
+    np.testing.assert_allclose(o[:, 0, 0], [1.0, 1.5, 7.0 / 3.0], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse[0], [math.log(2 * (i + 1)) for i in range(3)], rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------------------------ invariants
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_prob_rows_sum_to_one_and_mask(causal):
+    q, k, _ = make_custom(1, 37, 2, 16, seed=3)
+    cu = [0, 37]
+    for h in range(2):
+        P = oracle.probs(_packed(q), _packed(k), cu, causal, 0.25, 0, h)
+        assert np.all(P >= 0)
+        np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+        if causal:
+            assert np.all(np.triu(P, 1) == 0.0)
+            assert P[0, 0] == 1.0
+        else:
+            assert np.all(P > 0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_v_returns_constant(causal):
+    q, k, _ = make_custom(2, 50, 3, 8, seed=4)
+    v = np.full((100, 3, 8), 0.0)
+    v[:, :, :] = np.arange(8)[None, None, :] * 0.5 - 1.0
+    o, _, _ = oracle.fwd(_packed(q), _packed(k), v, oracle.dense_cu(2, 50), causal, 0.3)
+    np.testing.assert_allclose(o, v, rtol=0, atol=1e-12)
+
+
+def test_causal_row0_returns_v0_exactly():
+    q, k, v = make_custom(2, 40, 2, 32, seed=5)
+    vp = _packed(v)
+    o, lse, _ = oracle.fwd(_packed(q), _packed(k), vp, oracle.dense_cu(2, 40), True, 0.17)
+    for b in range(2):
+        assert np.array_equal(o[b * 40], vp[b * 40])
+    # Row 0 sees one key: LSE = its scaled score.
+    qp, kp = _packed(q), _packed(k)
+    for h in range(2):
+        s00 = 0.17 * float(np.dot(qp[0, h], kp[0, h]))
+        assert abs(lse[h, 0] - s00) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_q_returns_mean_of_visible_v(causal):
+    _, k, v = make_custom(1, 33, 2, 16, seed=6)
+    q = np.zeros((33, 2, 16))
+    vp = _packed(v)
+    o, lse, _ = oracle.fwd(q, _packed(k), vp, [0, 33], causal, 0.25)
+    for i in range(33):
+        n = i + 1 if causal else 33
+        np.testing.assert_allclose(o[i], vp[:n].mean(axis=0), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[:, i], math.log(n), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_shift_invariance(causal):
+    """Adding the same constant to every score of a row changes neither O nor the
+    normalised weights; LSE moves by exactly that constant.  Realised by one extra
+    dimension: q' = [q, 1], k' = [k, c], so s'_ij = s_ij + scale*c."""
+    q, k, v = make_custom(1, 29, 2, 8, seed=7)
+    qp, kp, vp = _packed(q), _packed(k), _packed(v)
+    c = 3.0
+    q2 = np.concatenate([qp, np.ones((29, 2, 1))], axis=2)
+    k2 = np.concatenate([kp, np.full((29, 2, 1), c)], axis=2)
+    v2 = np.concatenate([vp, np.zeros((29, 2, 1))], axis=2)
+    o1, l1, _ = oracle.fwd(qp, kp, vp, [0, 29], causal, 0.5)
+    o2, l2, _ = oracle.fwd(q2, k2, v2, [0, 29], causal, 0.5)
+    np.testing.assert_allclose(o2[:, :, :8], o1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l2, l1 + 0.5 * c, rtol=0, atol=1e-12)
+
+
+def test_large_scores_do_not_overflow():
+    """Scores around 1e3 overflow exp() unless the row max is subtracted first."""
+    q, k, v = make_custom(1, 16, 1, 8, seed=8)
+    qp = _packed(q) * 200.0
+    o, lse, _ = oracle.fwd(qp, _packed(k), _packed(v), [0, 16], False, 1.0)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    assert np.max(np.abs(lse)) > 700  # the scores really are that large
+
+
+# ------------------------------------------------------- library special cases
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,N,H,d", [(1, 1, 1, 4), (2, 17, 3, 16), (1, 130, 2, 64)])
+def test_matches_torch_sdpa_fp64(B, N, H, d, causal):
+    q, k, v = make_custom(B, N, H, d, seed=11 + N)
+    o, lse, _ = oracle.fwd(_packed(q), _packed(k), _packed(v), oracle.dense_cu(B, N), causal,
+                           1.0 / math.sqrt(d))
+    ref = _sdpa_ref(q, k, v, causal, None)  # PyTorch's default scale is 1/sqrt(d)
+    np.testing.assert_allclose(o.reshape(B, N, H, d), ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_lse_matches_torch_logsumexp(causal):
+    B, N, H, d = 2, 23, 2, 16
+    scale = 0.3
+    q, k, v = make_custom(B, N, H, d, seed=12)
+    _, lse, _ = oracle.fwd(_packed(q), _packed(k), _packed(v), oracle.dense_cu(B, N), causal, scale)
+    lse = oracle.lse_to_dense(lse, B, N)
+    s = torch.einsum("bihc,bjhc->bhij", q.double(), k.double()) * scale
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(N, N, dtype=torch.bool), 1), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equals_per_sequence_sdpa(causal):
+    lengths = [5, 1, 40, 17]
+    H, d = 2, 16
+    q, k, v = make_custom(0, 0, H, d, seed=13, lengths=lengths)
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    o, lse, _ = oracle.fwd(_packed(q), _packed(k), _packed(v), cu, causal, 0.25)
+    for b, L in enumerate(lengths):
+        sl = slice(cu[b], cu[b + 1])
+        ref = _sdpa_ref(q[sl][None], k[sl][None], v[sl][None], causal, 0.25)[0]
+        np.testing.assert_allclose(o[sl], ref, rtol=0, atol=1e-12)
+
+
+def test_fwd_rows_equals_fwd():
+    lengths = [70, 3, 129]
+    q, k, v = make_custom(0, 0, 3, 32, seed=14, lengths=lengths)
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    o, lse, _ = oracle.fwd(_packed(q), _packed(k), _packed(v), cu, True, 0.2)
+    rows = np.array([0, 69, 70, 72, 73, 150, 201])
+    heads = np.array([0, 2, 1, 0, 2, 1, 0])
+    o_r, l_r = oracle.fwd_rows(_packed(q), _packed(k), _packed(v), cu, True, 0.2, rows, heads)
+    np.testing.assert_allclose(o_r, o[rows, heads], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l_r, lse[heads, rows], rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------ online softmax == two-pass
+
+@pytest.mark.parametrize("Br,Bc", [(1, 1), (16, 16), (128, 128), (7, 5), (64, 128)])
+@pytest.mark.parametrize("tau", [0.0, 8.0 * math.log(2.0), 1e9])
+@pytest.mark.parametrize("causal", [False, True])
+def test_online_equals_two_pass(Br, Bc, tau, causal):
+    lengths = [131, 45]
+    q, k, v = make_custom(0, 0, 2, 16, seed=15, lengths=lengths, std=2.0)
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    args = (_packed(q), _packed(k), _packed(v), cu, causal, 0.4)
+    o_ref, l_ref, _ = oracle.fwd(*args)
+    o, l, n = oracle.online_fwd(*args, Br, Bc, tau)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l, l_ref, rtol=0, atol=1e-12)
+    if tau >= 1e9 or Bc >= 131:
+        assert n == 0
+
+
+def test_rescale_count_falls_with_threshold():
+    q, k, v = make_custom(1, 512, 2, 32, seed=16, std=2.0)
+    args = (_packed(q), _packed(k), _packed(v), [0, 512], False, 0.5)
+    counts = [oracle.online_fwd(*args, 128, 32, tau)[2] for tau in (0.0, 1.0, 4.0, 1e9)]
+    assert counts[0] > 0 and counts[-1] == 0
+    assert all(a >= b for a, b in zip(counts, counts[1:]))
+
+
+# ------------------------------------------------------------------- backward
+
+def _loss_grad_torch(q, k, v, dout, causal, scale):
+    qt, kt, vt = (x.double().permute(0, 2, 1, 3).requires_grad_(True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=causal, scale=scale)
+    (o * dout.double().permute(0, 2, 1, 3)).sum().backward()
+    return [t.grad.permute(0, 2, 1, 3).numpy() for t in (qt, kt, vt)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_matches_torch_autograd_fp64(causal):
+    B, N, H, d = 2, 19, 2, 8
+    q, k, v, do = make_custom(B, N, H, d, seed=17, n=4)
+    grads = oracle.bwd(_packed(q), _packed(k), _packed(v), _packed(do), oracle.dense_cu(B, N),
+                       causal, 0.35)
+    ref = _loss_grad_torch(q, k, v, do, causal, 0.35)
+    for g, r in zip(grads, ref):
+        np.testing.assert_allclose(g.reshape(B, N, H, d), r, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_central_finite_differences(causal):
+    """dL/dx for L = sum(dO * O), by central differences on a tiny problem."""
+    lengths = [6, 4]
+    H, d = 1, 3
+    q, k, v, do = (t.double().numpy() for t in make_custom(0, 0, H, d, seed=18, lengths=lengths, n=4))
+    cu = np.array([0, 6, 10])
+    scale = 0.7
+    grads = oracle.bwd(q, k, v, do, cu, causal, scale)
+
+    def loss(qq, kk, vv):
+        o, _, _ = oracle.fwd(qq, kk, vv, cu, causal, scale)
+        return float(np.sum(o * do))
+
+    eps = 1e-6
+    for which, g in enumerate(grads):
+        base = [q, k, v]
+        num = np.zeros_like(g)
+        for idx in np.ndindex(g.shape):
+            plus = [a.copy() for a in base]
+            minus = [a.copy() for a in base]
+            plus[which][idx] += eps
+            minus[which][idx] -= eps
+            num[idx] = (loss(*plus) - loss(*minus)) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_key_shift_invariance(causal):
+    """Adding one vector c to every key adds scale*<q_i,c> to each score of row i,
+    which the softmax ignores; so sum_j dK_j = 0 for every (sequence, head)."""
+    lengths = [33, 12]
+    q, k, v, do = make_custom(0, 0, 2, 16, seed=19, lengths=lengths, n=4)
+    cu = np.array([0, 33, 45])
+    _, dk, _ = oracle.bwd(_packed(q), _packed(k), _packed(v), _packed(do), cu, causal, 0.25)
+    for b in range(2):
+        np.testing.assert_allclose(dk[cu[b]:cu[b + 1]].sum(axis=0), 0.0, rtol=0, atol=1e-11)
