@@ -1,0 +1,347 @@
+"""Benchmark: exact-attention forward TFLOP/s on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one forward pass (the whole hot path: schedule, TMA loads, S = QK^T,
+online softmax, O += PV, epilogue) over one batch of the workload, inputs
+resident in HBM.  L2 is flushed (a 256 MiB write) before every timed step; the
+flush is outside the CUDA-event-timed interval.  FLOPs: 4*B*H*N^2*d, halved for
+causal, summed per sequence for varlen.
+
+N > 1 (torchrun): every rank runs an independent replica of the workload on its
+own GPU (the forward pass needs no exchange); value = all ranks' FLOPs / the
+slowest rank's time (max over ranks).
+
+--impl reference times the fp64 CPU oracle (the correctness reference, not a
+tuned program) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import attn_inputs as ai  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (bf16, d=128, 1 B200) and % of dense-BF16 tensor peak"
+FLUSH_BYTES = 256 << 20
+MUFU_EX2_PER_CLK_PER_SM = 16  # 4 SFU lanes per SM sub-partition, 4 sub-partitions
+
+
+def workload_flops(w: ai.Workload) -> float:
+    per_seq = [4.0 * w.H * L * L * w.d for L in w.seq_lengths()]
+    total = sum(per_seq)
+    return total / 2.0 if w.causal else total
+
+
+def workload_exps(w: ai.Workload) -> float:
+    """Score elements the method exponentiates (visible (query, key) pairs)."""
+    return workload_flops(w) / (4.0 * w.d)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"),
+                "sm_max_mhz": p.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML unavailable: report no samples
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        for name, bit in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+            if not self.samples:
+                try:
+                    self._sample()
+                except Exception:
+                    pass
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def dist_setup(gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def make_inputs(w: ai.Workload, device):
+    q, k, v = ai.make_qkv(w)
+    cu = None
+    if w.varlen:
+        cu = torch.tensor(w.cu_seqlens(), dtype=torch.int32)
+    return q, k, v, cu
+
+
+def cpu_oracle_sample(w: ai.Workload, q, k, v, budget_s: float):
+    """Times the fp64 oracle on whole (sequence, head) units of the workload until
+    about budget_s of CPU time is spent; returns (TFLOP/s, threads, description)."""
+    import numpy as np
+    import oracle
+    lengths = w.seq_lengths()
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    qp, kp, vp = (t.reshape(-1, w.H, w.d) for t in (q, k, v))
+    scale = 1.0 / math.sqrt(w.d)
+    done_flops, spent, units, threads = 0.0, 0.0, 0, 0
+    order = sorted(range(len(lengths)), key=lambda b: lengths[b])  # cheapest sequences first
+    for b in order:
+        L = lengths[b]
+        sl = slice(int(cu[b]), int(cu[b + 1]))
+        for h in range(w.H):
+            rows = np.arange(cu[b], cu[b + 1])
+            heads = np.full(L, h)
+            t0 = time.perf_counter()
+            oracle.fwd_rows(qp, kp, vp, cu, w.causal, scale, rows, heads)
+            spent += time.perf_counter() - t0
+            f = 4.0 * L * L * w.d * (0.5 if w.causal else 1.0)
+            done_flops += f
+            units += 1
+            if spent >= budget_s:
+                break
+        if spent >= budget_s:
+            break
+        del sl
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    desc = f"{units} of {len(lengths) * w.H} (sequence, head) units, {done_flops / 1e9:.1f} GFLOP"
+    return done_flops / spent / 1e12, threads, desc
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = ai.ALL[args.workload]
+    q, k, v, _ = make_inputs(w, "cpu")
+    flops = workload_flops(w)
+    # warm-up: build / load the oracle
+    import oracle
+    oracle.build()
+    vals = []
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        tf, threads, desc = cpu_oracle_sample(w, q, k, v, per_step)
+        if i >= args.warmup:
+            vals.append(tf)
+    value = statistics.median(vals)
+    ms = flops / (value * 1e12) * 1e3
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "causal": w.causal, "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": desc + " per step; ms_per_step extrapolated to the workload"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local):
+    import exact_attention_103_b200 as ea
+    ea.load_library()
+    w = ai.ALL[args.workload]
+    dev = torch.device("cuda", local)
+    q_h, k_h, v_h, cu_h = make_inputs(w, "cpu")
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    cu = None if cu_h is None else cu_h.to(dev)
+    max_len = w.N if w.varlen else None
+    scale = 1.0 / math.sqrt(w.d)
+    out = torch.empty_like(q)
+    lse_shape = (w.H, w.total_tokens) if w.varlen else (w.B, w.H, w.N)
+    lse = torch.empty(lse_shape, dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flops = workload_flops(w)
+    peaks = load_peaks()
+
+    def step():
+        ea.fwd(q, k, v, causal=w.causal, scale=scale, cu_seqlens=cu, max_seqlen=max_len,
+               out=out, lse=lse)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    ea.get_device_status()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ea.get_device_status()
+    times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(times), world)
+    ms_per_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    achieved = flops / (statistics.mean(times) / 1e3) / 1e12  # per launch, this rank
+    peak = peaks["bf16_tflops"]
+    clk = clocks.summary()
+    mhz = clk["sm_mhz"] or peaks["sm_max_mhz"]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mufu_peak = sms * MUFU_EX2_PER_CLK_PER_SM * mhz * 1e6
+    mufu_achieved = workload_exps(w) / (statistics.mean(times) / 1e3)
+
+    # End to end through the public API from pinned host buffers: H2D of Q/K/V
+    # (and cu_seqlens), the forward, D2H of O and LSE, every step.
+    q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
+    cu_p = None if cu_h is None else cu_h.pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        ea.fwd_from_host(q_p, k_p, v_p, causal=w.causal, scale=scale, cu_seqlens_host=cu_p,
+                         max_seqlen=max_len)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        o_h, l_h = ea.fwd_from_host(q_p, k_p, v_p, causal=w.causal, scale=scale,
+                                    cu_seqlens_host=cu_p, max_seqlen=max_len)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    h2d = 3 * q_h.numel() * 2 + (0 if cu_h is None else cu_h.numel() * 4)
+    d2h = o_h.numel() * 2 + l_h.numel() * 4
+    barrier(world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, threads, desc = cpu_oracle_sample(w, q_h, k_h, v_h, args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                           "causal": w.causal, "global_batch": w.B * world,
+                           "seq_len": w.N, "parallelism": f"replicas{world}",
+                           "l2": "flushed (256 MiB write) before every timed step"},
+                "pct_of_peak": 100.0 * achieved / peak,
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                             "unit": "TFLOP/s", "frac": achieved / peak,
+                             "peak_source": f"bf16_tflops (burst), {peaks['source']}",
+                             "traffic": None},
+                "mufu": {"achieved_ex2_per_s": mufu_achieved, "peak_ex2_per_s": mufu_peak,
+                         "frac": mufu_achieved / mufu_peak,
+                         "note": "all exponentials on MUFU ex2; peak at the median sampled SM clock"},
+                "e2e": {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                        "ms_per_step": e2e_ms},
+                "gpu_launches": args.steps,
+                "clocks": clk,
+                "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=ai.DENSE.name, choices=sorted(ai.ALL))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, rank, world)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

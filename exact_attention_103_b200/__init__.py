@@ -1,0 +1,215 @@
+"""Python binding of libattn: B200-native exact attention.
+
+Argument marshalling only.  Every step of the computation runs in the CUDA
+library ``libattn.so`` (built in-tree by ``build.py``); this module checks torch
+tensors, allocates outputs with torch, and passes raw device pointers and the
+current CUDA stream through the C ABI declared in ``include/attn.h``.  There is no
+fallback: if the library is missing or the device is not an sm_100 GPU, calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED = 0, 1, 2
+ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_WORKSPACE = 3, 4, 5
+
+# Every symbol include/attn.h and include/attn_selftest.h declare.
+EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_ex", "attn_bwd", "attn_bwd_workspace_size",
+                    "attn_get_device_status", "attn_status_string", "attn_last_error",
+                    "attn_selftest_umma")
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{status_string(status) if _lib else status}: {message}")
+        self.status = status
+
+
+class FwdOpts(ctypes.Structure):
+    _fields_ = [("rescale_threshold", ctypes.c_float),
+                ("stats", ctypes.c_void_p),
+                ("timeout_ns", ctypes.c_uint64),
+                ("total_tokens", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads libattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libattn.so not found at {path}; build it with "
+                           "`python -m exact_attention_103_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, ci, cf, cs = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp]
+    lib.attn_fwd.restype = ci
+    lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp,
+                                ctypes.POINTER(FwdOpts), vp]
+    lib.attn_fwd_ex.restype = ci
+    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, ci,
+                             vp, cs, vp]
+    lib.attn_bwd.restype = ci
+    lib.attn_bwd_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci]
+    lib.attn_bwd_workspace_size.restype = cs
+    lib.attn_get_device_status.argtypes = [vp]
+    lib.attn_get_device_status.restype = ci
+    lib.attn_status_string.argtypes = [ci]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_last_error.argtypes = []
+    lib.attn_last_error.restype = ctypes.c_char_p
+    lib.attn_selftest_umma.argtypes = [vp, vp, vp, vp, vp, ci, vp]
+    lib.attn_selftest_umma.restype = ci
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().attn_status_string(status).decode()
+
+
+def last_error() -> str:
+    return load_library().attn_last_error().decode()
+
+
+def _check(status: int):
+    if status != ATTN_OK:
+        raise AttnError(status, last_error())
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+        scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
+        max_seqlen: Optional[int] = None, out: Optional[torch.Tensor] = None,
+        lse: Optional[torch.Tensor] = None, rescale_threshold: Optional[float] = None,
+        stats: Optional[torch.Tensor] = None, timeout_ns: int = 0,
+        stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Exact attention forward on the GPU.
+
+    Dense: q, k, v are bf16 ``[B, N, H, d]``; returns O ``[B, N, H, d]`` and LSE
+    ``[B, H, N]`` (fp32, natural log).  Varlen: q, k, v are packed ``[T, H, d]``,
+    ``cu_seqlens`` is int32 ``[B+1]`` on the device and ``max_seqlen`` the longest
+    sequence; LSE is ``[H, T]``.  ``scale`` defaults to ``1/sqrt(d)``.
+    """
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape")
+    d = q.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    opts = FwdOpts(-1.0 if rescale_threshold is None else float(rescale_threshold),
+                   None if stats is None else stats.data_ptr(), int(timeout_ns), 0)
+    if stats is not None:
+        _need(stats, "stats", torch.int64)
+    if cu_seqlens is None:
+        if q.dim() != 4:
+            raise ValueError("dense q must be [B, N, H, d]")
+        B, N, H, _ = q.shape
+        lse_shape = (B, H, N)
+    else:
+        if q.dim() != 3:
+            raise ValueError("varlen q must be [T, H, d]")
+        _need(cu_seqlens, "cu_seqlens", torch.int32)
+        B = cu_seqlens.numel() - 1
+        H = q.shape[1]
+        if max_seqlen is None:
+            raise ValueError("varlen needs max_seqlen")
+        N = int(max_seqlen)
+        lse_shape = (H, q.shape[0])
+        opts.total_tokens = q.shape[0]
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out")
+        if out.shape != q.shape:
+            raise ValueError("out has the wrong shape")
+    if lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    else:
+        _need(lse, "lse", torch.float32)
+        if tuple(lse.shape) != lse_shape:
+            raise ValueError("lse has the wrong shape")
+    if cu_seqlens is not None and q.shape[0] == 0:
+        return out, lse
+    with torch.cuda.device(q.device):
+        st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                             None if cu_seqlens is None else cu_seqlens.data_ptr(),
+                             ctypes.byref(opts), _stream_ptr(stream))
+    _check(st)
+    return out, lse
+
+
+def fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int, N: int,
+            d: int, causal: bool, scale: float, cu_ptr: Optional[int] = None,
+            stream_ptr: int = 0) -> None:
+    """The plain C entry point ``attn_fwd`` on raw device pointers."""
+    _check(load_library().attn_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d,
+                                   int(bool(causal)), float(scale), cu_ptr, stream_ptr))
+
+
+def fwd_from_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
+                  causal: bool = False, scale: Optional[float] = None,
+                  cu_seqlens_host: Optional[torch.Tensor] = None,
+                  max_seqlen: Optional[int] = None, device: str = "cuda",
+                  stream: Optional[torch.cuda.Stream] = None):
+    """End-to-end call from (pinned) host tensors: copies Q/K/V (and cu_seqlens) to
+    the device, runs the forward, copies O and LSE back to host tensors."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    with torch.cuda.stream(s):
+        q = q_host.to(device, non_blocking=True)
+        k = k_host.to(device, non_blocking=True)
+        v = v_host.to(device, non_blocking=True)
+        cu = None if cu_seqlens_host is None else cu_seqlens_host.to(device, non_blocking=True)
+        o, lse = fwd(q, k, v, causal=causal, scale=scale, cu_seqlens=cu, max_seqlen=max_seqlen,
+                     stream=s)
+        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        o_h.copy_(o, non_blocking=True)
+        l_h.copy_(lse, non_blocking=True)
+    return o_h, l_h
+
+
+def get_device_status(stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Synchronises the stream; raises AttnError if a kernel recorded an error."""
+    _check(load_library().attn_get_device_status(_stream_ptr(stream)))
+
+
+def selftest_umma(a: torch.Tensor, b: torch.Tensor, v: torch.Tensor):
+    """Runs the one-tile tensor-core check: returns (S = A B^T, O = bf16(S) V), fp32."""
+    for t, n in ((a, "a"), (b, "b"), (v, "v")):
+        _need(t, n)
+    d = a.shape[1]
+    s_out = torch.empty((128, 128), dtype=torch.float32, device=a.device)
+    o_out = torch.empty((128, d), dtype=torch.float32, device=a.device)
+    _check(load_library().attn_selftest_umma(a.data_ptr(), b.data_ptr(), v.data_ptr(),
+                                             s_out.data_ptr(), o_out.data_ptr(), d,
+                                             _stream_ptr(None)))
+    return s_out, o_out

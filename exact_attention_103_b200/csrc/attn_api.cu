@@ -1,0 +1,251 @@
+// attn_api.cu -- the C ABI of libattn (declared in include/attn.h): argument
+// validation, TMA descriptor construction, per-device state, and launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "attn_fwd_sm100.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+attn_status_t fail(attn_status_t s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+attn_status_t fail(attn_status_t s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+attn_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(ATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int sms = 0;
+  int* err = nullptr;  // device error word
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+// Lazily prepares the current device: checks for sm_100, allocates the error word.
+attn_status_t device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(ATTN_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    if (prop.major != 10 || prop.minor != 0)
+      return fail(ATTN_ERR_UNSUPPORTED, "libattn needs an sm_100 GPU (B200); device %d is sm_%d%d",
+                  dev, prop.major, prop.minor);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+      if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+        return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    e = cudaMalloc(&st.err, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(error word)");
+    e = cudaMemset(st.err, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(error word)");
+    st.sms = prop.multiProcessorCount;
+    st.ready = true;
+  }
+  *out = &st;
+  return ATTN_OK;
+}
+
+// 3-D bf16 view {d, H, total} of a token-major [total, H, d] tensor; box
+// {64, 1, 128} (one 128-byte swizzle chunk by 128 rows), 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, int64_t total, int H, int d) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(total)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(H) * d * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+constexpr float kDefaultTau = 8.0f;
+constexpr int kMaxVarlenB = 1024;
+constexpr int kMaxVarlenN = 131072;
+
+attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
+                       int64_t total_hint, const attn_fwd_opts_t* opts, attn_stream_t stream) {
+  if (B < 0 || H <= 0 || N < 0) return fail(ATTN_ERR_INVALID_ARG, "B=%d H=%d N=%d", B, H, N);
+  if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (!(std::isfinite(scale) && scale > 0.f)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (B == 0 || N == 0) return ATTN_OK;
+  if (!q || !k || !v || !o || !lse) return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return fail(ATTN_ERR_INVALID_ARG, "q/k/v/o must be 16-byte aligned and lse 4-byte aligned");
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen && (B > kMaxVarlenB || N > kMaxVarlenN))
+    return fail(ATTN_ERR_UNSUPPORTED, "varlen supports B <= %d and N <= %d", kMaxVarlenB, kMaxVarlenN);
+  const int64_t T256 = (static_cast<int64_t>(N) + 255) / 256;
+  const int64_t items_bound = static_cast<int64_t>(B) * T256 * H;
+  const int64_t dense_tokens = static_cast<int64_t>(B) * N;
+  if (items_bound > INT32_MAX / 2 || dense_tokens * H > INT64_MAX / 256 || dense_tokens > INT32_MAX)
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for 32-bit tile indexing");
+  if (varlen && !aligned(cu_seqlens, 4)) return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens misaligned");
+  float tau = kDefaultTau;
+  uint64_t timeout = kDefaultTimeoutNs;
+  unsigned long long* stats = nullptr;
+  if (opts) {
+    if (opts->rescale_threshold >= 0.f) tau = opts->rescale_threshold;
+    if (!std::isfinite(tau)) return fail(ATTN_ERR_INVALID_ARG, "rescale_threshold must be finite");
+    if (opts->timeout_ns) timeout = opts->timeout_ns;
+    stats = opts->stats;
+    if (stats && !aligned(stats, 8)) return fail(ATTN_ERR_INVALID_ARG, "stats misaligned");
+  }
+
+  DeviceState* dev = nullptr;
+  attn_status_t st = device_state(&dev);
+  if (st != ATTN_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  int64_t total = dense_tokens;
+  if (varlen) {
+    if (total_hint >= 0) {
+      total = total_hint;
+    } else {
+      // The TMA views need the packed token count; read cu_seqlens[B] (4 bytes).
+      int32_t t = 0;
+      cudaError_t e = cudaMemcpyAsync(&t, cu_seqlens + B, sizeof(int32_t), cudaMemcpyDeviceToHost, cs);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+      if (e != cudaSuccess) return cuda_fail(e, "reading cu_seqlens[B]");
+      total = t;
+    }
+    if (total < 0 || total > dense_tokens)
+      return fail(ATTN_ERR_INVALID_ARG, "packed token count %lld outside [0, B*N]", (long long)total);
+    if (total == 0) return ATTN_OK;
+  }
+
+  attn::FwdLaunch a;
+  std::memset(&a, 0, sizeof(a));
+  if (!make_map(&a.tm_q, q, total, H, d) || !make_map(&a.tm_k, k, total, H, d) ||
+      !make_map(&a.tm_v, v, total, H, d))
+    return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled rejected the Q/K/V views");
+  a.p.o = static_cast<__nv_bfloat16*>(o);
+  a.p.lse = lse;
+  a.p.cu_seqlens = cu_seqlens;
+  a.p.B = B;
+  a.p.H = H;
+  a.p.N = N;
+  a.p.T = static_cast<int>(T256);
+  a.p.total = static_cast<int>(total);
+  a.p.scale_log2 = scale * 1.4426950408889634f;
+  a.p.tau = tau;
+  a.p.err = dev->err;
+  a.p.stats = stats;
+  a.p.timeout_ns = timeout;
+  a.grid = static_cast<int>(items_bound < dev->sms ? items_bound : dev->sms);
+  a.smem = attn::fwd_smem_bytes(d, B, static_cast<int>(T256), varlen ? 1 : 0);
+  const cudaError_t e = attn::launch_fwd(a, d, causal ? 1 : 0, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
+  return ATTN_OK;
+}
+
+}  // namespace
+
+namespace attn_internal {
+// Device preparation and the TMA view builder, for the diagnostic entry point.
+attn_status_t prepare_selftest(int** err, bool (**mk)(CUtensorMap*, const void*, int64_t, int, int)) {
+  DeviceState* dev = nullptr;
+  const attn_status_t st = device_state(&dev);
+  if (st != ATTN_OK) return st;
+  *err = dev->err;
+  *mk = make_map;
+  return ATTN_OK;
+}
+}  // namespace attn_internal
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
+                       attn_stream_t stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, -1, nullptr, stream);
+}
+
+attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
+                          const attn_fwd_opts_t* opts, attn_stream_t stream) {
+  const int64_t hint = (opts && opts->total_tokens > 0) ? opts->total_tokens : -1;
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, hint, opts, stream);
+}
+
+attn_status_t attn_bwd(const void*, const void*, const void*, const void*, const float*,
+                       const void*, void*, void*, void*, int, int, int, int, int, float,
+                       const int32_t*, int, void*, size_t, attn_stream_t) {
+  return fail(ATTN_ERR_UNSUPPORTED, "attn_bwd is not provided by this build");
+}
+
+size_t attn_bwd_workspace_size(int, int, int, int, int, int) { return 0; }
+
+attn_status_t attn_get_device_status(attn_stream_t stream) {
+  DeviceState* dev = nullptr;
+  attn_status_t st = device_state(&dev);
+  if (st != ATTN_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int word = 0;
+  e = cudaMemcpy(&word, dev->err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (word == 0) return ATTN_OK;
+  e = cudaMemset(dev->err, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  const int code = word & 0xff, site = word >> 8;
+  return fail(static_cast<attn_status_t>(code), "device error %d recorded at site %d", code, site);
+}
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+  }
+  return "unknown attn_status_t";
+}
+
+const char* attn_last_error(void) { return g_last_error; }
+
+}  // extern "C"

@@ -1,0 +1,554 @@
+// attn_fwd_sm100.cu -- fused exact-attention forward kernel for B200 (sm_100a).
+//
+// One persistent CTA per SM walks a static list of work items.  A work item is
+// (sequence b, head h, query tile-pair t): 256 query rows split into two 128-row
+// sub-tiles that share every K/V tile, so the tensor core alternates between the
+// two sub-tiles while the other one's softmax runs ("FlashAttention V4 deep-dive"
+// (pnsm.cn), section 3.1, two Q tiles in ping-pong).
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax + epilogue of sub-tile 0 (one thread per query row)
+//   warps 4-7  softmax + epilogue of sub-tile 1
+//   warp  8    TMA producer: Q pair, then K_j / V_j tiles into an smem ring
+//   warp  9    TMEM owner and tcgen05.mma issuer (one elected lane)
+//
+// Per sub-tile s and key tile j ("FlashAttention 1-4 详解", FlashAttention 1 /
+// Online Softmax 数学推导; FlashAttention 2 / 减少非矩阵乘运算占比):
+//   S_s = Q_s K_j^T                    tcgen05.mma, A and B from smem, fp32 in TMEM
+//   m   = rowmax(scale*S) (log2 units) the row's own thread, from TMEM
+//   conditional rescale: only when m exceeds the reference maximum by > tau
+//       ("FlashAttention V4 deep-dive", section 3.2; "FlashAttention 1-4 详解",
+//        FlashAttention 4 / 三项核心技术 (2)): O_s, l scaled by 2^(m_ref - m)
+//   P~  = 2^(scale*S*log2e - m_ref)    MUFU ex2; l += sum P~ (fp32, before rounding)
+//   P~ -> bf16, written back over S_s in TMEM
+//   O_s += P~ V_j                      tcgen05.mma, A = P~ from TMEM, B = V from smem
+// after the last key tile: O = O_s / l -> bf16 -> global; LSE = ln2*(m_ref + log2 l).
+// Causal items skip key tiles above the diagonal ("FlashAttention 1-4 详解",
+// 其他优化 / FlashAttention 2 的工程优化) and mask the diagonal tile; packed
+// variable-length batches mask keys past the sequence end.
+//
+// Scheduling ("FlashAttention V4 deep-dive", section 3.4 dynamic tile scheduling;
+// FlashAttention-4 summary (reportify.cn) item [14], the new tile scheduler):
+// items are ordered longest-first (causal: by tile-pair index t, descending) and
+// dealt to CTAs in a snake order (wave k goes left-to-right when k is even,
+// right-to-left when odd), which balances causal and varlen work without atomics.
+//
+// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D, 256+2D).
+// Every wait is bounded (see sm100_ptx.cuh); on expiry the CTA stops, drains
+// its in-flight copies and MMAs, frees TMEM and returns.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "attn_fwd_sm100.h"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kBM = 128;  // query rows per sub-tile
+constexpr int kBN = 128;  // keys per key tile
+constexpr float kLn2 = 0.693147180559945309f;
+
+// Error codes recorded in the device error word: 4 (= ATTN_ERR_TIMEOUT) in the
+// low byte, the waiting site above it.
+__host__ __device__ constexpr int timeout_code(int site) { return 4 | (site << 8); }
+enum WaitSite {
+  kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteOFull,
+  kSiteDrain, kSiteBadLen
+};
+
+template <int D>
+struct Layout {
+  static constexpr int TILE = kBM * D * 2;            // bytes of one 128 x D bf16 tile
+  static constexpr int CHUNK = kBM * 128;             // one 64-column swizzle chunk
+  static constexpr int NSTAGE = (D == 128) ? 4 : 8;   // K/V ring slots
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = 2 * TILE;
+  static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE;
+  // barrier indices
+  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_OFULL = 6,
+                       B_DRAIN = 8, B_KVFULL = 9, B_KVEMPTY = 9 + NSTAGE;
+  static constexpr int NBARS = 9 + 2 * NSTAGE;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int TABLE_OFF = MISC_OFF + 64;
+  static constexpr int TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
+};
+
+// Work-item decoding shared by every role (all roles walk the same list).
+struct Sched {
+  const int* cu;  // device cu_seqlens or null (dense)
+  int B, H, N, T;
+  const int* order;  // varlen: sequences sorted by tile-pair count, descending
+  const int* start;  // varlen: first pair index of bucket t (buckets by t descending)
+  int count;         // number of items
+
+  __device__ __forceinline__ int item(int k) const {
+    const int G = gridDim.x, c = blockIdx.x;
+    const int idx = k * G + ((k & 1) ? (G - 1 - c) : c);
+    return idx < count ? idx : -1;
+  }
+  __device__ __forceinline__ void decode(int idx, int& b, int& t, int& h, int& seq_start,
+                                         int& L) const {
+    const int pr = idx / H;
+    h = idx - pr * H;
+    if (cu == nullptr) {
+      const int tt = pr / B;
+      t = T - 1 - tt;
+      b = pr - tt * B;
+      seq_start = b * N;
+      L = N;
+    } else {
+      int lo = 0, hi = T - 1;  // smallest t with start[t] <= pr
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (start[mid] <= pr) hi = mid; else lo = mid + 1;
+      }
+      t = lo;
+      b = order[pr - start[lo]];
+      seq_start = __ldg(cu + b);
+      L = __ldg(cu + b + 1) - seq_start;
+    }
+  }
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Key tiles sub-tile s of pair t processes (0 when its rows are all past L).
+template <bool CAUSAL>
+__device__ __forceinline__ int num_kv_tiles(int t, int s, int L) {
+  const int row0 = t * 2 * kBM + s * kBM;
+  if (row0 >= L) return 0;
+  const int all = ceil_div(L, kBN);
+  if (!CAUSAL) return all;
+  const int diag = row0 / kBN + 1;  // tiles up to and including the diagonal
+  return diag < all ? diag : all;
+}
+
+// Inclusive warp scan (sum) of one value per lane.
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// Builds the varlen tables (one warp).  tab layout: order[B] | off[T+1] | cnt[T] | start[T].
+// Returns the number of (sequence, tile-pair) pairs, or -1 if cu[0] != 0,
+// cu[B] != total, or some length is negative or exceeds T*256.
+__device__ int build_varlen_tables(const int* cu, int B, int T, int total, int* tab, int lane) {
+  int* order = tab;
+  int* off = tab + B;
+  int* cnt = off + T + 1;
+  int* start = cnt + T;
+  for (int i = lane; i <= T; i += 32) off[i] = 0;
+  __syncwarp();
+  int bad = (lane == 0 && (__ldg(cu) != 0 || __ldg(cu + B) != total)) ? 1 : 0;
+  for (int b = lane; b < B; b += 32) {
+    const int L = __ldg(cu + b + 1) - __ldg(cu + b);
+    const int nt = L < 0 ? 0 : ceil_div(L, 2 * kBM);
+    if (L < 0 || nt > T) { bad = 1; continue; }
+    atomicAdd(&off[nt], 1);
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  __syncwarp();
+  if (bad) return -1;
+  // off[n] = #{b : nt_b > n}: exclusive suffix scan of the histogram from n = T down.
+  int carry = 0;
+  for (int base = 0; base <= T; base += 32) {
+    const int n = T - (base + lane);
+    const int v = n >= 0 ? off[n] : 0;
+    const int incl = warp_incl_scan(v, lane);
+    __syncwarp();
+    if (n >= 0) off[n] = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+    __syncwarp();
+  }
+  for (int t = lane; t < T; t += 32) cnt[t] = off[t];
+  __syncwarp();
+  // Stable placement of sequences by tile-pair count, descending.
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < B; base += 32) {
+    const int b = base + lane;
+    int key = -1;
+    if (b < B) key = ceil_div(__ldg(cu + b + 1) - __ldg(cu + b), 2 * kBM);
+    const uint32_t same = __match_any_sync(0xffffffffu, key);
+    const int rank = __popc(same & lt_mask);
+    if (b < B) order[off[key] + rank] = b;
+    __syncwarp();
+    if (b < B && lane == __ffs(same) - 1) off[key] += __popc(same);
+    __syncwarp();
+  }
+  // start[t] = sum_{t' > t} cnt[t']: exclusive suffix scan over t = T-1 down.
+  carry = 0;
+  for (int base = 0; base < T; base += 32) {
+    const int t = T - 1 - (base + lane);
+    const int v = t >= 0 ? cnt[t] : 0;
+    const int incl = warp_incl_scan(v, lane);
+    if (t >= 0) start[t] = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+  return carry;  // total pairs
+}
+
+// Bounded wait that ignores the abort flag (used to drain before exit).
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using Lay = Layout<D>;
+  constexpr int NS = Lay::NSTAGE;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+  // misc[0] TMEM base, misc[1] abort flag, misc[2] item count
+  int* tab = reinterpret_cast<int*>(smem + Lay::TABLE_OFF);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(Lay::B_QFULL), 1);
+    mbar_init(bar(Lay::B_QEMPTY), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(Lay::B_SFULL + s), 1);
+      mbar_init(bar(Lay::B_PFULL + s), 128);
+      mbar_init(bar(Lay::B_OFULL + s), 1);
+    }
+    mbar_init(bar(Lay::B_DRAIN), 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(bar(Lay::B_KVFULL + i), 1);
+      mbar_init(bar(Lay::B_KVEMPTY + i), 1);
+    }
+    misc[1] = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(sb + Lay::MISC_OFF, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8) {
+    int count;
+    if (p.cu_seqlens == nullptr) {
+      count = p.B * p.T * p.H;
+    } else {
+      const int pairs = build_varlen_tables(p.cu_seqlens, p.B, p.T, p.total, tab, lane);
+      if (pairs < 0) {
+        count = 0;
+        if (lane == 0 && p.err) atomicCAS(p.err, 0, 1 | (kSiteBadLen << 8));
+      } else {
+        count = pairs * p.H;
+      }
+    }
+    if (lane == 0) misc[2] = static_cast<uint32_t>(count);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = misc[0];
+  Sched sch;
+  sch.cu = p.cu_seqlens;
+  sch.B = p.B; sch.H = p.H; sch.N = p.N; sch.T = p.T;
+  sch.order = tab;
+  sch.start = tab + p.B + 2 * p.T + 1;
+  sch.count = static_cast<int>(misc[2]);
+  WaitCtl wc;
+  wc.abort = reinterpret_cast<volatile uint32_t*>(misc + 1);
+  wc.err = p.err;
+  wc.limit_ns = p.timeout_ns;
+
+  if (warp < 8) {
+    // ------------------------------------------------------------ softmax
+    const int s = warp >> 2, wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t t_s = tmem + lane_bits + (s ? Lay::TM_S1 : Lay::TM_S0);
+    const uint32_t t_o = tmem + lane_bits + (s ? Lay::TM_O1 : Lay::TM_O0);
+    const float sl = p.scale_log2;
+    uint32_t s_phase = 0, o_phase = 0;
+    unsigned long long n_rescale = 0, n_rowtiles = 0;
+    for (int k = 0;; ++k) {
+      const int idx = sch.item(k);
+      if (idx < 0) break;
+      int b, t, h, seq_start, L;
+      sch.decode(idx, b, t, h, seq_start, L);
+      const int nkv = num_kv_tiles<CAUSAL>(t, s, L);
+      if (nkv == 0) continue;
+      const int row0 = t * 2 * kBM + s * kBM;
+      const int q_row = row0 + r;
+      float m_ref = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nkv; ++j) {
+        ok = mbar_wait(bar(Lay::B_SFULL + s), s_phase, wc, timeout_code(kSiteSFull));
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        s_phase ^= 1u;
+        tc_fence_after();
+        uint32_t sv[128];
+        tmem_ld_x128(t_s, sv);
+        const int kb = j * kBN;
+        if ((CAUSAL && kb + kBN - 1 > row0) || kb + kBN > L) {
+          int lim = L - kb;  // keys [kb, kb+lim) are visible to this row
+          if (CAUSAL && q_row - kb + 1 < lim) lim = q_row - kb + 1;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) sv[c] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+        const float m_tile = mx * sl;
+        bool need = false;
+        float alpha = 1.f;
+        if (j == 0) {
+          m_ref = m_tile;
+        } else {
+          ++n_rowtiles;
+          if (m_tile - m_ref > p.tau) {
+            need = true;
+            alpha = fast_exp2(m_ref - m_tile);
+            m_ref = m_tile;
+            l *= alpha;
+            ++n_rescale;
+          }
+        }
+        const float nm = -m_ref;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float a = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sl, nm));
+          const float e = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sl, nm));
+          l += a + e;
+          pk[c] = pack_bf16x2(a, e);
+        }
+        tmem_st_x64(t_s, pk);
+        // O_s is stable here: the commit that signalled S(s, j) also covers PV(s, j-1).
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld_x32(t_o + 32 * c, ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st_x32(t_o + 32 * c, ov);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_PFULL + s));
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      ok = mbar_wait(bar(Lay::B_OFULL + s), o_phase, wc, timeout_code(kSiteOFull));
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      o_phase ^= 1u;
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const bool store = q_row < L;
+      __nv_bfloat16* dst =
+          p.o + (static_cast<int64_t>(seq_start + q_row) * p.H + h) * static_cast<int64_t>(D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld_x32(t_o + 32 * c, ov);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
+        if (store) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (store) {
+        const float lse = (m_ref + __log2f(l)) * kLn2;
+        int64_t li;
+        if (p.cu_seqlens == nullptr)
+          li = (static_cast<int64_t>(b) * p.H + h) * p.N + q_row;
+        else
+          li = static_cast<int64_t>(h) * p.total + seq_start + q_row;
+        p.lse[li] = lse;
+      }
+    }
+    if (p.stats) {
+      atomicAdd(p.stats, n_rescale);
+      atomicAdd(p.stats + 1, n_rowtiles);
+    }
+  } else if (warp == 8) {
+    // ----------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      const uint64_t pol_kv = l2_policy_evict_last();
+      const uint64_t pol_q = l2_policy_evict_first();
+      uint32_t n_ld = 0, qe_phase = 0;
+      int n_items = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = sch.item(k);
+        if (idx < 0) break;
+        int b, t, h, seq_start, L;
+        sch.decode(idx, b, t, h, seq_start, L);
+        const int nkv0 = num_kv_tiles<CAUSAL>(t, 0, L), nkv1 = num_kv_tiles<CAUSAL>(t, 1, L);
+        const int nkv = nkv0 > nkv1 ? nkv0 : nkv1;
+        if (k > 0) {
+          if (!mbar_wait(bar(Lay::B_QEMPTY), qe_phase, wc, timeout_code(kSiteQEmpty))) break;
+          qe_phase ^= 1u;
+        }
+        mbar_arrive_expect_tx(bar(Lay::B_QFULL), 2 * Lay::TILE);
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sb + Lay::Q_OFF + s * Lay::TILE + c * Lay::CHUNK, &tm_q, bar(Lay::B_QFULL),
+                        c * 64, h, seq_start + t * 2 * kBM + s * kBM, pol_q);
+        ++n_items;
+        for (int j = 0; j < nkv && ok; ++j) {
+#pragma unroll
+          for (int which = 0; which < 2; ++which) {
+            const uint32_t slot = n_ld % NS;
+            if (n_ld >= static_cast<uint32_t>(NS)) {
+              if (!mbar_wait(bar(Lay::B_KVEMPTY + slot), ((n_ld / NS) - 1) & 1u, wc,
+                             timeout_code(kSiteKvEmpty))) {
+                ok = false;
+                break;
+              }
+            }
+            mbar_arrive_expect_tx(bar(Lay::B_KVFULL + slot), Lay::TILE);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(sb + Lay::KV_OFF + slot * Lay::TILE + c * Lay::CHUNK,
+                          which ? &tm_v : &tm_k, bar(Lay::B_KVFULL + slot), c * 64, h,
+                          seq_start + j * kBN, pol_kv);
+            ++n_ld;
+          }
+        }
+      }
+      // Drain: every issued copy must have landed before the CTA may exit.
+      const uint32_t first = n_ld > static_cast<uint32_t>(NS) ? n_ld - NS : 0u;
+      for (uint32_t n = first; n < n_ld; ++n)
+        drain_wait(bar(Lay::B_KVFULL + n % NS), (n / NS) & 1u, p.timeout_ns);
+      if (n_items > 0) drain_wait(bar(Lay::B_QFULL), (n_items - 1) & 1u, p.timeout_ns);
+    }
+  } else {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 0, 1);
+      const uint32_t tS0 = tmem + Lay::TM_S0, tS1 = tmem + Lay::TM_S1;
+      const uint32_t tO0 = tmem + Lay::TM_O0, tO1 = tmem + Lay::TM_O1;
+      uint32_t n_ld = 0, q_phase = 0, p_phase0 = 0, p_phase1 = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = sch.item(k);
+        if (idx < 0) break;
+        int b, t, h, seq_start, L;
+        sch.decode(idx, b, t, h, seq_start, L);
+        const int nk0 = num_kv_tiles<CAUSAL>(t, 0, L), nk1 = num_kv_tiles<CAUSAL>(t, 1, L);
+        const int nkv = nk0 > nk1 ? nk0 : nk1;
+        if (!mbar_wait(bar(Lay::B_QFULL), q_phase, wc, timeout_code(kSiteQFull))) break;
+        q_phase ^= 1u;
+        tc_fence_after();
+        for (int j = 0; j <= nkv; ++j) {
+          const uint32_t nK = n_ld + 2u * j;  // load sequence number of K_j
+          const uint32_t nV = nK - 1u;        // ... and of V_{j-1}
+          const uint32_t slotK = nK % NS, slotV = nV % NS;
+          if (j < nkv && !mbar_wait(bar(Lay::B_KVFULL + slotK), (nK / NS) & 1u, wc,
+                                    timeout_code(kSiteKvFull))) { ok = false; break; }
+          if (j > 0 && !mbar_wait(bar(Lay::B_KVFULL + slotV), (nV / NS) & 1u, wc,
+                                  timeout_code(kSiteKvFull))) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int s = 0; s < 2; ++s) {
+            const uint32_t tS = s ? tS1 : tS0, tO = s ? tO1 : tO0;
+            const int nks = s ? nk1 : nk0;
+            if (ok && j > 0 && j - 1 < nks) {
+              uint32_t& ph = s ? p_phase1 : p_phase0;
+              if (!mbar_wait(bar(Lay::B_PFULL + s), ph, wc, timeout_code(kSitePFull))) {
+                ok = false;
+              } else {
+                ph ^= 1u;
+                tc_fence_after();
+                const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::TILE;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                  mma_ts(tO, tS + kk * 8, sdesc_sw128(vbase + kk * 2048, Lay::CHUNK, 1024), idesc_o,
+                         (j > 1 || kk > 0) ? 1u : 0u);
+                if (j == nks) tc_commit(bar(Lay::B_OFULL + s));
+              }
+            }
+            if (ok && j < nks) {
+              const uint32_t qbase = sb + Lay::Q_OFF + s * Lay::TILE;
+              const uint32_t kbase = sb + Lay::KV_OFF + slotK * Lay::TILE;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+                mma_ss(tS, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
+                       idesc_s, kk > 0 ? 1u : 0u);
+              }
+              tc_commit(bar(Lay::B_SFULL + s));
+            }
+          }
+          if (!ok) break;
+          if (j < nkv) tc_commit(bar(Lay::B_KVEMPTY + slotK));
+          if (j > 0) tc_commit(bar(Lay::B_KVEMPTY + slotV));
+          if (j == nkv - 1) tc_commit(bar(Lay::B_QEMPTY));
+        }
+        n_ld += 2u * nkv;
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is freed.
+      tc_commit(bar(Lay::B_DRAIN));
+      if (!drain_wait(bar(Lay::B_DRAIN), 0u, p.timeout_ns) && p.err)
+        atomicCAS(p.err, 0, timeout_code(kSiteDrain));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+template <int D>
+constexpr int smem_bytes_fixed() { return 1024 + Layout<D>::TABLE_OFF; }
+
+}  // namespace
+
+int fwd_smem_bytes(int D, int B, int T, int varlen) {
+  const int fixed = D == 128 ? smem_bytes_fixed<128>() : smem_bytes_fixed<64>();
+  return fixed + (varlen ? (B + 3 * T + 1) * 4 : 0);
+}
+
+template <int D, bool CAUSAL>
+static cudaError_t launch_t(const FwdLaunch& a, cudaStream_t st) {
+  auto kern = fwd_kernel<D, CAUSAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem);
+  if (e != cudaSuccess) return e;
+  kern<<<a.grid, kThreads, a.smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(const FwdLaunch& a, int D, int causal, cudaStream_t st) {
+  if (D == 128) return causal ? launch_t<128, true>(a, st) : launch_t<128, false>(a, st);
+  return causal ? launch_t<64, true>(a, st) : launch_t<64, false>(a, st);
+}
+
+}  // namespace attn

@@ -1,0 +1,35 @@
+// attn_fwd_sm100.h -- internal launch interface of the forward kernel (not part of
+// the public C ABI; see include/attn.h for that).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace attn {
+
+struct FwdParams {
+  __nv_bfloat16* o;      // [T, H, D] bf16 (dense T = B*N)
+  float* lse;            // dense [B, H, N]; varlen [H, total]
+  const int* cu_seqlens; // device int32[B+1] or null (dense)
+  int B, H, N;
+  int T;                 // ceil(N / 256): query tile-pairs of the longest sequence
+  int total;             // packed tokens (dense: B*N)
+  float scale_log2;      // scale * log2(e)
+  float tau;             // conditional-rescale threshold, log2 units
+  int* err;              // device error word
+  unsigned long long* stats;  // optional [rescaled rows, row-tiles]
+  uint64_t timeout_ns;   // limit of every internal wait
+};
+
+struct FwdLaunch {
+  CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps {D, H, total}, box {64, 1, 128}, 128B swizzle
+  FwdParams p;
+  int grid;
+  int smem;
+};
+
+int fwd_smem_bytes(int D, int B, int T, int varlen);
+cudaError_t launch_fwd(const FwdLaunch& a, int D, int causal, cudaStream_t st);
+
+}  // namespace attn

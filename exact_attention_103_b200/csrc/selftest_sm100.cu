@@ -1,0 +1,132 @@
+// selftest_sm100.cu -- one-tile check of the forward kernel's tensor-core building
+// blocks (see include/attn_selftest.h).  Uses exactly the descriptors, tensor-map
+// format and TMEM moves of attn_fwd_sm100.cu, in a plain sequential order.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/attn_selftest.h"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+namespace {
+
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+    selftest_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+                    const __grid_constant__ CUtensorMap tv, float* s_out, float* o_out, int* err) {
+  constexpr int TILE = 128 * D * 2, CHUNK = 128 * 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t bar_tma = sb + 3 * TILE, bar_mma = bar_tma + 8;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + 3 * TILE + 16);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(bar_tma, 1);
+    mbar_init(bar_mma, 1);
+    misc[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(sb + 3 * TILE + 16, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  WaitCtl wc;
+  wc.abort = reinterpret_cast<volatile uint32_t*>(misc + 1);
+  wc.err = err;
+  wc.limit_ns = 1000000000ull;
+  const uint64_t pol = l2_policy_evict_first();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar_tma, 3 * TILE);
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sb + 0 * TILE + c * CHUNK, &ta, bar_tma, c * 64, 0, 0, pol);
+      tma_load_3d(sb + 1 * TILE + c * CHUNK, &tb, bar_tma, c * 64, 0, 0, pol);
+      tma_load_3d(sb + 2 * TILE + c * CHUNK, &tv, bar_tma, c * 64, 0, 0, pol);
+    }
+  }
+  bool ok = __all_sync(0xffffffffu, mbar_wait(bar_tma, 0, wc, 4 | (1 << 8)));
+  const uint32_t tS = tmem, tO = tmem + 256;
+  if (ok && threadIdx.x == 0) {
+    tc_fence_after();
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+      mma_ss(tS, sdesc_sw128(sb + off, 16, 1024), sdesc_sw128(sb + TILE + off, 16, 1024),
+             idesc_bf16_f32(128, 128, 0, 0), kk > 0 ? 1u : 0u);
+    }
+    tc_commit(bar_mma);
+  }
+  if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_mma, 0, wc, 4 | (2 << 8)));
+  const int r = warp * 32 + lane;
+  const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+  if (ok) {
+    tc_fence_after();
+    uint32_t sv[128];
+    tmem_ld_x128(tS + lane_bits, sv);
+    for (int c = 0; c < 128; ++c) s_out[r * 128 + c] = __uint_as_float(sv[c]);
+    uint32_t pk[64];
+    for (int c = 0; c < 64; ++c) pk[c] = pack_bf16x2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1]));
+    tmem_st_x64(tS + lane_bits, pk);
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (ok && threadIdx.x == 0) {
+    for (int kk = 0; kk < 128 / 16; ++kk)
+      mma_ts(tO, tS + kk * 8, sdesc_sw128(sb + 2 * TILE + kk * 2048, CHUNK, 1024),
+             idesc_bf16_f32(128, D, 0, 1), kk > 0 ? 1u : 0u);
+    tc_commit(bar_mma);
+  }
+  if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_mma, 1, wc, 4 | (3 << 8)));
+  if (ok) {
+    tc_fence_after();
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t ov[32];
+      tmem_ld_x32(tO + lane_bits + 32 * c, ov);
+      for (int i = 0; i < 32; ++i) o_out[r * D + 32 * c + i] = __uint_as_float(ov[i]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+}  // namespace attn
+
+// Shared with attn_api.cu (defined there).
+namespace attn_internal {
+attn_status_t prepare_selftest(int** err, bool (**mk)(CUtensorMap*, const void*, int64_t, int, int));
+}
+
+extern "C" attn_status_t attn_selftest_umma(const void* a, const void* b, const void* v,
+                                            float* s_out, float* o_out, int d,
+                                            attn_stream_t stream) {
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!a || !b || !v || !s_out || !o_out) return ATTN_ERR_INVALID_ARG;
+  int* err = nullptr;
+  bool (*mk)(CUtensorMap*, const void*, int64_t, int, int) = nullptr;
+  attn_status_t st = attn_internal::prepare_selftest(&err, &mk);
+  if (st != ATTN_OK) return st;
+  alignas(64) CUtensorMap ta, tb, tv;
+  if (!mk(&ta, a, 128, 1, d) || !mk(&tb, b, 128, 1, d) || !mk(&tv, v, 128, 1, d))
+    return ATTN_ERR_INVALID_ARG;
+  const int smem = 1024 + 3 * 128 * d * 2 + 64;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (d == 128) {
+    e = cudaFuncSetAttribute(attn::selftest_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) attn::selftest_kernel<128><<<1, 128, smem, cs>>>(ta, tb, tv, s_out, o_out, err);
+  } else {
+    e = cudaFuncSetAttribute(attn::selftest_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) attn::selftest_kernel<64><<<1, 128, smem, cs>>>(ta, tb, tv, s_out, o_out, err);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}

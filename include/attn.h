@@ -1,0 +1,135 @@
+/*
+ * attn.h -- C ABI of libattn: exact scaled-dot-product attention on NVIDIA B200
+ * (sm_100a), computed as one fused tiled kernel with online softmax so that the
+ * score matrix S and the probability matrix P never reach device memory.
+ *
+ * The operation (the pages' definition; "FlashAttention 1-4 详解", section 原算法,
+ * and "FlashAttention V4 deep-dive" (pnsm.cn), section 1.1):
+ *
+ *     O = softmax(scale * Q K^T) V,   LSE_i = ln sum_j exp(scale * <q_i, k_j>)
+ *
+ * row by row for every (sequence, head).  With `causal`, query i sees only keys
+ * j <= i ("FlashAttention 1-4 详解", 其他优化 / FlashAttention 2 的工程优化: causal
+ * lower triangle); indices are local to each sequence.
+ *
+ * Conventions shared by every entry point:
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller; the library
+ *    never frees or retains it.  Calls are asynchronous on `stream`; argument
+ *    errors are returned before anything is launched.
+ *  - Q, K, V, O are bf16, contiguous, head dimension innermost:
+ *      dense:  [B, N, H, d]   (row stride H*d elements)
+ *      varlen: [T, H, d]      packed, T = cu_seqlens[B]
+ *    Their base addresses must be 16-byte aligned.
+ *  - LSE is fp32, natural log, scale included:
+ *      dense:  [B, H, N]      varlen: [H, T]
+ *  - cu_seqlens (varlen only): DEVICE int32[B+1], non-decreasing prefix sums of the
+ *    sequence lengths with cu_seqlens[0] = 0; N is then the maximum length.  Q and
+ *    K/V of a sequence have the same length.  Pass NULL for a dense batch.
+ *    attn_fwd reads cu_seqlens[B] back to the host (a 4-byte copy that
+ *    synchronises `stream`); attn_fwd_ex with opts->total_tokens avoids that.
+ *    Inconsistent cu_seqlens (cu[0] != 0, a negative length, cu[B] != the token
+ *    count) make the kernel write nothing and record ATTN_ERR_INVALID_ARG in the
+ *    device error word.
+ *  - Supported: d in {64, 128}; scale finite and > 0.  Varlen: B <= 1024 and
+ *    N <= 131072.  B == 0 or N == 0 is a no-op.
+ *  - The library allocates, lazily and once per device, a small device error word.
+ *    A kernel whose internal waits exceed their time limit stops, records
+ *    ATTN_ERR_TIMEOUT there, and leaves its outputs undefined;
+ *    attn_get_device_status() reports and clears it.
+ */
+#ifndef LIBATTN_ATTN_H
+#define LIBATTN_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA stream handle type (identical to cudaStream_t / CUstream). */
+typedef struct CUstream_st* attn_stream_t;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or scale     */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid but not supported (d, limits, no sm_100) */
+  ATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed              */
+  ATTN_ERR_TIMEOUT = 4,     /* a kernel's bounded wait expired (device status) */
+  ATTN_ERR_WORKSPACE = 5    /* workspace pointer/size too small               */
+} attn_status_t;
+
+/*
+ * Forward pass.  Writes O (bf16, layout of Q) and LSE (fp32, layout above).
+ * Online softmax: "FlashAttention 1-4 详解", FlashAttention 1 / Online Softmax
+ * 数学推导, with deferred normalisation (FlashAttention 2 / 减少非矩阵乘运算占比)
+ * and the conditional rescale of "FlashAttention V4 deep-dive", section 3.2.
+ * The result does not depend on how the work is scheduled: each output row is
+ * produced by one CTA with a fixed key order, so repeated calls are bitwise equal.
+ */
+ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int H, int N, int d, int causal, float scale,
+                       const int32_t* cu_seqlens, attn_stream_t stream);
+
+/* Tuning / test knobs for attn_fwd_ex.  Zero-initialise, then set fields.
+ *  rescale_threshold: conditional-rescale threshold tau in log2 units; the
+ *      running maximum is replaced (and O, l rescaled) only when a new tile's row
+ *      maximum exceeds it by more than tau.  < 0 selects the default (8.0).
+ *  stats: optional DEVICE pointer to two uint64 counters the kernel ADDS to:
+ *      [0] rows rescaled, [1] row-tiles processed after each row's first tile.
+ *  timeout_ns: limit of every internal wait; 0 selects the default (2 s).
+ *  total_tokens: varlen only; if > 0 it must equal cu_seqlens[B] (checked on the
+ *      device).  When 0, attn_fwd_ex (like attn_fwd) reads cu_seqlens[B] back
+ *      to the host with a 4-byte copy and a stream synchronisation, because the
+ *      TMA views of Q/K/V must not extend past the packed tensors. */
+typedef struct {
+  float rescale_threshold;
+  unsigned long long* stats;
+  uint64_t timeout_ns;
+  int64_t total_tokens;
+} attn_fwd_opts_t;
+
+/* attn_fwd with options (opts may be NULL = defaults). */
+ATTN_API attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int N, int d, int causal, float scale,
+                          const int32_t* cu_seqlens, const attn_fwd_opts_t* opts,
+                          attn_stream_t stream);
+
+/*
+ * Backward pass (dQ, dK, dV) from Q, K, V, O, LSE and dO, recomputing P from LSE
+ * ("FlashAttention 1-4 详解", 总结 table: 反向传播重计算; "FlashAttention V4
+ * deep-dive", section 3.3).  Same layouts as the forward; dq/dk/dv are bf16.
+ * `deterministic` != 0 makes the result bitwise reproducible run to run.
+ * `workspace` is a caller-owned DEVICE buffer of at least
+ * attn_bwd_workspace_size(...) bytes, 256-byte aligned (may be NULL when that
+ * size is 0).  Not yet provided by this build: returns ATTN_ERR_UNSUPPORTED.
+ */
+ATTN_API attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                       int B, int H, int N, int d, int causal, float scale,
+                       const int32_t* cu_seqlens, int deterministic, void* workspace,
+                       size_t workspace_bytes, attn_stream_t stream);
+
+/* Workspace bytes attn_bwd needs (total_tokens = B*N dense, cu_seqlens[B] varlen). */
+ATTN_API size_t attn_bwd_workspace_size(int B, int H, int N, int d, int total_tokens, int deterministic);
+
+/* Synchronises `stream`, then returns and clears the device error word of the
+ * current device (ATTN_OK if no kernel recorded an error). */
+ATTN_API attn_status_t attn_get_device_status(attn_stream_t stream);
+
+/* Static string for a status code. */
+ATTN_API const char* attn_status_string(attn_status_t s);
+
+/* Message describing the last non-OK status returned on the calling thread. */
+ATTN_API const char* attn_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LIBATTN_ATTN_H */

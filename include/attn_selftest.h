@@ -1,0 +1,23 @@
+/*
+ * attn_selftest.h -- diagnostic entry point of libattn (not part of the attention
+ * API).  It runs the tensor-core building blocks of the forward kernel on one
+ * 128-row tile so a test can check each against a plain matrix product:
+ *   TMA load of three bf16 [128, d] row-major tiles A, B, V (128-byte swizzle),
+ *   S = A B^T with tcgen05.mma from shared memory (K-major A and B), fp32 in TMEM;
+ *   P = bf16(S) written back into TMEM;
+ *   O = P V with tcgen05.mma, A = P from TMEM, B = V from shared memory (MN-major).
+ * a, b, v: DEVICE bf16 [128, d] (16-byte aligned); s_out: DEVICE fp32 [128, 128];
+ * o_out: DEVICE fp32 [128, d]; d in {64, 128}.  Asynchronous on `stream`.
+ */
+#ifndef LIBATTN_ATTN_SELFTEST_H
+#define LIBATTN_ATTN_SELFTEST_H
+#include "attn.h"
+#ifdef __cplusplus
+extern "C" {
+#endif
+ATTN_API attn_status_t attn_selftest_umma(const void* a, const void* b, const void* v, float* s_out,
+                                 float* o_out, int d, attn_stream_t stream);
+#ifdef __cplusplus
+}
+#endif
+#endif

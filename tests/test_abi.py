@@ -1,0 +1,97 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the public
+headers declare, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_103_b200 as ea
+from exact_attention_103_b200 import build as ea_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ea_build.build()
+    return ea.load_library()
+
+
+def _declared_symbols():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names |= set(re.findall(r"ATTN_API\s+[^;(]*?\b(attn_\w+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared_symbols()
+    assert {"attn_fwd", "attn_fwd_ex", "attn_bwd", "attn_get_device_status"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(ea.EXPORTED_SYMBOLS)
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(["ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
+                                 "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "ATTN_ERR_WORKSPACE"]):
+        assert ea.status_string(code) == name
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation returns first
+
+
+def _fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, H=1, N=128, d=128, causal=0,
+         scale=0.125, cu=None):
+    return lib.attn_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, cu, None)
+
+
+def test_unsupported_head_dim(lib):
+    assert _fwd(lib, d=96) == ea.ATTN_ERR_UNSUPPORTED
+    assert "head dim" in ea.last_error()
+
+
+@pytest.mark.parametrize("scale", [0.0, -1.0, float("inf"), float("nan")])
+def test_bad_scale(lib, scale):
+    assert _fwd(lib, scale=scale) == ea.ATTN_ERR_INVALID_ARG
+
+
+def test_null_and_misaligned_pointers(lib):
+    assert _fwd(lib, q=None) == ea.ATTN_ERR_INVALID_ARG
+    assert _fwd(lib, o=None) == ea.ATTN_ERR_INVALID_ARG
+    assert _fwd(lib, k=FAKE + 8) == ea.ATTN_ERR_INVALID_ARG
+    assert _fwd(lib, lse=FAKE + 2) == ea.ATTN_ERR_INVALID_ARG
+
+
+def test_negative_sizes(lib):
+    assert _fwd(lib, B=-1) == ea.ATTN_ERR_INVALID_ARG
+    assert _fwd(lib, H=0) == ea.ATTN_ERR_INVALID_ARG
+    assert _fwd(lib, N=-5) == ea.ATTN_ERR_INVALID_ARG
+
+
+def test_empty_problem_is_a_noop(lib):
+    # Nothing is launched, so this succeeds without a device.
+    assert _fwd(lib, B=0) == ea.ATTN_OK
+    assert _fwd(lib, N=0, q=None) == ea.ATTN_OK
+
+
+def test_varlen_limits(lib):
+    assert _fwd(lib, B=1025, cu=FAKE) == ea.ATTN_ERR_UNSUPPORTED
+    assert _fwd(lib, B=2, N=131073, cu=FAKE) == ea.ATTN_ERR_UNSUPPORTED
+    assert _fwd(lib, B=2, cu=FAKE + 2) == ea.ATTN_ERR_INVALID_ARG
+
+
+def test_bad_options(lib):
+    opts = ea.FwdOpts(float("inf"), None, 0, 0)
+    st = lib.attn_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0, 0.1, None,
+                         ctypes.byref(opts), None)
+    assert st == ea.ATTN_ERR_INVALID_ARG
+
+
+def test_backward_not_provided_yet(lib):
+    st = lib.attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0,
+                      0.1, None, 0, None, 0, None)
+    assert st == ea.ATTN_ERR_UNSUPPORTED

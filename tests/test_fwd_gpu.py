@@ -1,0 +1,228 @@
+"""GPU parity of the forward kernel against the fp64 oracle, through the C ABI.
+
+Small and ragged shapes are compared element by element over the whole output;
+the full benchmark workloads are compared on sampled rows (the oracle computes
+those one by one) plus whole-output properties.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import attn_inputs as ai
+import oracle
+from attn_check import compare_lse, compare_o, to_np
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _lib():
+    import exact_attention_103_b200 as ea
+    return ea
+
+
+def _dense_ref(q, k, v, causal, scale):
+    B, N, H, d = q.shape
+    o, lse, _ = oracle.fwd(q.reshape(B * N, H, d), k.reshape(B * N, H, d), v.reshape(B * N, H, d),
+                           oracle.dense_cu(B, N), causal, scale)
+    return o.reshape(B, N, H, d), oracle.lse_to_dense(lse, B, N)
+
+
+def _run_dense(q, k, v, causal, scale, **kw):
+    ea = _lib()
+    o, lse = ea.fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, scale=scale, **kw)
+    ea.get_device_status()
+    return o.cpu(), lse.cpu()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_selftest_umma_tile(d):
+    """The kernel's tensor-core building blocks on one tile: S = A B^T (K-major
+    smem operands), then bf16(S) V with P from TMEM and V MN-major."""
+    ea = _lib()
+    g = torch.Generator().manual_seed(d)
+    a, b, v = (torch.randn(128, d, generator=g).to(torch.bfloat16) for _ in range(3))
+    s, o = ea.selftest_umma(a.to(DEV), b.to(DEV), v.to(DEV))
+    torch.cuda.synchronize()
+    s_ref = a.double() @ b.double().T
+    np.testing.assert_allclose(s.cpu().double().numpy(), s_ref.numpy(), rtol=0, atol=1e-3)
+    p = s.cpu().to(torch.bfloat16).double()
+    o_ref = p @ v.double()
+    np.testing.assert_allclose(o.cpu().double().numpy(), o_ref.numpy(), rtol=1e-5, atol=1e-2)
+
+
+SMALL = [
+    # B, N, H, d, causal, q_mult
+    (1, 256, 1, 64, False, 1.0),     # the tiny latency workload
+    (1, 256, 1, 64, True, 1.0),
+    (1, 1, 1, 128, False, 1.0),
+    (1, 1, 1, 64, True, 1.0),
+    (2, 300, 3, 128, False, 1.0),    # ragged last tile, two batches
+    (2, 300, 3, 128, True, 1.0),
+    (1, 129, 2, 64, True, 1.0),
+    (3, 513, 2, 128, True, 1.0),     # several tile pairs plus a 1-row tail
+    (1, 1000, 1, 64, False, 1.0),
+    (2, 640, 2, 128, False, 4.0),    # Q x4: the running maximum moves often
+    (1, 768, 2, 128, True, 4.0),
+]
+
+
+@pytest.mark.parametrize("B,N,H,d,causal,qm", SMALL)
+def test_fwd_parity_dense(B, N, H, d, causal, qm):
+    q, k, v = ai.make_custom(B, N, H, d, seed=B * 1000 + N + d)
+    if qm != 1.0:
+        q = (q.float() * qm).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = _run_dense(q, k, v, causal, scale)
+    o_ref, lse_ref = _dense_ref(q, k, v, causal, scale)
+    compare_o(o, o_ref, f"dense B{B} N{N} H{H} d{d} causal={causal} x{qm}")
+    compare_lse(lse, lse_ref)
+
+
+VARLEN = [
+    ([5, 0, 300, 129], 128, True),
+    ([5, 0, 300, 129], 128, False),
+    ([1, 127, 128, 129, 256, 257, 700], 64, True),
+    ([1, 127, 128, 129, 256, 257, 700], 128, False),
+    ([1024, 3, 511], 128, True),
+]
+
+
+@pytest.mark.parametrize("lengths,d,causal", VARLEN)
+def test_fwd_parity_varlen(lengths, d, causal):
+    H = 2
+    q, k, v = ai.make_custom(0, 0, H, d, seed=sum(lengths) + d, lengths=lengths)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    scale = 1.0 / math.sqrt(d)
+    ea = _lib()
+    o, lse = ea.fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, scale=scale,
+                    cu_seqlens=torch.from_numpy(cu).to(DEV), max_seqlen=max(lengths))
+    ea.get_device_status()
+    o_ref, lse_ref, _ = oracle.fwd(q, k, v, cu, causal, scale)
+    compare_o(o.cpu(), o_ref, f"varlen {lengths} d{d} causal={causal}")
+    compare_lse(lse.cpu(), lse_ref)
+
+
+def test_plain_c_entry_point_varlen_reads_total():
+    """attn_fwd (no options) reads cu_seqlens[B] itself; results equal attn_fwd_ex's."""
+    ea = _lib()
+    lengths = [200, 77, 390]
+    H, d = 2, 128
+    q, k, v = (t.to(DEV) for t in ai.make_custom(0, 0, H, d, seed=5, lengths=lengths))
+    cu = torch.tensor([0, 200, 277, 667], dtype=torch.int32, device=DEV)
+    o1, l1 = ea.fwd(q, k, v, causal=True, cu_seqlens=cu, max_seqlen=390)
+    o2, l2 = torch.empty_like(q), torch.empty_like(l1)
+    ea.fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), o2.data_ptr(), l2.data_ptr(), 3, H, 390,
+               d, True, 1 / math.sqrt(d), cu.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    ea.get_device_status()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fwd_deterministic_bitwise():
+    ea = _lib()
+    q, k, v = (t.to(DEV) for t in ai.make_custom(2, 1100, 4, 128, seed=21))
+    o1, l1 = ea.fwd(q, k, v, causal=True)
+    o2, l2 = ea.fwd(q, k, v, causal=True)
+    ea.get_device_status()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fwd_writes_nothing_outside_outputs():
+    """Guard regions around O and LSE keep their canary pattern."""
+    ea = _lib()
+    B, N, H, d = 1, 333, 3, 128
+    q, k, v = (t.to(DEV) for t in ai.make_custom(B, N, H, d, seed=22))
+    n_o, n_l, pad = B * N * H * d, B * H * N, 4096
+    o_buf = torch.full((n_o + 2 * pad,), 7.0, dtype=torch.bfloat16, device=DEV)
+    l_buf = torch.full((n_l + 2 * pad,), -3.0, dtype=torch.float32, device=DEV)
+    o = o_buf[pad:pad + n_o].view(B, N, H, d)
+    lse = l_buf[pad:pad + n_l].view(B, H, N)
+    ea.fwd(q, k, v, causal=False, out=o, lse=lse)
+    ea.get_device_status()
+    for buf, val in ((o_buf, 7.0), (l_buf, -3.0)):
+        assert torch.all(buf[:pad] == val) and torch.all(buf[-pad:] == val)
+    o_ref, l_ref = _dense_ref(q.cpu(), k.cpu(), v.cpu(), False, 1 / math.sqrt(d))
+    compare_o(o.cpu(), o_ref)
+    compare_lse(lse.cpu(), l_ref)
+
+
+def test_rescale_threshold_readings_agree():
+    """tau = 0 (rescale whenever the maximum grows), 8 (default) and 1e9 (never
+    after the first tile) are all exact readings: same result within tolerance."""
+    ea = _lib()
+    B, N, H, d = 1, 1024, 2, 128
+    q, k, v = ai.make_custom(B, N, H, d, seed=23)
+    q = (q.float() * 4).to(torch.bfloat16)
+    o_ref, l_ref = _dense_ref(q, k, v, False, 1 / math.sqrt(d))
+    outs = {}
+    for tau in (0.0, 8.0, 1e9):
+        stats = torch.zeros(2, dtype=torch.int64, device=DEV)
+        o, lse = ea.fwd(q.to(DEV), k.to(DEV), v.to(DEV), rescale_threshold=tau, stats=stats)
+        ea.get_device_status()
+        compare_o(o.cpu(), o_ref, f"tau={tau}")
+        compare_lse(lse.cpu(), l_ref)
+        outs[tau] = stats.cpu().tolist()
+    # row-tiles after the first tile: every row of every 128-row sub-tile, 7 tiles each
+    expected = B * H * (N // 128) * 128 * (N // 128 - 1)
+    for tau, (resc, tiles) in outs.items():
+        assert tiles == expected, (tau, tiles, expected)
+    assert outs[0.0][0] >= outs[8.0][0] >= outs[1e9][0] == 0
+
+
+def test_invalid_cu_seqlens_recorded_on_device():
+    """cu_seqlens that disagree with the packed token count make the kernel write
+    nothing and record ATTN_ERR_INVALID_ARG in the device error word."""
+    ea = _lib()
+    q, k, v = (t.to(DEV) for t in ai.make_custom(0, 0, 1, 64, seed=24, lengths=[100, 100]))
+    cu = torch.tensor([0, 100, 150], dtype=torch.int32, device=DEV)  # total 150 != 200
+    ea.fwd(q, k, v, cu_seqlens=cu, max_seqlen=100)
+    with pytest.raises(ea.AttnError) as e:
+        ea.get_device_status()
+    assert e.value.status == ea.ATTN_ERR_INVALID_ARG
+    ea.get_device_status()  # cleared
+
+
+# ----------------------------------------------------- full-size workloads
+def _sample_rows(lengths, H, n, seed):
+    """Sampled (token, head) rows: each sequence's first/last rows, rows around
+    128-row tile boundaries, and random rows."""
+    rng = np.random.default_rng(seed)
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    rows, heads = [], []
+    for b, L in enumerate(lengths):
+        picks = {0, L - 1, min(127, L - 1), min(128, L - 1), min(255, L - 1), min(256, L - 1),
+                 (L - 1) // 2}
+        picks |= set(rng.integers(0, L, size=max(1, n // len(lengths))).tolist())
+        for i in sorted(picks):
+            rows.append(cu[b] + i)
+            heads.append(int(rng.integers(0, H)))
+    return np.array(rows), np.array(heads), cu
+
+
+@pytest.mark.parametrize("name", ["B1-H1-N256-d64", "B4-H16-N2048-d128",
+                                  "B4-H16-N2048-d128-qx4", "B2-H16-N8192-d128-causal",
+                                  "varlen16-H16-d128-causal"])
+def test_fwd_full_workload_sampled(name):
+    ea = _lib()
+    w = ai.ALL[name]
+    q, k, v = ai.make_qkv(w)
+    scale = 1.0 / math.sqrt(w.d)
+    cu_t = None
+    if w.varlen:
+        cu_t = torch.tensor(w.cu_seqlens(), dtype=torch.int32, device=DEV)
+    o, lse = ea.fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=w.causal, scale=scale,
+                    cu_seqlens=cu_t, max_seqlen=w.N if w.varlen else None)
+    ea.get_device_status()
+    o = o.cpu().reshape(-1, w.H, w.d)
+    lse = lse.cpu()
+    if not w.varlen:
+        lse = lse.permute(1, 0, 2).reshape(w.H, -1)  # [B,H,N] -> [H, B*N]
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    rows, heads, cu = _sample_rows(w.seq_lengths(), w.H, 192, seed=len(name))
+    qp, kp, vp = (t.reshape(-1, w.H, w.d) for t in (q, k, v))
+    o_ref, l_ref = oracle.fwd_rows(qp, kp, vp, cu, w.causal, scale, rows, heads)
+    compare_o(o[rows, heads], o_ref, name)
+    compare_lse(lse[heads, rows], l_ref, name)
