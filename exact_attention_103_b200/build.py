@@ -20,6 +20,8 @@ SOURCES = ["attn_api.cu", "attn_fwd_sm100.cu", "selftest_sm100.cu"]
 HEADERS = ["attn_fwd_sm100.h", "sm100_ptx.cuh"]
 PUBLIC_HEADERS = [os.path.join(ROOT, "include", h) for h in ("attn.h", "attn_selftest.h")]
 NVCC = os.environ.get("NVCC", "nvcc")
+# Extra nvcc flags (e.g. -DATTN_POLY_PAIRS_PER_8=4 to change the MUFU/FMA exp split).
+EXTRA = os.environ.get("ATTN_NVCC_EXTRA", "").split()
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-Xptxas", "-v",
          "-I", os.path.join(ROOT, "include")]
@@ -38,7 +40,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     def compile_one(src):
         obj = os.path.join(OBJ, os.path.basename(src).replace(".cu", ".o"))
-        cmd = [NVCC, *FLAGS, "-c", src, "-o", obj]
+        cmd = [NVCC, *FLAGS, *EXTRA, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")

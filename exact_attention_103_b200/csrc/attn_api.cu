@@ -127,7 +127,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   unsigned long long* stats = nullptr;
   if (opts) {
     if (opts->rescale_threshold >= 0.f) tau = opts->rescale_threshold;
-    if (!std::isfinite(tau)) return fail(ATTN_ERR_INVALID_ARG, "rescale_threshold must be finite");
+    if (!(tau <= 64.f)) return fail(ATTN_ERR_INVALID_ARG, "rescale_threshold must be <= 64");
     if (opts->timeout_ns) timeout = opts->timeout_ns;
     stats = opts->stats;
     if (stats && !aligned(stats, 8)) return fail(ATTN_ERR_INVALID_ARG, "stats misaligned");

@@ -6,11 +6,14 @@
 // two sub-tiles while the other one's softmax runs ("FlashAttention V4 deep-dive"
 // (pnsm.cn), section 3.1, two Q tiles in ping-pong).
 //
-// Warp roles (320 threads):
-//   warps 0-3  softmax + epilogue of sub-tile 0 (one thread per query row)
-//   warps 4-7  softmax + epilogue of sub-tile 1
-//   warp  8    TMA producer: Q pair, then K_j / V_j tiles into an smem ring
-//   warp  9    TMEM owner and tcgen05.mma issuer (one elected lane)
+// Warp roles (576 threads):
+//   warps 0-7   softmax + epilogue of sub-tile 0: warp w owns TMEM lanes
+//               32(w%4)..+31 (one query row per thread) and key columns
+//               64*((w/4)%2)..+63 of every tile, so two threads share each row
+//   warps 8-15  the same for sub-tile 1
+//   warp  16    TMA producer: Q pair, then K_j / V_j tiles into an smem ring
+//   warp  17    TMEM owner and tcgen05.mma issuer (whole warp; one elected lane
+//               issues each instruction)
 //
 // Per sub-tile s and key tile j ("FlashAttention 1-4 详解", FlashAttention 1 /
 // Online Softmax 数学推导; FlashAttention 2 / 减少非矩阵乘运算占比):
@@ -40,23 +43,49 @@
 #include <cuda_runtime.h>
 
 #include "attn_fwd_sm100.h"
+#include "exp2_poly.h"
 #include "sm100_ptx.cuh"
 
 namespace attn {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
 constexpr int kBM = 128;  // query rows per sub-tile
 constexpr int kBN = 128;  // keys per key tile
 constexpr float kLn2 = 0.693147180559945309f;
+
+// Of every 8 consecutive (even, odd) column pairs of a score row, this many are
+// exponentiated on the FMA pipe by the polynomial below; the rest use MUFU ex2.
+#ifndef ATTN_POLY_PAIRS_PER_8
+#define ATTN_POLY_PAIRS_PER_8 1
+#endif
+constexpr int kPolyPairsPer8 = ATTN_POLY_PAIRS_PER_8;
+static_assert(kPolyPairsPer8 >= 0 && kPolyPairsPer8 <= 8, "pairs per 8");
+
+// 2^y without MUFU: j = round(y) by the 1.5*2^23 trick, f = y - j in [-1/2, 1/2],
+// p(f) ~ 2^f (minimax, exp2_poly.h), then 2^j is added to the exponent field as an
+// integer.  y is clamped below at -125 so the result stays a normal float (the
+// exact value there is < 2^-125, far below a bf16 P~).  Valid for y <= 64 (the
+// conditional-rescale threshold keeps y <= tau <= 64).  Scalar FMA-pipe
+// instructions only: one max, three adds, three FMAs and an integer shift-add.
+__device__ __forceinline__ float exp2_poly(float y) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  y = fmaxf(y, -125.f);
+  const float t = y + kMagic;            // rounds y to an integer in t's low bits
+  const float f = y - (t - kMagic);
+  float p = fmaf(f, ATTN_EXP2_C3, ATTN_EXP2_C2);
+  p = fmaf(p, f, ATTN_EXP2_C1);
+  p = fmaf(p, f, ATTN_EXP2_C0);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
 
 // Error codes recorded in the device error word: 4 (= ATTN_ERR_TIMEOUT) in the
 // low byte, the waiting site above it.
 __host__ __device__ constexpr int timeout_code(int site) { return 4 | (site << 8); }
 enum WaitSite {
   kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteOFull,
-  kSiteDrain, kSiteBadLen
+  kSiteDrain, kSiteBadLen, kSiteXch
 };
 
 template <int D>
@@ -69,10 +98,11 @@ struct Layout {
   static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE;
   // barrier indices
   static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_OFULL = 6,
-                       B_DRAIN = 8, B_KVFULL = 9, B_KVEMPTY = 9 + NSTAGE;
-  static constexpr int NBARS = 9 + 2 * NSTAGE;
+                       B_DRAIN = 8, B_XCH = 9, B_KVFULL = 17, B_KVEMPTY = 17 + NSTAGE;
+  static constexpr int NBARS = 17 + 2 * NSTAGE;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-  static constexpr int TABLE_OFF = MISC_OFF + 64;
+  static constexpr int EXCH_OFF = MISC_OFF + 64;          // float [2][2][128][2]
+  static constexpr int TABLE_OFF = EXCH_OFF + 2 * 2 * 128 * 2 * 4;
   static constexpr int TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
 };
 
@@ -226,10 +256,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(Lay::B_QEMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Lay::B_SFULL + s), 1);
-      mbar_init(bar(Lay::B_PFULL + s), 128);
+      mbar_init(bar(Lay::B_PFULL + s), 8);
       mbar_init(bar(Lay::B_OFULL + s), 1);
     }
     mbar_init(bar(Lay::B_DRAIN), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar(Lay::B_XCH + i), 2);
     for (int i = 0; i < NS; ++i) {
       mbar_init(bar(Lay::B_KVFULL + i), 1);
       mbar_init(bar(Lay::B_KVEMPTY + i), 1);
@@ -237,11 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     misc[1] = 0u;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == 17) {
     tmem_alloc(sb + Lay::MISC_OFF, 512);
     tmem_relinquish();
   }
-  if (warp == 8) {
+  if (warp == 16) {
     int count;
     if (p.cu_seqlens == nullptr) {
       count = p.B * p.T * p.H;
@@ -272,13 +303,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   wc.err = p.err;
   wc.limit_ns = p.timeout_ns;
 
-  if (warp < 8) {
+  if (warp < 16) {
     // ------------------------------------------------------------ softmax
-    const int s = warp >> 2, wq = warp & 3;
+    // Sub-tile s, TMEM lane quarter q (rows 32q..32q+31), column half hf: the two
+    // warps of a (s, q) pair share the rows and split each row's 128 key columns,
+    // exchanging partial row maxima (and, at the end, partial row sums) through
+    // shared memory with a 64-thread named barrier.
+    const int s = warp >> 3, hf = (warp >> 2) & 1, wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t t_s = tmem + lane_bits + (s ? Lay::TM_S1 : Lay::TM_S0);
-    const uint32_t t_o = tmem + lane_bits + (s ? Lay::TM_O1 : Lay::TM_O0);
+    const uint32_t t_p = t_s + 32 * hf;        // this half's packed bf16 P columns
+    const uint32_t t_o = tmem + lane_bits + (s ? Lay::TM_O1 : Lay::TM_O0) + (D / 2) * hf;
+    // Pair exchange: write a value, arrive (one arrival per warp), wait for the
+    // partner's arrival, read its value.  Slots alternate with the exchange count,
+    // so a slot is rewritten only after the partner has passed the next exchange.
+    const uint32_t xbar = bar(Lay::B_XCH + s * 4 + wq);
+    float* xch = reinterpret_cast<float*>(smem + Lay::EXCH_OFF);
+    uint32_t n_x = 0;
+    auto exchange = [&](float mine, float& theirs) -> bool {
+      float* slot = xch + (((n_x & 1) * 2 + s) * 128 + r) * 2;
+      slot[hf] = mine;
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xbar);
+      bool okx = mbar_wait(xbar, n_x & 1, wc, timeout_code(kSiteXch));
+      okx = __all_sync(0xffffffffu, okx);
+      theirs = slot[hf ^ 1];
+      ++n_x;
+      return okx;
+    };
     const float sl = p.scale_log2;
     uint32_t s_phase = 0, o_phase = 0;
     unsigned long long n_rescale = 0, n_rowtiles = 0;
@@ -299,48 +353,75 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         s_phase ^= 1u;
         tc_fence_after();
-        uint32_t sv[128];
-        tmem_ld_x128(t_s, sv);
-        const int kb = j * kBN;
-        if ((CAUSAL && kb + kBN - 1 > row0) || kb + kBN > L) {
-          int lim = L - kb;  // keys [kb, kb+lim) are visible to this row
+        uint32_t sv[64];
+        tmem_ld_x64(t_s + 64 * hf, sv);
+        const int kb = j * kBN + 64 * hf;  // key index of this thread's first column
+        if ((CAUSAL && j * kBN + kBN - 1 > row0) || kb + 64 > L) {
+          int lim = L - kb;  // columns [0, lim) hold visible keys for this row
           if (CAUSAL && q_row - kb + 1 < lim) lim = q_row - kb + 1;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < 64; ++c)
             if (c >= lim) sv[c] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        // Partial row maximum over this half: four 3-input max chains and a tree.
+        float m4[4];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+        for (int i = 0; i < 4; ++i)
+          m4[i] = fmax3(__uint_as_float(sv[i]), __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 8]));
+#pragma unroll
+        for (int c = 12; c < 60; c += 8)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            m4[i] = fmax3(m4[i], __uint_as_float(sv[c + i]), __uint_as_float(sv[c + 4 + i]));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], __uint_as_float(sv[60 + i]));
+        const float mx_half = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+        float mx_other;
+        ok = exchange(mx_half, mx_other);
+        if (!ok) break;
+        const float mx = fmaxf(mx_half, mx_other);
         const float m_tile = mx * sl;
         bool need = false;
         float alpha = 1.f;
         if (j == 0) {
           m_ref = m_tile;
         } else {
-          ++n_rowtiles;
+          if (hf == 0) ++n_rowtiles;
           if (m_tile - m_ref > p.tau) {
             need = true;
             alpha = fast_exp2(m_ref - m_tile);
             m_ref = m_tile;
             l *= alpha;
-            ++n_rescale;
+            if (hf == 0) ++n_rescale;
           }
         }
+        // P~ = 2^(s*scale*log2e - m_ref): one FMA for the argument, MUFU ex2 or the
+        // FMA-pipe polynomial for the exponential, four partial row sums, then
+        // bf16 packing.
         const float nm = -m_ref;
-        uint32_t pk[64];
+        uint32_t pk[32];
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float a = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sl, nm));
-          const float e = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sl, nm));
-          l += a + e;
+        for (int c = 0; c < 32; ++c) {
+          float a = fmaf(__uint_as_float(sv[2 * c]), sl, nm);
+          float e = fmaf(__uint_as_float(sv[2 * c + 1]), sl, nm);
+          if ((c & 7) >= 8 - kPolyPairsPer8) {
+            a = exp2_poly(a);
+            e = exp2_poly(e);
+          } else {
+            a = fast_exp2(a);
+            e = fast_exp2(e);
+          }
+          ls[2 * (c & 1)] += a;
+          ls[2 * (c & 1) + 1] += e;
           pk[c] = pack_bf16x2(a, e);
         }
-        tmem_st_x64(t_s, pk);
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        tmem_st_x32(t_p, pk);
         // O_s is stable here: the commit that signalled S(s, j) also covers PV(s, j-1).
         if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < D / 64; ++c) {
             uint32_t ov[32];
             tmem_ld_x32(t_o + 32 * c, ov);
 #pragma unroll
@@ -349,22 +430,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tmem_st_wait();
+        // One arrival per warp: every lane's TMEM stores are complete (wait::st) and
+        // fenced before the warp converges; lane 0 then releases them to the MMA warp.
         tc_fence_before();
-        mbar_arrive(bar(Lay::B_PFULL + s));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(Lay::B_PFULL + s));
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
+      float l_other;
+      ok = exchange(l, l_other);
+      if (!ok) break;
       ok = mbar_wait(bar(Lay::B_OFULL + s), o_phase, wc, timeout_code(kSiteOFull));
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       o_phase ^= 1u;
       tc_fence_after();
+      l += l_other;
       const float inv = 1.f / l;
       const bool store = q_row < L;
-      __nv_bfloat16* dst =
-          p.o + (static_cast<int64_t>(seq_start + q_row) * p.H + h) * static_cast<int64_t>(D);
+      __nv_bfloat16* dst = p.o + (static_cast<int64_t>(seq_start + q_row) * p.H + h) *
+                                     static_cast<int64_t>(D) + (D / 2) * hf;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t ov[32];
         tmem_ld_x32(t_o + 32 * c, ov);
         uint32_t w[16];
@@ -377,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (store) {
+      if (store && hf == 0) {
         const float lse = (m_ref + __log2f(l)) * kLn2;
         int64_t li;
         if (p.cu_seqlens == nullptr)
@@ -391,28 +479,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       atomicAdd(p.stats, n_rescale);
       atomicAdd(p.stats + 1, n_rowtiles);
     }
-  } else if (warp == 8) {
+  } else if (warp == 16) {
     // ----------------------------------------------------------- producer
-    if (lane == 0) {
+    // Whole warp walks the loop and waits; one elected lane issues the copies.
+    if (elect_one()) {
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
-      const uint64_t pol_kv = l2_policy_evict_last();
-      const uint64_t pol_q = l2_policy_evict_first();
-      uint32_t n_ld = 0, qe_phase = 0;
-      int n_items = 0;
-      bool ok = true;
-      for (int k = 0; ok; ++k) {
-        const int idx = sch.item(k);
-        if (idx < 0) break;
-        int b, t, h, seq_start, L;
-        sch.decode(idx, b, t, h, seq_start, L);
-        const int nkv0 = num_kv_tiles<CAUSAL>(t, 0, L), nkv1 = num_kv_tiles<CAUSAL>(t, 1, L);
-        const int nkv = nkv0 > nkv1 ? nkv0 : nkv1;
-        if (k > 0) {
-          if (!mbar_wait(bar(Lay::B_QEMPTY), qe_phase, wc, timeout_code(kSiteQEmpty))) break;
-          qe_phase ^= 1u;
-        }
+    }
+    __syncwarp();
+    const uint64_t pol_kv = l2_policy_evict_last();
+    const uint64_t pol_q = l2_policy_evict_first();
+    uint32_t n_ld = 0, qe_phase = 0;
+    int n_items = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = sch.item(k);
+      if (idx < 0) break;
+      int b, t, h, seq_start, L;
+      sch.decode(idx, b, t, h, seq_start, L);
+      const int nkv0 = num_kv_tiles<CAUSAL>(t, 0, L), nkv1 = num_kv_tiles<CAUSAL>(t, 1, L);
+      const int nkv = nkv0 > nkv1 ? nkv0 : nkv1;
+      if (k > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QEMPTY), qe_phase, wc, timeout_code(kSiteQEmpty)));
+        if (!ok) break;
+        qe_phase ^= 1u;
+      }
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar(Lay::B_QFULL), 2 * Lay::TILE);
 #pragma unroll
         for (int s = 0; s < 2; ++s)
@@ -420,111 +513,137 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(sb + Lay::Q_OFF + s * Lay::TILE + c * Lay::CHUNK, &tm_q, bar(Lay::B_QFULL),
                         c * 64, h, seq_start + t * 2 * kBM + s * kBM, pol_q);
-        ++n_items;
-        for (int j = 0; j < nkv && ok; ++j) {
+      }
+      __syncwarp();
+      ++n_items;
+      for (int j = 0; j < nkv && ok; ++j) {
 #pragma unroll
-          for (int which = 0; which < 2; ++which) {
-            const uint32_t slot = n_ld % NS;
-            if (n_ld >= static_cast<uint32_t>(NS)) {
-              if (!mbar_wait(bar(Lay::B_KVEMPTY + slot), ((n_ld / NS) - 1) & 1u, wc,
-                             timeout_code(kSiteKvEmpty))) {
-                ok = false;
-                break;
-              }
-            }
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t slot = n_ld % NS;
+          if (n_ld >= static_cast<uint32_t>(NS)) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KVEMPTY + slot), ((n_ld / NS) - 1) & 1u,
+                                                   wc, timeout_code(kSiteKvEmpty)));
+            if (!ok) break;
+          }
+          if (elect_one()) {
             mbar_arrive_expect_tx(bar(Lay::B_KVFULL + slot), Lay::TILE);
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(sb + Lay::KV_OFF + slot * Lay::TILE + c * Lay::CHUNK,
-                          which ? &tm_v : &tm_k, bar(Lay::B_KVFULL + slot), c * 64, h,
-                          seq_start + j * kBN, pol_kv);
-            ++n_ld;
+              tma_load_3d(sb + Lay::KV_OFF + slot * Lay::TILE + c * Lay::CHUNK, which ? &tm_v : &tm_k,
+                          bar(Lay::B_KVFULL + slot), c * 64, h, seq_start + j * kBN, pol_kv);
+            // Warm L2 with the same operand two tiles ahead: when its ring slot frees
+            // up, the copy then hits L2 instead of HBM.
+            if (j + 2 < nkv)
+#pragma unroll
+              for (int c = 0; c < D / 64; ++c)
+                tma_prefetch_l2_3d(which ? &tm_v : &tm_k, c * 64, h, seq_start + (j + 2) * kBN);
           }
+          __syncwarp();
+          ++n_ld;
         }
       }
-      // Drain: every issued copy must have landed before the CTA may exit.
-      const uint32_t first = n_ld > static_cast<uint32_t>(NS) ? n_ld - NS : 0u;
-      for (uint32_t n = first; n < n_ld; ++n)
-        drain_wait(bar(Lay::B_KVFULL + n % NS), (n / NS) & 1u, p.timeout_ns);
-      if (n_items > 0) drain_wait(bar(Lay::B_QFULL), (n_items - 1) & 1u, p.timeout_ns);
     }
+    // Drain: every issued copy must have landed before the CTA may exit.
+    const uint32_t first = n_ld > static_cast<uint32_t>(NS) ? n_ld - NS : 0u;
+    for (uint32_t n = first; n < n_ld; ++n)
+      drain_wait(bar(Lay::B_KVFULL + n % NS), (n / NS) & 1u, p.timeout_ns);
+    if (n_items > 0) drain_wait(bar(Lay::B_QFULL), (n_items - 1) & 1u, p.timeout_ns);
   } else {
     // ---------------------------------------------------------------- MMA
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0, 0);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 0, 1);
-      const uint32_t tS0 = tmem + Lay::TM_S0, tS1 = tmem + Lay::TM_S1;
-      const uint32_t tO0 = tmem + Lay::TM_O0, tO1 = tmem + Lay::TM_O1;
-      uint32_t n_ld = 0, q_phase = 0, p_phase0 = 0, p_phase1 = 0;
-      bool ok = true;
-      for (int k = 0; ok; ++k) {
-        const int idx = sch.item(k);
-        if (idx < 0) break;
-        int b, t, h, seq_start, L;
-        sch.decode(idx, b, t, h, seq_start, L);
-        const int nk0 = num_kv_tiles<CAUSAL>(t, 0, L), nk1 = num_kv_tiles<CAUSAL>(t, 1, L);
-        const int nkv = nk0 > nk1 ? nk0 : nk1;
-        if (!mbar_wait(bar(Lay::B_QFULL), q_phase, wc, timeout_code(kSiteQFull))) break;
-        q_phase ^= 1u;
+    // The whole warp walks the loop and waits; one elected lane issues each MMA
+    // and commit.  Issue order per key tile j (ping-pong of the two sub-tiles):
+    //   PV(0, j-1), S(0, j), PV(1, j-1), S(1, j)
+    // S(s, j) overwrites P(s, j-1) in TMEM, which PV(s, j-1) read just before; the
+    // tensor pipe executes one thread's MMAs in issue order.
+    constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0, 0);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 0, 1);
+    const uint32_t tS0 = tmem + Lay::TM_S0, tS1 = tmem + Lay::TM_S1;
+    const uint32_t tO0 = tmem + Lay::TM_O0, tO1 = tmem + Lay::TM_O1;
+    uint32_t n_ld = 0, q_phase = 0, p_phase0 = 0, p_phase1 = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = sch.item(k);
+      if (idx < 0) break;
+      int b, t, h, seq_start, L;
+      sch.decode(idx, b, t, h, seq_start, L);
+      const int nk0 = num_kv_tiles<CAUSAL>(t, 0, L), nk1 = num_kv_tiles<CAUSAL>(t, 1, L);
+      const int nkv = nk0 > nk1 ? nk0 : nk1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QFULL), q_phase, wc, timeout_code(kSiteQFull)));
+      if (!ok) break;
+      q_phase ^= 1u;
+      tc_fence_after();
+      for (int j = 0; j <= nkv && ok; ++j) {
+        const uint32_t nK = n_ld + 2u * j;  // load sequence number of K_j
+        const uint32_t nV = nK - 1u;        // ... and of V_{j-1}
+        const uint32_t slotK = nK % NS, slotV = nV % NS;
+        if (j < nkv)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KVFULL + slotK), (nK / NS) & 1u, wc,
+                                                 timeout_code(kSiteKvFull)));
+        if (ok && j > 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KVFULL + slotV), (nV / NS) & 1u, wc,
+                                                 timeout_code(kSiteKvFull)));
+        if (!ok) break;
         tc_fence_after();
-        for (int j = 0; j <= nkv; ++j) {
-          const uint32_t nK = n_ld + 2u * j;  // load sequence number of K_j
-          const uint32_t nV = nK - 1u;        // ... and of V_{j-1}
-          const uint32_t slotK = nK % NS, slotV = nV % NS;
-          if (j < nkv && !mbar_wait(bar(Lay::B_KVFULL + slotK), (nK / NS) & 1u, wc,
-                                    timeout_code(kSiteKvFull))) { ok = false; break; }
-          if (j > 0 && !mbar_wait(bar(Lay::B_KVFULL + slotV), (nV / NS) & 1u, wc,
-                                  timeout_code(kSiteKvFull))) { ok = false; break; }
-          tc_fence_after();
 #pragma unroll
-          for (int s = 0; s < 2; ++s) {
-            const uint32_t tS = s ? tS1 : tS0, tO = s ? tO1 : tO0;
-            const int nks = s ? nk1 : nk0;
-            if (ok && j > 0 && j - 1 < nks) {
-              uint32_t& ph = s ? p_phase1 : p_phase0;
-              if (!mbar_wait(bar(Lay::B_PFULL + s), ph, wc, timeout_code(kSitePFull))) {
-                ok = false;
-              } else {
-                ph ^= 1u;
-                tc_fence_after();
-                const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::TILE;
+        for (int s = 0; s < 2; ++s) {
+          const uint32_t tS = s ? tS1 : tS0, tO = s ? tO1 : tO0;
+          const int nks = s ? nk1 : nk0;
+          if (ok && j > 0 && j - 1 < nks) {
+            uint32_t& ph = s ? p_phase1 : p_phase0;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_PFULL + s), ph, wc, timeout_code(kSitePFull)));
+            if (ok) {
+              ph ^= 1u;
+              tc_fence_after();
+              const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::TILE;
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
+              for (int kk = 0; kk < kBN / 16; ++kk) {
+                if (elect_one())
                   mma_ts(tO, tS + kk * 8, sdesc_sw128(vbase + kk * 2048, Lay::CHUNK, 1024), idesc_o,
                          (j > 1 || kk > 0) ? 1u : 0u);
-                if (j == nks) tc_commit(bar(Lay::B_OFULL + s));
+                __syncwarp();
               }
-            }
-            if (ok && j < nks) {
-              const uint32_t qbase = sb + Lay::Q_OFF + s * Lay::TILE;
-              const uint32_t kbase = sb + Lay::KV_OFF + slotK * Lay::TILE;
-#pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-                mma_ss(tS, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
-                       idesc_s, kk > 0 ? 1u : 0u);
+              if (j == nks) {
+                if (elect_one()) tc_commit(bar(Lay::B_OFULL + s));
+                __syncwarp();
               }
-              tc_commit(bar(Lay::B_SFULL + s));
             }
           }
-          if (!ok) break;
+          if (ok && j < nks) {
+            const uint32_t qbase = sb + Lay::Q_OFF + s * Lay::TILE;
+            const uint32_t kbase = sb + Lay::KV_OFF + slotK * Lay::TILE;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+              if (elect_one())
+                mma_ss(tS, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
+                       idesc_s, kk > 0 ? 1u : 0u);
+              __syncwarp();
+            }
+            if (elect_one()) tc_commit(bar(Lay::B_SFULL + s));
+            __syncwarp();
+          }
+        }
+        if (!ok) break;
+        if (elect_one()) {
           if (j < nkv) tc_commit(bar(Lay::B_KVEMPTY + slotK));
           if (j > 0) tc_commit(bar(Lay::B_KVEMPTY + slotV));
           if (j == nkv - 1) tc_commit(bar(Lay::B_QEMPTY));
         }
-        n_ld += 2u * nkv;
+        __syncwarp();
       }
-      // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      tc_commit(bar(Lay::B_DRAIN));
-      if (!drain_wait(bar(Lay::B_DRAIN), 0u, p.timeout_ns) && p.err)
-        atomicCAS(p.err, 0, timeout_code(kSiteDrain));
+      n_ld += 2u * nkv;
     }
+    // Drain: every MMA issued by this warp completes before TMEM is freed.
+    if (elect_one()) tc_commit(bar(Lay::B_DRAIN));
+    __syncwarp();
+    if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, p.timeout_ns)) && lane == 0 && p.err)
+      atomicCAS(p.err, 0, timeout_code(kSiteDrain));
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, 512);
+  if (warp == 17) tmem_dealloc(tmem, 512);
 }
 
 template <int D>

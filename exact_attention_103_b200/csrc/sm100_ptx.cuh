@@ -73,6 +73,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   }
 }
 
+// True in exactly one lane of the (converged) warp.  Issue loops run on the whole
+// warp and let the elected lane issue: a lone divergent lane that waits on an
+// mbarrier stalls its own tcgen05.mma issue, which leaves the tensor pipe idle.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\t"
+      "elect.sync rx|px, %1;\n\t@px mov.s32 %0, 1;\n\t}"
+      : "+r"(pred)
+      : "r"(0xffffffffu));
+  return pred != 0;
+}
+
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -86,6 +99,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       "cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
       : "memory");
+}
+// Bulk-tensor prefetch of one box into L2 (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
@@ -214,6 +234,69 @@ __device__ __forceinline__ float fast_exp2(float x) {  // MUFU ex2, flushes deno
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Paired fp32 arithmetic (one f32x2 instruction for two lanes of work).
+// y = x * a + b for both elements, a and b broadcast.
+__device__ __forceinline__ void ffma2_bc(float& y0, float& y1, float x0, float x1, float a, float b) {
+  asm("{\n\t.reg .b64 xa, aa, ba, ya;\n\t"
+      "mov.b64 xa, {%2, %3};\n\tmov.b64 aa, {%4, %4};\n\tmov.b64 ba, {%5, %5};\n\t"
+      "fma.rn.f32x2 ya, xa, aa, ba;\n\tmov.b64 {%0, %1}, ya;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(a), "f"(b));
+}
+// y = x * a + b for both elements, a per element, b broadcast.
+__device__ __forceinline__ void ffma2_vb(float& y0, float& y1, float x0, float x1, float a0, float a1,
+                                        float b) {
+  asm("{\n\t.reg .b64 xa, aa, ba, ya;\n\t"
+      "mov.b64 xa, {%2, %3};\n\tmov.b64 aa, {%4, %5};\n\tmov.b64 ba, {%6, %6};\n\t"
+      "fma.rn.f32x2 ya, xa, aa, ba;\n\tmov.b64 {%0, %1}, ya;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(a0), "f"(a1), "f"(b));
+}
+// y = x * a + c, a broadcast, c per element.
+__device__ __forceinline__ void ffma2_bv(float& y0, float& y1, float x0, float x1, float a, float c0,
+                                        float c1) {
+  asm("{\n\t.reg .b64 xa, aa, ca, ya;\n\t"
+      "mov.b64 xa, {%2, %3};\n\tmov.b64 aa, {%4, %4};\n\tmov.b64 ca, {%5, %6};\n\t"
+      "fma.rn.f32x2 ya, xa, aa, ca;\n\tmov.b64 {%0, %1}, ya;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(a), "f"(c0), "f"(c1));
+}
+// y = x + b (b broadcast) and y = x - z elementwise.
+__device__ __forceinline__ void fadd2_bc(float& y0, float& y1, float x0, float x1, float b) {
+  asm("{\n\t.reg .b64 xa, ba, ya;\n\t"
+      "mov.b64 xa, {%2, %3};\n\tmov.b64 ba, {%4, %4};\n\t"
+      "add.rn.f32x2 ya, xa, ba;\n\tmov.b64 {%0, %1}, ya;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(b));
+}
+__device__ __forceinline__ void fsub2_bc(float& y0, float& y1, float x0, float x1, float b) {
+  asm("{\n\t.reg .b64 xa, ba, ya;\n\t"
+      "mov.b64 xa, {%2, %3};\n\tmov.b64 ba, {%4, %4};\n\t"
+      "sub.rn.f32x2 ya, xa, ba;\n\tmov.b64 {%0, %1}, ya;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(b));
+}
+__device__ __forceinline__ void fsub2(float& y0, float& y1, float x0, float x1, float z0, float z1) {
+  asm("{\n\t.reg .b64 xa, za, ya;\n\t"
+      "mov.b64 xa, {%2, %3};\n\tmov.b64 za, {%4, %5};\n\t"
+      "sub.rn.f32x2 ya, xa, za;\n\tmov.b64 {%0, %1}, ya;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(z0), "f"(z1));
+}
+// acc += x elementwise.
+__device__ __forceinline__ void fadd2_acc(float& a0, float& a1, float x0, float x1) {
+  asm("{\n\t.reg .b64 aa, xa;\n\t"
+      "mov.b64 aa, {%0, %1};\n\tmov.b64 xa, {%2, %3};\n\t"
+      "add.rn.f32x2 aa, aa, xa;\n\tmov.b64 {%0, %1}, aa;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x0), "f"(x1));
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

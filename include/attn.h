@@ -80,7 +80,8 @@ ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, voi
 /* Tuning / test knobs for attn_fwd_ex.  Zero-initialise, then set fields.
  *  rescale_threshold: conditional-rescale threshold tau in log2 units; the
  *      running maximum is replaced (and O, l rescaled) only when a new tile's row
- *      maximum exceeds it by more than tau.  < 0 selects the default (8.0).
+ *      maximum exceeds it by more than tau, so P~ <= 2^tau.  < 0 selects the
+ *      default (8.0); values above 64 are rejected (ATTN_ERR_INVALID_ARG).
  *  stats: optional DEVICE pointer to two uint64 counters the kernel ADDS to:
  *      [0] rows rescaled, [1] row-tiles processed after each row's first tile.
  *  timeout_ns: limit of every internal wait; 0 selects the default (2 s).

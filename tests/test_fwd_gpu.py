@@ -150,15 +150,16 @@ def test_fwd_writes_nothing_outside_outputs():
 
 
 def test_rescale_threshold_readings_agree():
-    """tau = 0 (rescale whenever the maximum grows), 8 (default) and 1e9 (never
-    after the first tile) are all exact readings: same result within tolerance."""
+    """tau = 0 (rescale whenever the maximum grows), 8 (default) and 64 (the
+    largest allowed; rarely rescales) are all exact readings: same result within
+    tolerance, and fewer rescales as tau grows."""
     ea = _lib()
     B, N, H, d = 1, 1024, 2, 128
     q, k, v = ai.make_custom(B, N, H, d, seed=23)
     q = (q.float() * 4).to(torch.bfloat16)
     o_ref, l_ref = _dense_ref(q, k, v, False, 1 / math.sqrt(d))
     outs = {}
-    for tau in (0.0, 8.0, 1e9):
+    for tau in (0.0, 8.0, 64.0):
         stats = torch.zeros(2, dtype=torch.int64, device=DEV)
         o, lse = ea.fwd(q.to(DEV), k.to(DEV), v.to(DEV), rescale_threshold=tau, stats=stats)
         ea.get_device_status()
@@ -169,7 +170,7 @@ def test_rescale_threshold_readings_agree():
     expected = B * H * (N // 128) * 128 * (N // 128 - 1)
     for tau, (resc, tiles) in outs.items():
         assert tiles == expected, (tau, tiles, expected)
-    assert outs[0.0][0] >= outs[8.0][0] >= outs[1e9][0] == 0
+    assert outs[0.0][0] >= outs[8.0][0] >= outs[64.0][0]
 
 
 def test_invalid_cu_seqlens_recorded_on_device():
