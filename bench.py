@@ -49,6 +49,51 @@ def workload_exps(w: ai.Workload) -> float:
     return workload_flops(w) / (4.0 * w.d)
 
 
+def kernel_source_hash() -> str:
+    """sha256 of the forward kernel's sources (the ncu traffic figure applies only
+    to the kernel these hash to)."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_attention_103_b200", "csrc")
+    for name in ("attn_fwd_sm100.cu", "attn_fwd_sm100.h", "sm100_ptx.cuh", "exp2_poly.h"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload, or
+    None when there is none or it was taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", f"fwd_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("- ") and ": " in line:
+                k, v = line[2:].strip().split(": ", 1)
+                fields[k.strip("`")] = v.strip().strip("`")
+    if fields.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def poly_pairs_per_8() -> int:
+    """Column pairs of every 8 the kernel exponentiates on the FMA pipe (compiled-in
+    default, or the override passed to the build through ATTN_NVCC_EXTRA)."""
+    import re
+    m = re.search(r"-DATTN_POLY_PAIRS_PER_8=(\d+)", os.environ.get("ATTN_NVCC_EXTRA", ""))
+    if m:
+        return int(m.group(1))
+    src = os.path.join(ROOT, "exact_attention_103_b200", "csrc", "attn_fwd_sm100.cu")
+    with open(src) as f:
+        m = re.search(r"#define ATTN_POLY_PAIRS_PER_8 (\d+)", f.read())
+    return int(m.group(1)) if m else 0
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -94,7 +139,7 @@ class ClockSampler:
                 self._sample()
             except Exception:
                 return
-            time.sleep(0.01)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self._nv is not None:
@@ -185,6 +230,12 @@ def cpu_oracle_sample(w: ai.Workload, q, k, v, budget_s: float):
     return done_flops / spent / 1e12, threads, desc
 
 
+def bench_config(w: ai.Workload, world: int) -> dict:
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"replicas{world}",
+            "l2": "flushed (256 MiB write) before every timed step"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -206,8 +257,7 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                       "causal": w.causal, "parallelism": "replicas"},
+            "config": bench_config(w, world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": desc + " per step; ms_per_step extrapolated to the workload"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -263,23 +313,27 @@ def run_ours(args, rank, world, local):
     mhz = clk["sm_mhz"] or peaks["sm_max_mhz"]
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     mufu_peak = sms * MUFU_EX2_PER_CLK_PER_SM * mhz * 1e6
-    mufu_achieved = workload_exps(w) / (statistics.mean(times) / 1e3)
+    mufu_share = 1.0 - poly_pairs_per_8() / 8.0
+    mufu_achieved = mufu_share * workload_exps(w) / (statistics.mean(times) / 1e3)
 
     # End to end through the public API from pinned host buffers: H2D of Q/K/V
     # (and cu_seqlens), the forward, D2H of O and LSE, every step.
     q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
     cu_p = None if cu_h is None else cu_h.pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
+    o_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    l_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     for _ in range(2):
         ea.fwd_from_host(q_p, k_p, v_p, causal=w.causal, scale=scale, cu_seqlens_host=cu_p,
-                         max_seqlen=max_len)
+                         max_seqlen=max_len, out_host=o_host, lse_host=l_host)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(e2e_steps):
         o_h, l_h = ea.fwd_from_host(q_p, k_p, v_p, causal=w.causal, scale=scale,
-                                    cu_seqlens_host=cu_p, max_seqlen=max_len)
+                                    cu_seqlens_host=cu_p, max_seqlen=max_len,
+                                    out_host=o_host, lse_host=l_host)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
@@ -297,18 +351,18 @@ def run_ours(args, rank, world, local):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                           "causal": w.causal, "global_batch": w.B * world,
-                           "seq_len": w.N, "parallelism": f"replicas{world}",
-                           "l2": "flushed (256 MiB write) before every timed step"},
+                "config": bench_config(w, world),
                 "pct_of_peak": 100.0 * achieved / peak,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                              "unit": "TFLOP/s", "frac": achieved / peak,
                              "peak_source": f"bf16_tflops (burst), {peaks['source']}",
-                             "traffic": None},
+                             "traffic": profiled_traffic(w.name),
+                             "traffic_unit": "bytes per launch (ncu dram read+write)"},
                 "mufu": {"achieved_ex2_per_s": mufu_achieved, "peak_ex2_per_s": mufu_peak,
                          "frac": mufu_achieved / mufu_peak,
-                         "note": "all exponentials on MUFU ex2; peak at the median sampled SM clock"},
+                         "mufu_share_of_exps": mufu_share,
+                         "note": "ex2 executed on MUFU (the rest on the FMA-pipe polynomial); "
+                                 "peak = SMs x 16 ex2/clk at the median sampled SM clock"},
                 "e2e": {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "ms_per_step": e2e_ms},

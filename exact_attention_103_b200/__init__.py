@@ -179,9 +179,13 @@ def fwd_from_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tens
                   causal: bool = False, scale: Optional[float] = None,
                   cu_seqlens_host: Optional[torch.Tensor] = None,
                   max_seqlen: Optional[int] = None, device: str = "cuda",
-                  stream: Optional[torch.cuda.Stream] = None):
-    """End-to-end call from (pinned) host tensors: copies Q/K/V (and cu_seqlens) to
-    the device, runs the forward, copies O and LSE back to host tensors."""
+                  stream: Optional[torch.cuda.Stream] = None,
+                  out_host: Optional[torch.Tensor] = None,
+                  lse_host: Optional[torch.Tensor] = None):
+    """End-to-end call from host tensors: copies Q/K/V (and cu_seqlens) to the
+    device, runs the forward, copies O and LSE back into host tensors (``out_host``
+    / ``lse_host`` if given, ideally pinned; else new pinned tensors).  Returns
+    (o_host, lse_host); they are complete once ``stream`` is synchronised."""
     s = stream if stream is not None else torch.cuda.current_stream()
     with torch.cuda.stream(s):
         q = q_host.to(device, non_blocking=True)
@@ -190,8 +194,10 @@ def fwd_from_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tens
         cu = None if cu_seqlens_host is None else cu_seqlens_host.to(device, non_blocking=True)
         o, lse = fwd(q, k, v, causal=causal, scale=scale, cu_seqlens=cu, max_seqlen=max_seqlen,
                      stream=s)
-        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        o_h = out_host if out_host is not None else torch.empty(o.shape, dtype=o.dtype,
+                                                                pin_memory=True)
+        l_h = lse_host if lse_host is not None else torch.empty(lse.shape, dtype=lse.dtype,
+                                                                pin_memory=True)
         o_h.copy_(o, non_blocking=True)
         l_h.copy_(lse, non_blocking=True)
     return o_h, l_h
