@@ -25,7 +25,7 @@ ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_WORKSPACE = 3, 4, 5
 # Every symbol include/attn.h and include/attn_selftest.h declare.
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_ex", "attn_bwd", "attn_bwd_workspace_size",
                     "attn_get_device_status", "attn_status_string", "attn_last_error",
-                    "attn_selftest_umma")
+                    "attn_selftest_umma", "attn_fwd_noalloc")
 
 
 class AttnError(RuntimeError):
@@ -72,6 +72,9 @@ def load_library(path: str = LIB_PATH):
     lib.attn_last_error.restype = ctypes.c_char_p
     lib.attn_selftest_umma.argtypes = [vp, vp, vp, vp, vp, ci, vp]
     lib.attn_selftest_umma.restype = ci
+    lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp,
+                                     ctypes.c_int64, ci, vp]
+    lib.attn_fwd_noalloc.restype = ci
     _lib = lib
     return lib
 
@@ -201,6 +204,34 @@ def fwd_from_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tens
         o_h.copy_(o, non_blocking=True)
         l_h.copy_(lse, non_blocking=True)
     return o_h, l_h
+
+
+def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                lse: torch.Tensor, causal: bool = False, scale: Optional[float] = None,
+                cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: Optional[int] = None,
+                check: bool = True, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """The allocation-free forward ``attn_fwd_noalloc``: the caller supplies ``out``
+    and ``lse`` (layouts as for ``fwd``); the library allocates no device memory.
+    With ``check`` the call synchronises the stream and raises on a kernel-recorded
+    error."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, n)
+    _need(lse, "lse", torch.float32)
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if cu_seqlens is None:
+        B, N, H, _ = q.shape
+        total, cu_ptr = 0, None
+    else:
+        _need(cu_seqlens, "cu_seqlens", torch.int32)
+        B, H, N = cu_seqlens.numel() - 1, q.shape[1], int(max_seqlen)
+        total, cu_ptr = q.shape[0], cu_seqlens.data_ptr()
+    with torch.cuda.device(q.device):
+        st = lib.attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                  lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                  cu_ptr, total, int(bool(check)), _stream_ptr(stream))
+    _check(st)
 
 
 def get_device_status(stream: Optional[torch.cuda.Stream] = None) -> None:

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libattn.so")
-SOURCES = ["attn_api.cu", "attn_fwd_sm100.cu", "selftest_sm100.cu"]
+SOURCES = ["attn_api.cu", "attn_fwd_sm100.cu", "selftest_sm100.cu", "attn_noalloc.cu"]
 HEADERS = ["attn_fwd_sm100.h", "sm100_ptx.cuh"]
 PUBLIC_HEADERS = [os.path.join(ROOT, "include", h) for h in ("attn.h", "attn_selftest.h")]
 NVCC = os.environ.get("NVCC", "nvcc")

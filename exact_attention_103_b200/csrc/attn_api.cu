@@ -192,6 +192,23 @@ attn_status_t prepare_selftest(int** err, bool (**mk)(CUtensorMap*, const void*,
   *mk = make_map;
   return ATTN_OK;
 }
+// Pieces shared with the allocation-free entry point (attn_noalloc.cu).  None of
+// them allocates device memory.
+attn_status_t load_tensor_map_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return ATTN_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+    return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return ATTN_OK;
+}
+bool make_tensor_map(CUtensorMap* m, const void* ptr, int64_t total, int H, int d) {
+  return make_map(m, ptr, total, H, d);
+}
+attn_status_t report(attn_status_t s, const char* message) { return fail(s, "%s", message); }
 }  // namespace attn_internal
 
 extern "C" {

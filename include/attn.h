@@ -120,6 +120,33 @@ ATTN_API attn_status_t attn_bwd(const void* q, const void* k, const void* v, con
 /* Workspace bytes attn_bwd needs (total_tokens = B*N dense, cu_seqlens[B] varlen). */
 ATTN_API size_t attn_bwd_workspace_size(int B, int H, int N, int d, int total_tokens, int deterministic);
 
+/*
+ * Forward pass that allocates nothing, for callers that cannot call cudaMalloc:
+ * a framework that has reserved all device memory for its own pool, code that
+ * must not trigger the implicit synchronisation an allocation may cause, or code
+ * that runs while a stream is being captured.  (The pages have no counterpart:
+ * this is an interface of this library.)  The ordinary entry points allocate a
+ * 4-byte device status word on a device's first call; here that scratch lives in
+ * a static device array of 256 bytes inside the library, which every GPU that
+ * loads the library holds until the process exits.  Same operation, layouts and
+ * limits as attn_fwd, default rescale threshold.
+ *  - total_tokens: varlen only, must equal cu_seqlens[B] (no device read-back);
+ *    ignored for dense batches.
+ *  - check: 0 = return after launching; != 0 = synchronise `stream` and return the
+ *    status the kernel recorded (ATTN_ERR_TIMEOUT, or ATTN_ERR_INVALID_ARG for bad
+ *    cu_seqlens).
+ *  - The first call on a device does its set-up there (looks up the array's
+ *    device address); make that first call before any stream capture.
+ *  - Every call shares the array: each call clears the status word on `stream`
+ *    before its launch, and calls whose kernels overlap on the GPU race on it.
+ *  - A kernel that needed more scratch than the array holds would be rejected with
+ *    ATTN_ERR_WORKSPACE; the forward kernel needs 4 bytes.
+ */
+ATTN_API attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, int B, int H, int N, int d, int causal,
+                                        float scale, const int32_t* cu_seqlens,
+                                        int64_t total_tokens, int check, attn_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device error word of the
  * current device (ATTN_OK if no kernel recorded an error). */
 ATTN_API attn_status_t attn_get_device_status(attn_stream_t stream);
