@@ -313,7 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = wq * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t t_s = tmem + lane_bits + (s ? Lay::TM_S1 : Lay::TM_S0);
-    const uint32_t t_p = t_s + 32 * hf;        // this half's packed bf16 P columns
+    // This half's packed bf16 P columns.  Half 1 writes columns 32..63, which hold
+    // half 0's scores; that is safe because half 1 passes the pair's max exchange
+    // of the tile only after half 0 arrived there, i.e. after half 0's TMEM load.
+    const uint32_t t_p = t_s + 32 * hf;
     const uint32_t t_o = tmem + lane_bits + (s ? Lay::TM_O1 : Lay::TM_O0) + (D / 2) * hf;
     // Pair exchange: write a value, arrive (one arrival per warp), wait for the
     // partner's arrival, read its value.  Slots alternate with the exchange count,

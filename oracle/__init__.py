@@ -61,6 +61,9 @@ def _load():
         lib.oracle_online_fwd.restype = ctypes.c_int64
         lib.oracle_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, ci, i64p, ci, ci, ci, cd, ci]
         lib.oracle_bwd.restype = ci
+        lib.oracle_bwd_sampled.argtypes = [dp, dp, dp, dp, ci, i64p, ci, ci, ci, cd, ci, ci,
+                                           ip, ci, ip, ci, dp, dp, dp, ci]
+        lib.oracle_bwd_sampled.restype = ci
         _lib = lib
     return _lib
 
@@ -163,6 +166,26 @@ def bwd(q, k, v, dout, cu, causal: bool, scale: float, nthreads: int = 0):
                             float(scale), int(nthreads))
     if rc < 0:
         raise ValueError("oracle_bwd rejected its arguments")
+    return dq, dk, dv
+
+
+def bwd_sampled(q, k, v, dout, cu, causal: bool, scale: float, b: int, h: int, q_rows, k_rows,
+                nthreads: int = 0):
+    """Backward at selected local query rows (dQ) and key rows (dK, dV) of sequence b,
+    head h: returns (dq [nq,d], dk [nk,d], dv [nk,d]) in fp64."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    T, H, d = q.shape
+    cu = _cu(cu, T)
+    qi = np.ascontiguousarray(np.asarray(q_rows, dtype=np.int32))
+    kj = np.ascontiguousarray(np.asarray(k_rows, dtype=np.int32))
+    dq = np.zeros((qi.size, d)); dk = np.zeros((kj.size, d)); dv = np.zeros((kj.size, d))
+    rc = _load().oracle_bwd_sampled(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), cu.size - 1,
+                                    _ptr(cu, ctypes.c_int64), H, d, int(causal), float(scale),
+                                    int(b), int(h), _ptr(qi, ctypes.c_int), qi.size,
+                                    _ptr(kj, ctypes.c_int), kj.size, _ptr(dq), _ptr(dk), _ptr(dv),
+                                    int(nthreads))
+    if rc < 0:
+        raise ValueError("oracle_bwd_sampled rejected its arguments")
     return dq, dk, dv
 
 

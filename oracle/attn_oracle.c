@@ -24,6 +24,8 @@
  *                      (FlashAttention 1 recurrences, FlashAttention 2 deferred
  *                      normalisation, FlashAttention 4 conditional rescale)
  *   oracle_bwd         the textbook backward pass (recomputes P)
+ *   oracle_bwd_sampled the same gradients for selected query rows (dQ) and key
+ *                      rows (dK, dV) of one (sequence, head), for full-size checks
  *
  * Empty rows cannot occur: a causal row always sees its own key, a non-causal row
  * sees every key of a non-empty sequence.  Zero-length sequences are skipped.
@@ -337,5 +339,102 @@ int oracle_bwd(const double* q, const double* k, const double* v, const double* 
     free(prow);
     free(orow);
   }
+  return used;
+}
+
+/* The textbook backward of oracle_bwd, for one (sequence b, head h), evaluated only
+ * at selected positions so that long sequences stay affordable:
+ *   dQ_i for the local query rows qi[0..nq), dK_j and dV_j for the local key rows
+ *   kj[0..nk).
+ * Per query row it first computes, from the definition, m_i, l_i (so P_ij =
+ * exp(s_ij - m_i) / l_i), the exact O_i and D_i = <dO_i, O_i> (rows in parallel).
+ * Then dQ_i = scale sum_j P_ij (<dO_i, v_j> - D_i) k_j, and for a key j
+ * dV_j = sum_i P_ij dO_i and dK_j = scale sum_i P_ij (<dO_i, v_j> - D_i) q_i over the
+ * query rows that see key j.  dq_out is [nq][d], dk_out and dv_out [nk][d]. */
+int oracle_bwd_sampled(const double* q, const double* k, const double* v, const double* dout,
+                       int nseq, const int64_t* cu, int H, int d, int causal, double scale,
+                       int b, int h, const int* qi, int nq, const int* kj, int nk,
+                       double* dq_out, double* dk_out, double* dv_out, int nthreads) {
+  if (b < 0 || b >= nseq || h < 0 || h >= H || d <= 0) return -1;
+  const int used = set_threads(nthreads);
+  const int64_t base = cu[b];
+  const int L = (int)(cu[b + 1] - cu[b]);
+  for (int r = 0; r < nq; ++r) if (qi[r] < 0 || qi[r] >= L) return -1;
+  for (int r = 0; r < nk; ++r) if (kj[r] < 0 || kj[r] >= L) return -1;
+  double* m = (double*)malloc(sizeof(double) * (L > 0 ? L : 1));
+  double* l = (double*)malloc(sizeof(double) * (L > 0 ? L : 1));
+  double* Dv = (double*)malloc(sizeof(double) * (L > 0 ? L : 1));
+#define QROW(i) (q + ((base + (i)) * H + h) * (int64_t)d)
+#define KROW(j) (k + ((base + (j)) * H + h) * (int64_t)d)
+#define VROW(j) (v + ((base + (j)) * H + h) * (int64_t)d)
+#define DOROW(i) (dout + ((base + (i)) * H + h) * (int64_t)d)
+  /* Pass 1: per query row, the softmax statistics, O_i and D_i. */
+#pragma omp parallel
+  {
+    double* srow = (double*)malloc(sizeof(double) * (L > 0 ? L : 1));
+    double* orow = (double*)malloc(sizeof(double) * d);
+#pragma omp for schedule(dynamic, 16)
+    for (int i = 0; i < L; ++i) {
+      const int nvis = visible_keys(i, L, causal);
+      double mi = -INFINITY;
+      for (int j = 0; j < nvis; ++j) {
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += QROW(i)[c] * KROW(j)[c];
+        srow[j] = scale * acc;
+        if (srow[j] > mi) mi = srow[j];
+      }
+      double li = 0.0;
+      for (int j = 0; j < nvis; ++j) { srow[j] = exp(srow[j] - mi); li += srow[j]; }
+      for (int c = 0; c < d; ++c) orow[c] = 0.0;
+      for (int j = 0; j < nvis; ++j)
+        for (int c = 0; c < d; ++c) orow[c] += (srow[j] / li) * VROW(j)[c];
+      double di = 0.0;
+      for (int c = 0; c < d; ++c) di += DOROW(i)[c] * orow[c];
+      m[i] = mi; l[i] = li; Dv[i] = di;
+    }
+    free(srow);
+    free(orow);
+  }
+  /* P_ij and dS_ij from the statistics. */
+#define P_OF(i, j, pij, dsij)                                        \
+  do {                                                                \
+    double acc_ = 0.0, dp_ = 0.0;                                     \
+    for (int c = 0; c < d; ++c) acc_ += QROW(i)[c] * KROW(j)[c];      \
+    pij = exp(scale * acc_ - m[i]) / l[i];                            \
+    for (int c = 0; c < d; ++c) dp_ += DOROW(i)[c] * VROW(j)[c];      \
+    dsij = pij * (dp_ - Dv[i]);                                       \
+  } while (0)
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int r = 0; r < nq; ++r) {
+    const int i = qi[r];
+    double* out = dq_out + (int64_t)r * d;
+    for (int c = 0; c < d; ++c) out[c] = 0.0;
+    for (int j = 0; j < visible_keys(i, L, causal); ++j) {
+      double pij, dsij;
+      P_OF(i, j, pij, dsij);
+      for (int c = 0; c < d; ++c) out[c] += scale * dsij * KROW(j)[c];
+    }
+  }
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int r = 0; r < nk; ++r) {
+    const int j = kj[r];
+    double* dko = dk_out + (int64_t)r * d;
+    double* dvo = dv_out + (int64_t)r * d;
+    for (int c = 0; c < d; ++c) { dko[c] = 0.0; dvo[c] = 0.0; }
+    for (int i = causal ? j : 0; i < L; ++i) {
+      double pij, dsij;
+      P_OF(i, j, pij, dsij);
+      for (int c = 0; c < d; ++c) {
+        dvo[c] += pij * DOROW(i)[c];
+        dko[c] += scale * dsij * QROW(i)[c];
+      }
+    }
+  }
+#undef P_OF
+#undef QROW
+#undef KROW
+#undef VROW
+#undef DOROW
+  free(m); free(l); free(Dv);
   return used;
 }

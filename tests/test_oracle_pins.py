@@ -284,3 +284,21 @@ def test_bwd_key_shift_invariance(causal):
     _, dk, _ = oracle.bwd(_packed(q), _packed(k), _packed(v), _packed(do), cu, causal, 0.25)
     for b in range(2):
         np.testing.assert_allclose(dk[cu[b]:cu[b + 1]].sum(axis=0), 0.0, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_sampled_matches_torch_autograd(causal):
+    """The per-position backward equals PyTorch fp64 autograd at the chosen rows."""
+    lengths = [37, 70]
+    H, d = 2, 16
+    q, k, v, do = make_custom(0, 0, H, d, seed=20, lengths=lengths, n=4)
+    cu = np.array([0, 37, 107])
+    b, h = 1, 1
+    sl = slice(37, 107)
+    ref = _loss_grad_torch(q[sl][None], k[sl][None], v[sl][None], do[sl][None], causal, 0.3)
+    rows = [0, 5, 69, 33]
+    dq, dk, dv = oracle.bwd_sampled(_packed(q), _packed(k), _packed(v), _packed(do), cu, causal,
+                                    0.3, b, h, rows, rows)
+    np.testing.assert_allclose(dq, ref[0][0][rows, h], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dk, ref[1][0][rows, h], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv, ref[2][0][rows, h], rtol=0, atol=1e-11)
