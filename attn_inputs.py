@@ -65,6 +65,7 @@ CAUSAL = Workload("B2-H16-N8192-d128-causal", 2, 16, 8192, 128, True)
 _VL = varlen_lengths()
 VARLEN = Workload("varlen16-H16-d128-causal", len(_VL), 16, max(_VL), 128, True, lengths=_VL)
 BWD_CAUSAL = CAUSAL  # the backward problem uses the causal forward's shapes
+BWD_NAME = CAUSAL.name + "-bwd"
 
 ALL = {w.name: w for w in (TINY, DENSE, DENSE_X4, CAUSAL, VARLEN)}
 

@@ -268,6 +268,8 @@ def run_reference(args, rank, world):
 def run_ours(args, rank, world, local):
     import exact_attention_103_b200 as ea
     ea.load_library()
+    if args.workload == ai.BWD_NAME:
+        return run_bwd(args, rank, world, local)
     w = ai.ALL[args.workload]
     dev = torch.device("cuda", local)
     q_h, k_h, v_h, cu_h = make_inputs(w, "cpu")
@@ -372,12 +374,61 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def run_bwd(args, rank, world, local):
+    """Backward of the causal B2-H16-N8192-d128 problem: a step is one attn_bwd call
+    (D = rowsum(dO*O), dK/dV kernel, dQ kernel) with O and LSE from an untimed forward.
+    FLOPs counted as 2.5x the forward's."""
+    import exact_attention_103_b200 as ea
+    w = ai.BWD_CAUSAL
+    dev = torch.device("cuda", local)
+    q, k, v, do = (t.to(dev) for t in ai.make_qkv(w, with_dout=True))
+    scale = 1.0 / math.sqrt(w.d)
+    o, lse = ea.fwd(q, k, v, causal=True, scale=scale)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flops = 2.5 * workload_flops(w)
+    peaks = load_peaks()
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        ea.bwd(q, k, v, o, lse, do, causal=True, scale=scale)
+    ea.get_device_status()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            starts[i].record()
+            ea.bwd(q, k, v, o, lse, do, causal=True, scale=scale)
+            ends[i].record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ea.get_device_status()
+    times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(times), world)
+    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    achieved = flops / (statistics.mean(times) / 1e3) / 1e12
+    if rank == 0:
+        cfg = bench_config(w, world)
+        cfg["workload"] = ai.BWD_NAME
+        line = {"metric": "attention bwd TFLOP/s (bf16, d=128, 1 B200; 2.5x forward FLOPs)",
+                "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "config": cfg,
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                             "traffic": None},
+                "gpu_launches": 3 * args.steps, "clocks": clocks.summary()}
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=ai.DENSE.name, choices=sorted(ai.ALL))
+    ap.add_argument("--workload", default=ai.DENSE.name, choices=sorted(ai.ALL) + [ai.BWD_NAME])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

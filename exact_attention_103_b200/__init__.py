@@ -234,6 +234,40 @@ def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Te
     _check(st)
 
 
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+        dout: torch.Tensor, causal: bool = False, scale: Optional[float] = None,
+        cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: Optional[int] = None,
+        deterministic: bool = False, stream: Optional[torch.cuda.Stream] = None):
+    """Exact attention backward on the GPU: returns (dq, dk, dv), bf16, layout of q.
+
+    ``o`` and ``lse`` are the forward's outputs.  The workspace (the per-row
+    <dO, O>) is allocated with torch.  Results are bitwise reproducible whether or
+    not ``deterministic`` is set."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _need(t, n)
+    _need(lse, "lse", torch.float32)
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if cu_seqlens is None:
+        B, N, H, _ = q.shape
+        total, cu_ptr = B * N, None
+    else:
+        _need(cu_seqlens, "cu_seqlens", torch.int32)
+        B, H, N = cu_seqlens.numel() - 1, q.shape[1], int(max_seqlen)
+        total, cu_ptr = q.shape[0], cu_seqlens.data_ptr()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws_bytes = lib.attn_bwd_workspace_size(B, H, N, d, total, int(bool(deterministic)))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                          int(bool(causal)), float(scale), cu_ptr, int(bool(deterministic)),
+                          ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    _check(st)
+    return dq, dk, dv
+
+
 def get_device_status(stream: Optional[torch.cuda.Stream] = None) -> None:
     """Synchronises the stream; raises AttnError if a kernel recorded an error."""
     _check(load_library().attn_get_device_status(_stream_ptr(stream)))

@@ -16,8 +16,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libattn.so")
-SOURCES = ["attn_api.cu", "attn_fwd_sm100.cu", "selftest_sm100.cu", "attn_noalloc.cu"]
-HEADERS = ["attn_fwd_sm100.h", "sm100_ptx.cuh"]
+SOURCES = ["attn_api.cu", "attn_fwd_sm100.cu", "attn_bwd_sm100.cu", "selftest_sm100.cu",
+           "attn_noalloc.cu"]
+HEADERS = ["attn_fwd_sm100.h", "attn_bwd_sm100.h", "sm100_ptx.cuh", "exp2_poly.h"]
 PUBLIC_HEADERS = [os.path.join(ROOT, "include", h) for h in ("attn.h", "attn_selftest.h")]
 NVCC = os.environ.get("NVCC", "nvcc")
 # Extra nvcc flags (e.g. -DATTN_POLY_PAIRS_PER_8=4 to change the MUFU/FMA exp split).

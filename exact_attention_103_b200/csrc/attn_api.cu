@@ -11,6 +11,7 @@
 
 #include "../../include/attn.h"
 #include "attn_fwd_sm100.h"
+#include "attn_bwd_sm100.h"
 
 namespace {
 
@@ -226,13 +227,81 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
   return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, hint, opts, stream);
 }
 
-attn_status_t attn_bwd(const void*, const void*, const void*, const void*, const float*,
-                       const void*, void*, void*, void*, int, int, int, int, int, float,
-                       const int32_t*, int, void*, size_t, attn_stream_t) {
-  return fail(ATTN_ERR_UNSUPPORTED, "attn_bwd is not provided by this build");
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                       int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
+                       int deterministic, void* workspace, size_t workspace_bytes,
+                       attn_stream_t stream) {
+  (void)deterministic;  // every call is deterministic: no atomic accumulation
+  if (B < 0 || H <= 0 || N < 0) return fail(ATTN_ERR_INVALID_ARG, "B=%d H=%d N=%d", B, H, N);
+  if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (!(std::isfinite(scale) && scale > 0.f)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (B == 0 || N == 0) return ATTN_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv)
+    return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+    return fail(ATTN_ERR_INVALID_ARG, "tensors must be 16-byte aligned (lse 4-byte)");
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen && (B > kMaxVarlenB || N > kMaxVarlenN))
+    return fail(ATTN_ERR_UNSUPPORTED, "varlen supports B <= %d and N <= %d", kMaxVarlenB, kMaxVarlenN);
+  const int64_t ntiles = (static_cast<int64_t>(N) + 127) / 128;
+  const int64_t grid = static_cast<int64_t>(B) * ntiles * H;
+  const int64_t dense_tokens = static_cast<int64_t>(B) * N;
+  if (grid > INT32_MAX / 2 || dense_tokens > INT32_MAX)
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for 32-bit tile indexing");
+  DeviceState* dev = nullptr;
+  attn_status_t st = device_state(&dev);
+  if (st != ATTN_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  int64_t total = dense_tokens;
+  if (varlen) {
+    int32_t t = 0;
+    cudaError_t e = cudaMemcpyAsync(&t, cu_seqlens + B, sizeof(int32_t), cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return cuda_fail(e, "reading cu_seqlens[B]");
+    total = t;
+    if (total < 0 || total > dense_tokens)
+      return fail(ATTN_ERR_INVALID_ARG, "packed token count %lld outside [0, B*N]", (long long)total);
+    if (total == 0) return ATTN_OK;
+  }
+  const size_t need = attn_bwd_workspace_size(B, H, N, d, static_cast<int>(total), deterministic);
+  if (workspace_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 256))))
+    return fail(ATTN_ERR_WORKSPACE, "workspace of %zu bytes (256-byte aligned) needed", need);
+  attn::BwdLaunch a;
+  std::memset(&a, 0, sizeof(a));
+  if (!make_map(&a.tm_q, q, total, H, d) || !make_map(&a.tm_k, k, total, H, d) ||
+      !make_map(&a.tm_v, v, total, H, d) || !make_map(&a.tm_do, dout, total, H, d))
+    return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled rejected the Q/K/V/dO views");
+  a.p.lse = lse;
+  a.p.dpre = static_cast<float*>(workspace);
+  a.p.dq = static_cast<__nv_bfloat16*>(dq);
+  a.p.dk = static_cast<__nv_bfloat16*>(dk);
+  a.p.dv = static_cast<__nv_bfloat16*>(dv);
+  a.p.cu_seqlens = cu_seqlens;
+  a.p.B = B;
+  a.p.H = H;
+  a.p.N = N;
+  a.p.total = static_cast<int>(total);
+  a.p.ntiles = static_cast<int>(ntiles);
+  a.p.scale = scale;
+  a.p.scale_log2 = scale * 1.4426950408889634f;
+  a.p.err = dev->err;
+  a.p.timeout_ns = kDefaultTimeoutNs;
+  a.grid = static_cast<int>(grid);
+  const cudaError_t e = attn::launch_bwd(a, o, dout, d, causal ? 1 : 0, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+  return ATTN_OK;
 }
 
-size_t attn_bwd_workspace_size(int, int, int, int, int, int) { return 0; }
+size_t attn_bwd_workspace_size(int B, int H, int N, int d, int total_tokens, int deterministic) {
+  (void)N;
+  (void)d;
+  (void)deterministic;
+  if (B <= 0 || H <= 0 || total_tokens <= 0) return 0;
+  const size_t bytes = static_cast<size_t>(total_tokens) * static_cast<size_t>(H) * sizeof(float);
+  return (bytes + 255) / 256 * 256;
+}
 
 attn_status_t attn_get_device_status(attn_stream_t stream) {
   DeviceState* dev = nullptr;

@@ -1,0 +1,627 @@
+// attn_bwd_sm100.cu -- backward pass of exact attention for B200 (sm_100a).
+//
+// The pages say only that the backward recomputes P instead of storing it
+// ("FlashAttention 1-4 详解", 总结 table, 反向传播重计算; "FlashAttention V4
+// deep-dive" section 3.3: P and other intermediates kept in TMEM).  With
+// P_ij = exp(scale*<q_i,k_j> - LSE_i), D_i = <dO_i, O_i>, dP = dO V^T and
+// dS = P o (dP - D) (the textbook backward), three kernels run in order:
+//   bwd_pre_kernel   D_i for every (row, head)                (fp32, workspace)
+//   bwd_dkdv_kernel  one CTA per 128-key tile: loops over query tiles i and
+//                    accumulates dV += P^T dO_i and dK += scale dS^T Q_i in TMEM
+//   bwd_dq_kernel    one CTA per 128-query tile: loops over key tiles j and
+//                    accumulates dQ += scale dS K_j in TMEM
+// Computing dQ in its own kernel recomputes S and dP once more but needs no
+// atomic accumulation, so every result is bitwise reproducible run to run.
+//
+// Both main kernels: warps 0-7 elementwise work (warp w owns TMEM lanes
+// 32(w%4)..+31, one row per thread, and columns 64*(w/4)..+63 of each 128-column
+// tile), warp 8 TMA producer, warp 9 TMEM owner and MMA issuer (whole warp, one
+// elected lane issues).  Every wait is bounded as in the forward kernel.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "attn_bwd_sm100.h"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kTile = 128;  // rows of every tile (keys or queries)
+constexpr float kLog2e = 1.4426950408889634f;
+
+__host__ __device__ constexpr int timeout_code(int site) { return 4 | (site << 8); }
+enum BwdSite { kSiteKv = 32, kSiteStageFull, kSiteStageEmpty, kSiteS, kSiteP, kSiteDs, kSiteAcc,
+               kSiteDrain };
+
+template <int D>
+struct BwdLayout {
+  static constexpr int TILE = kTile * D * 2;
+  static constexpr int CHUNK = kTile * 128;
+  // smem: two resident tiles (A0, A1), then two ring stages of two tiles each,
+  // then per-stage vectors (128 LSE + 128 D floats), barriers, misc.
+  static constexpr int A0_OFF = 0;
+  static constexpr int A1_OFF = TILE;
+  static constexpr int STAGE_OFF = 2 * TILE;
+  static constexpr int NSTAGE = 2;
+  static constexpr int VEC_OFF = STAGE_OFF + NSTAGE * 2 * TILE;
+  static constexpr int BAR_OFF = VEC_OFF + NSTAGE * 2 * kTile * 4;
+  // barrier indices
+  static constexpr int B_RES = 0, B_FULL = 1, B_EMPTY = 3, B_S = 5, B_P = 6, B_DS = 7, B_ACC = 8,
+                       B_DRAIN = 9, NBARS = 10;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int SMEM = MISC_OFF + 64;
+  // TMEM columns: region A (S^T or S, then packed P^T), region B (dP^T or dP,
+  // then packed dS), accumulators.
+  static constexpr int TM_A = 0, TM_B = 128, TM_ACC0 = 256, TM_ACC1 = 256 + D;
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+__device__ __forceinline__ int64_t vec_index(const BwdParams& p, int b, int h, int seq_start,
+                                             int row) {
+  return p.cu_seqlens == nullptr ? (static_cast<int64_t>(b) * p.H + h) * p.N + row
+                                 : static_cast<int64_t>(h) * p.total + seq_start + row;
+}
+
+// Packed bf16 columns of a thread's 64-column half live in the first 32 TMEM
+// columns of that half (so the two halves never write into each other's scores);
+// the K-step kk of an MMA that reads them as its A operand starts here:
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
+
+// Block -> (sequence, head, tile) in longest-first order: for the key-tile
+// kernel (causal) small tile indices have the most query tiles; for the
+// query-tile kernel large indices have the most key tiles.
+struct BwdItem {
+  int b, h, tile, seq_start, L;
+};
+__device__ __forceinline__ bool decode_block(const BwdParams& p, bool key_tiles, bool causal,
+                                             BwdItem& it) {
+  const int nbh = p.B * p.H;
+  const int idx = blockIdx.x;
+  const int rank = idx / nbh, bh = idx - rank * nbh;
+  it.b = bh / p.H;
+  it.h = bh - it.b * p.H;
+  it.tile = (causal && !key_tiles) ? p.ntiles - 1 - rank : rank;
+  if (p.cu_seqlens == nullptr) {
+    it.seq_start = it.b * p.N;
+    it.L = p.N;
+  } else {
+    it.seq_start = __ldg(p.cu_seqlens + it.b);
+    it.L = __ldg(p.cu_seqlens + it.b + 1) - it.seq_start;
+  }
+  return it.tile * kTile < it.L;
+}
+
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+// Stores a thread's half row (D/2 columns) of a TMEM accumulator as bf16, times mul.
+template <int D>
+__device__ __forceinline__ void store_half_row(uint32_t t_acc, __nv_bfloat16* dst, float mul,
+                                               bool store) {
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) {
+    uint32_t v[32];
+    tmem_ld_x32(t_acc + 32 * c, v);
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      w[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+    if (store) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    }
+  }
+}
+
+// Shared set-up of both main kernels: barriers, TMEM (512 columns), abort flag.
+template <int D>
+__device__ __forceinline__ uint32_t bwd_setup(uint8_t* smem, uint32_t sb, int warp) {
+  using Lay = BwdLayout<D>;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+  if (threadIdx.x == 0) {
+    auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
+    mbar_init(bar(Lay::B_RES), 1);
+    for (int s = 0; s < Lay::NSTAGE; ++s) {
+      mbar_init(bar(Lay::B_FULL + s), 1);
+      mbar_init(bar(Lay::B_EMPTY + s), 1);
+    }
+    mbar_init(bar(Lay::B_S), 1);
+    mbar_init(bar(Lay::B_P), 8);
+    mbar_init(bar(Lay::B_DS), 8);
+    mbar_init(bar(Lay::B_ACC), 1);
+    mbar_init(bar(Lay::B_DRAIN), 1);
+    misc[1] = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(sb + Lay::MISC_OFF, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return misc[0];
+}
+
+// Arrive once per warp after this thread's TMEM stores are complete.
+__device__ __forceinline__ void warp_release(uint32_t bar, int lane) {
+  tmem_st_wait();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
+// ---------------------------------------------------------------------- D_i
+__global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                               const __nv_bfloat16* __restrict__ dout, BwdParams p, int d) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t units = static_cast<int64_t>(p.total) * p.H;
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       u < units; u += warps) {
+    const int64_t tok = u / p.H;
+    const int h = static_cast<int>(u - tok * p.H);
+    const __nv_bfloat16* orow = o + u * d;
+    const __nv_bfloat16* drow = dout + u * d;
+    float acc = 0.f;
+    for (int c = lane * 2; c < d; c += 64) {
+      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(orow + c);
+      const __nv_bfloat162 g = *reinterpret_cast<const __nv_bfloat162*>(drow + c);
+      acc = fmaf(__bfloat162float(a.x), __bfloat162float(g.x), acc);
+      acc = fmaf(__bfloat162float(a.y), __bfloat162float(g.y), acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      int64_t idx;
+      if (p.cu_seqlens == nullptr) {
+        const int b = static_cast<int>(tok / p.N);
+        idx = (static_cast<int64_t>(b) * p.H + h) * p.N + (tok - static_cast<int64_t>(b) * p.N);
+      } else {
+        idx = static_cast<int64_t>(h) * p.total + tok;
+      }
+      p.dpre[idx] = acc;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dK, dV
+// CTA: key tile j of (b, h).  Resident: K_j (A0), V_j (A1).  Ring: (Q_i, dO_i).
+// Per query tile i:  S^T = K_j Q_i^T (TMEM A), dP^T = V_j dO_i^T (TMEM B);
+//   P^T = exp2(scale*log2e*S^T - LSE2_i) (causal: zero where query < key) -> A;
+//   dV += P^T dO_i;  dS^T = P^T o (dP^T - D_i) -> B;  dK += dS^T Q_i.
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  using Lay = BwdLayout<D>;
+  BwdItem it;
+  if (!decode_block(p, true, CAUSAL, it)) return;  // uniform for the CTA
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t tmem = bwd_setup<D>(smem, sb, warp);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+  WaitCtl wc;
+  wc.abort = reinterpret_cast<volatile uint32_t*>(misc + 1);
+  wc.err = p.err;
+  wc.limit_ns = p.timeout_ns;
+
+  const int j = it.tile;
+  const int ntiles = ceil_div(it.L, kTile);
+  const int i_first = CAUSAL ? j : 0;
+  const int nq = ntiles - i_first;
+  float* vec = reinterpret_cast<float*>(smem + Lay::VEC_OFF);
+
+  if (warp < 8) {
+    // ---------------------------------------------------- elementwise work
+    const int hf = warp >> 2, wq = warp & 3;
+    const int r = wq * 32 + lane;  // key row within the tile
+    const int key = j * kTile + r;
+    const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tA = tmem + lane_bits + Lay::TM_A + 64 * hf;
+    const uint32_t tB = tmem + lane_bits + Lay::TM_B + 64 * hf;
+    const float sl = p.scale_log2;
+    uint32_t s_phase = 0;
+    bool ok = true;
+    for (int n = 0; n < nq && ok; ++n) {
+      const int i = i_first + n, st = n & 1;
+      const float* lse2 = vec + st * 2 * kTile + 64 * hf;
+      const float* dd = lse2 + kTile;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_S), s_phase, wc, timeout_code(kSiteS)));
+      if (!ok) break;
+      s_phase ^= 1u;
+      tc_fence_after();
+      uint32_t sv[64];
+      tmem_ld_x64(tA, sv);
+      // P^T for this thread's 64 query columns (causal diagonal tile: a query
+      // sees the key only if query >= key; rows past the sequence have LSE2 = +inf).
+      const int lim = (CAUSAL && i == j) ? r - 64 * hf : -1;  // columns < lim are masked
+      float pv[64];
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float e = fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lse2[c]));
+        pv[c] = (c < lim) ? 0.f : e;
+      }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+      tmem_st_x32(tA, pk);
+      warp_release(bar(Lay::B_P), lane);
+      // dS^T = P^T o (dP^T - D), in two 32-column halves to bound registers.
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t dv[32];
+        tmem_ld_x32(tB + 32 * q2, dv);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int c0 = 32 * q2 + 2 * c;
+          pk[16 * q2 + c] = pack_bf16x2(pv[c0] * (__uint_as_float(dv[2 * c]) - dd[c0]),
+                                        pv[c0 + 1] * (__uint_as_float(dv[2 * c + 1]) - dd[c0 + 1]));
+        }
+      }
+      tmem_st_x32(tB, pk);
+      warp_release(bar(Lay::B_DS), lane);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_ACC), 0, wc, timeout_code(kSiteAcc)));
+    if (ok) {
+      tc_fence_after();
+      const bool store = key < it.L;
+      const int64_t row = (static_cast<int64_t>(it.seq_start + key) * p.H + it.h) * D + (D / 2) * hf;
+      const uint32_t t_dv = tmem + lane_bits + Lay::TM_ACC0 + (D / 2) * hf;
+      const uint32_t t_dk = tmem + lane_bits + Lay::TM_ACC1 + (D / 2) * hf;
+      store_half_row<D>(t_dv, p.dv + row, 1.f, store);
+      store_half_row<D>(t_dk, p.dk + row, p.scale, store);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    const uint64_t pol_res = l2_policy_evict_first();
+    const uint64_t pol_ring = l2_policy_evict_last();
+    if (elect_one()) {
+      mbar_arrive_expect_tx(bar(Lay::B_RES), 2 * Lay::TILE);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(sb + Lay::A0_OFF + c * Lay::CHUNK, &tm_k, bar(Lay::B_RES), c * 64, it.h,
+                    it.seq_start + j * kTile, pol_res);
+        tma_load_3d(sb + Lay::A1_OFF + c * Lay::CHUNK, &tm_v, bar(Lay::B_RES), c * 64, it.h,
+                    it.seq_start + j * kTile, pol_res);
+      }
+    }
+    __syncwarp();
+    bool ok = true;
+    for (int n = 0; n < nq && ok; ++n) {
+      const int i = i_first + n, st = n & 1;
+      if (n >= Lay::NSTAGE) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_EMPTY + st), ((n >> 1) - 1) & 1u, wc,
+                                               timeout_code(kSiteStageEmpty)));
+        if (!ok) break;
+      }
+      // Per-query vectors of this tile: LSE in log2 units (+inf past the
+      // sequence, so P = 0 there) and D.
+      float* v = vec + st * 2 * kTile;
+      for (int rr = lane; rr < kTile; rr += 32) {
+        const int qrow = i * kTile + rr;
+        const bool in = qrow < it.L;
+        const int64_t vi = vec_index(p, it.b, it.h, it.seq_start, in ? qrow : 0);
+        v[rr] = in ? __ldg(p.lse + vi) * kLog2e : INFINITY;
+        v[kTile + rr] = in ? __ldg(p.dpre + vi) : 0.f;
+      }
+      __threadfence_block();
+      __syncwarp();
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(Lay::B_FULL + st), 2 * Lay::TILE);
+        const uint32_t base = sb + Lay::STAGE_OFF + st * 2 * Lay::TILE;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(base + c * Lay::CHUNK, &tm_q, bar(Lay::B_FULL + st), c * 64, it.h,
+                      it.seq_start + i * kTile, pol_ring);
+          tma_load_3d(base + Lay::TILE + c * Lay::CHUNK, &tm_do, bar(Lay::B_FULL + st), c * 64, it.h,
+                      it.seq_start + i * kTile, pol_ring);
+        }
+      }
+      __syncwarp();
+    }
+    // Drain: copies still in flight must land before the CTA exits.
+    drain_wait(bar(Lay::B_RES), 0u, p.timeout_ns);
+    for (int n = (nq > Lay::NSTAGE ? nq - Lay::NSTAGE : 0); n < nq; ++n)
+      drain_wait(bar(Lay::B_FULL + (n & 1)), (n >> 1) & 1u, p.timeout_ns);
+  } else {
+    // ---------------------------------------------------------------- MMA
+    constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0, 0);
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(kTile, D, 0, 1);
+    const uint32_t tA = tmem + Lay::TM_A, tB = tmem + Lay::TM_B;
+    const uint32_t tdV = tmem + Lay::TM_ACC0, tdK = tmem + Lay::TM_ACC1;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_RES), 0, wc, timeout_code(kSiteKv)));
+    uint32_t p_phase = 0, ds_phase = 0;
+    for (int n = 0; n < nq && ok; ++n) {
+      const int st = n & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL + st), (n >> 1) & 1u, wc,
+                                             timeout_code(kSiteStageFull)));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t qb = sb + Lay::STAGE_OFF + st * 2 * Lay::TILE, dob = qb + Lay::TILE;
+      // S^T = K Q^T and dP^T = V dO^T (A and B K-major from shared memory).
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+        if (elect_one())
+          mma_ss(tA, sdesc_sw128(sb + Lay::A0_OFF + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        __syncwarp();
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+        if (elect_one())
+          mma_ss(tB, sdesc_sw128(sb + Lay::A1_OFF + off, 16, 1024), sdesc_sw128(dob + off, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        __syncwarp();
+      }
+      if (elect_one()) tc_commit(bar(Lay::B_S));
+      __syncwarp();
+      // dV += P^T dO (A = P^T from TMEM, B = dO MN-major).
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_P), p_phase, wc, timeout_code(kSiteP)));
+      if (!ok) break;
+      p_phase ^= 1u;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) {
+        if (elect_one())
+          mma_ts(tdV, tA + packed_col(kk), sdesc_sw128(dob + kk * 2048, Lay::CHUNK, 1024), idesc_acc,
+                 (n > 0 || kk > 0) ? 1u : 0u);
+        __syncwarp();
+      }
+      // dK += dS^T Q (A = dS^T from TMEM, B = Q MN-major); scale applied at the end.
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DS), ds_phase, wc, timeout_code(kSiteDs)));
+      if (!ok) break;
+      ds_phase ^= 1u;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) {
+        if (elect_one())
+          mma_ts(tdK, tB + packed_col(kk), sdesc_sw128(qb + kk * 2048, Lay::CHUNK, 1024), idesc_acc,
+                 (n > 0 || kk > 0) ? 1u : 0u);
+        __syncwarp();
+      }
+      if (elect_one()) tc_commit(bar(Lay::B_EMPTY + st));
+      __syncwarp();
+    }
+    if (elect_one()) {
+      if (ok) tc_commit(bar(Lay::B_ACC));
+      tc_commit(bar(Lay::B_DRAIN));
+    }
+    __syncwarp();
+    if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, p.timeout_ns)) && lane == 0 && p.err)
+      atomicCAS(p.err, 0, timeout_code(kSiteDrain));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// ----------------------------------------------------------------------- dQ
+// CTA: query tile i of (b, h).  Resident: Q_i (A0), dO_i (A1).  Ring: (K_j, V_j).
+// Per key tile j:  S = Q_i K_j^T (TMEM A), dP = dO_i V_j^T (TMEM B);
+//   P = exp2(scale*log2e*S - LSE2_row) (causal: zero where key > query);
+//   dS = P o (dP - D_row) -> B;  dQ += dS K_j.  dQ is scaled at the end.
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdParams p) {
+  using Lay = BwdLayout<D>;
+  BwdItem it;
+  if (!decode_block(p, false, CAUSAL, it)) return;  // uniform for the CTA
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t tmem = bwd_setup<D>(smem, sb, warp);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+  WaitCtl wc;
+  wc.abort = reinterpret_cast<volatile uint32_t*>(misc + 1);
+  wc.err = p.err;
+  wc.limit_ns = p.timeout_ns;
+
+  const int i = it.tile;
+  const int ntiles = ceil_div(it.L, kTile);
+  const int nk = CAUSAL ? (i + 1 < ntiles ? i + 1 : ntiles) : ntiles;
+
+  if (warp < 8) {
+    const int hf = warp >> 2, wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const int q_row = i * kTile + r;
+    const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tA = tmem + lane_bits + Lay::TM_A + 64 * hf;
+    const uint32_t tB = tmem + lane_bits + Lay::TM_B + 64 * hf;
+    const float sl = p.scale_log2;
+    const bool in = q_row < it.L;
+    const int64_t vi = vec_index(p, it.b, it.h, it.seq_start, in ? q_row : 0);
+    const float lse2 = in ? __ldg(p.lse + vi) * kLog2e : INFINITY;
+    const float dd = in ? __ldg(p.dpre + vi) : 0.f;
+    uint32_t s_phase = 0;
+    bool ok = true;
+    for (int j = 0; j < nk && ok; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_S), s_phase, wc, timeout_code(kSiteS)));
+      if (!ok) break;
+      s_phase ^= 1u;
+      tc_fence_after();
+      uint32_t sv[64];
+      tmem_ld_x64(tA, sv);
+      // keys visible to this row: key < L and (causal) key <= q_row
+      const int kb = j * kTile + 64 * hf;
+      int lim = it.L - kb;
+      if (CAUSAL && q_row - kb + 1 < lim) lim = q_row - kb + 1;
+      float pv[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float e = fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lse2));
+        pv[c] = (c < lim) ? e : 0.f;
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t dv[32];
+        tmem_ld_x32(tB + 32 * q2, dv);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int c0 = 32 * q2 + 2 * c;
+          pk[16 * q2 + c] = pack_bf16x2(pv[c0] * (__uint_as_float(dv[2 * c]) - dd),
+                                        pv[c0 + 1] * (__uint_as_float(dv[2 * c + 1]) - dd));
+        }
+      }
+      tmem_st_x32(tB, pk);
+      warp_release(bar(Lay::B_DS), lane);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_ACC), 0, wc, timeout_code(kSiteAcc)));
+    if (ok) {
+      tc_fence_after();
+      const int64_t row = (static_cast<int64_t>(it.seq_start + q_row) * p.H + it.h) * D + (D / 2) * hf;
+      store_half_row<D>(tmem + lane_bits + Lay::TM_ACC0 + (D / 2) * hf, p.dq + row, p.scale, in);
+    }
+  } else if (warp == 8) {
+    const uint64_t pol_res = l2_policy_evict_first();
+    const uint64_t pol_ring = l2_policy_evict_last();
+    if (elect_one()) {
+      mbar_arrive_expect_tx(bar(Lay::B_RES), 2 * Lay::TILE);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(sb + Lay::A0_OFF + c * Lay::CHUNK, &tm_q, bar(Lay::B_RES), c * 64, it.h,
+                    it.seq_start + i * kTile, pol_res);
+        tma_load_3d(sb + Lay::A1_OFF + c * Lay::CHUNK, &tm_do, bar(Lay::B_RES), c * 64, it.h,
+                    it.seq_start + i * kTile, pol_res);
+      }
+    }
+    __syncwarp();
+    bool ok = true;
+    for (int j = 0; j < nk && ok; ++j) {
+      const int st = j & 1;
+      if (j >= Lay::NSTAGE) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_EMPTY + st), ((j >> 1) - 1) & 1u, wc,
+                                               timeout_code(kSiteStageEmpty)));
+        if (!ok) break;
+      }
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(Lay::B_FULL + st), 2 * Lay::TILE);
+        const uint32_t base = sb + Lay::STAGE_OFF + st * 2 * Lay::TILE;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(base + c * Lay::CHUNK, &tm_k, bar(Lay::B_FULL + st), c * 64, it.h,
+                      it.seq_start + j * kTile, pol_ring);
+          tma_load_3d(base + Lay::TILE + c * Lay::CHUNK, &tm_v, bar(Lay::B_FULL + st), c * 64, it.h,
+                      it.seq_start + j * kTile, pol_ring);
+        }
+      }
+      __syncwarp();
+    }
+    drain_wait(bar(Lay::B_RES), 0u, p.timeout_ns);
+    for (int j = (nk > Lay::NSTAGE ? nk - Lay::NSTAGE : 0); j < nk; ++j)
+      drain_wait(bar(Lay::B_FULL + (j & 1)), (j >> 1) & 1u, p.timeout_ns);
+  } else {
+    constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0, 0);
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(kTile, D, 0, 1);
+    const uint32_t tA = tmem + Lay::TM_A, tB = tmem + Lay::TM_B, tdQ = tmem + Lay::TM_ACC0;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_RES), 0, wc, timeout_code(kSiteKv)));
+    uint32_t ds_phase = 0;
+    for (int j = 0; j < nk && ok; ++j) {
+      const int st = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL + st), (j >> 1) & 1u, wc,
+                                             timeout_code(kSiteStageFull)));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t kb = sb + Lay::STAGE_OFF + st * 2 * Lay::TILE, vb = kb + Lay::TILE;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+        if (elect_one())
+          mma_ss(tA, sdesc_sw128(sb + Lay::A0_OFF + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        __syncwarp();
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+        if (elect_one())
+          mma_ss(tB, sdesc_sw128(sb + Lay::A1_OFF + off, 16, 1024), sdesc_sw128(vb + off, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        __syncwarp();
+      }
+      if (elect_one()) tc_commit(bar(Lay::B_S));
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DS), ds_phase, wc, timeout_code(kSiteDs)));
+      if (!ok) break;
+      ds_phase ^= 1u;
+      tc_fence_after();
+      // dQ += dS K (A = dS from TMEM, B = K MN-major).
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) {
+        if (elect_one())
+          mma_ts(tdQ, tB + packed_col(kk), sdesc_sw128(kb + kk * 2048, Lay::CHUNK, 1024), idesc_acc,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        __syncwarp();
+      }
+      if (elect_one()) tc_commit(bar(Lay::B_EMPTY + st));
+      __syncwarp();
+    }
+    if (elect_one()) {
+      if (ok) tc_commit(bar(Lay::B_ACC));
+      tc_commit(bar(Lay::B_DRAIN));
+    }
+    __syncwarp();
+    if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, p.timeout_ns)) && lane == 0 && p.err)
+      atomicCAS(p.err, 0, timeout_code(kSiteDrain));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_main(const BwdLaunch& a, cudaStream_t st) {
+  const int smem = 1024 + BwdLayout<D>::SMEM;
+  auto k1 = bwd_dkdv_kernel<D, CAUSAL>;
+  auto k2 = bwd_dq_kernel<D, CAUSAL>;
+  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  k1<<<a.grid, kThreads, smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k2<<<a.grid, kThreads, smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const BwdLaunch& a, const void* o, const void* dout, int D, int causal,
+                       cudaStream_t st) {
+  const int64_t units = static_cast<int64_t>(a.p.total) * a.p.H;
+  int blocks = static_cast<int>((units + 7) / 8);
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  bwd_pre_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
+                                          static_cast<const __nv_bfloat16*>(dout), a.p, D);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (D == 128) return causal ? launch_main<128, true>(a, st) : launch_main<128, false>(a, st);
+  return causal ? launch_main<64, true>(a, st) : launch_main<64, false>(a, st);
+}
+
+}  // namespace attn

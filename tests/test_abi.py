@@ -91,7 +91,19 @@ def test_bad_options(lib):
     assert st == ea.ATTN_ERR_INVALID_ARG
 
 
-def test_backward_not_provided_yet(lib):
-    st = lib.attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0,
-                      0.1, None, 0, None, 0, None)
-    assert st == ea.ATTN_ERR_UNSUPPORTED
+def test_backward_argument_checks(lib):
+    def bwd(d=128, scale=0.1, B=1, dq=FAKE):
+        return lib.attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, dq, FAKE, FAKE, B, 1, 128, d, 0,
+                            scale, None, 0, None, 0, None)
+    assert bwd(d=96) == ea.ATTN_ERR_UNSUPPORTED
+    assert bwd(scale=0.0) == ea.ATTN_ERR_INVALID_ARG
+    assert bwd(dq=None) == ea.ATTN_ERR_INVALID_ARG
+    assert bwd(dq=FAKE + 4) == ea.ATTN_ERR_INVALID_ARG
+    assert bwd(B=0) == ea.ATTN_OK
+
+
+def test_backward_workspace_size(lib):
+    # one fp32 per (token, head), rounded up to 256 bytes
+    assert lib.attn_bwd_workspace_size(2, 16, 8192, 128, 2 * 8192, 0) == 2 * 8192 * 16 * 4
+    assert lib.attn_bwd_workspace_size(1, 3, 5, 64, 5, 1) == 256
+    assert lib.attn_bwd_workspace_size(0, 3, 5, 64, 0, 1) == 0
