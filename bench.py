@@ -181,12 +181,18 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's value (NCCL on the GPU; gloo tests pass device="cpu")."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(flops_per_step: float, steps: int, world: int, max_total_ms: float) -> float:
+    """All ranks' FLOPs (each rank runs one replica) over the slowest rank's time."""
+    return world * flops_per_step * steps / (max_total_ms / 1e3) / 1e12
 
 
 def make_inputs(w: ai.Workload, device):
@@ -308,7 +314,7 @@ def run_ours(args, rank, world, local):
     times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(times), world)
     ms_per_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    value = whole_job_tflops(flops, args.steps, world, total_ms)
     achieved = flops / (statistics.mean(times) / 1e3) / 1e12  # per launch, this rank
     peak = peaks["bf16_tflops"]
     clk = clocks.summary()
@@ -406,7 +412,7 @@ def run_bwd(args, rank, world, local):
     ea.get_device_status()
     times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(times), world)
-    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    value = whole_job_tflops(flops, args.steps, world, total_ms)
     achieved = flops / (statistics.mean(times) / 1e3) / 1e12
     if rank == 0:
         cfg = bench_config(w, world)

@@ -174,7 +174,10 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   a.p.err = dev->err;
   a.p.stats = stats;
   a.p.timeout_ns = timeout;
-  a.grid = static_cast<int>(items_bound < dev->sms ? items_bound : dev->sms);
+  // Dense non-causal launches may split their last wave into half items (see the
+  // kernel), so up to twice as many CTAs can be useful there.
+  const int64_t useful = (!varlen && !causal) ? 2 * items_bound : items_bound;
+  a.grid = static_cast<int>(useful < dev->sms ? useful : dev->sms);
   a.smem = attn::fwd_smem_bytes(d, B, static_cast<int>(T256), varlen ? 1 : 0);
   const cudaError_t e = attn::launch_fwd(a, d, causal ? 1 : 0, cs);
   if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");

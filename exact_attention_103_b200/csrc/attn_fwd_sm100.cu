@@ -6,13 +6,11 @@
 // two sub-tiles while the other one's softmax runs ("FlashAttention V4 deep-dive"
 // (pnsm.cn), section 3.1, two Q tiles in ping-pong).
 //
-// Warp roles (576 threads):
-//   warps 0-7   softmax + epilogue of sub-tile 0: warp w owns TMEM lanes
-//               32(w%4)..+31 (one query row per thread) and key columns
-//               64*((w/4)%2)..+63 of every tile, so two threads share each row
-//   warps 8-15  the same for sub-tile 1
-//   warp  16    TMA producer: Q pair, then K_j / V_j tiles into an smem ring
-//   warp  17    TMEM owner and tcgen05.mma issuer (whole warp; one elected lane
+// Warp roles (320 threads):
+//   warps 0-3   softmax + epilogue of sub-tile 0 (one query row per thread)
+//   warps 4-7   softmax + epilogue of sub-tile 1
+//   warp  8     TMA producer: Q pair, then K_j / V_j tiles into an smem ring
+//   warp  9     TMEM owner and tcgen05.mma issuer (whole warp; one elected lane
 //               issues each instruction)
 //
 // Per sub-tile s and key tile j ("FlashAttention 1-4 详解", FlashAttention 1 /
@@ -50,15 +48,16 @@ namespace attn {
 
 namespace {
 
-constexpr int kThreads = 576;
+constexpr int kThreads = 320;
 constexpr int kBM = 128;  // query rows per sub-tile
 constexpr int kBN = 128;  // keys per key tile
 constexpr float kLn2 = 0.693147180559945309f;
 
 // Of every 8 consecutive (even, odd) column pairs of a score row, this many are
 // exponentiated on the FMA pipe by the polynomial below; the rest use MUFU ex2.
+// Measured on B200 (same-box A/B, this kernel): 0 is fastest; 1 costs ~1%, 2 ~4%.
 #ifndef ATTN_POLY_PAIRS_PER_8
-#define ATTN_POLY_PAIRS_PER_8 1
+#define ATTN_POLY_PAIRS_PER_8 0
 #endif
 constexpr int kPolyPairsPer8 = ATTN_POLY_PAIRS_PER_8;
 static_assert(kPolyPairsPer8 >= 0 && kPolyPairsPer8 <= 8, "pairs per 8");
@@ -85,7 +84,7 @@ __device__ __forceinline__ float exp2_poly(float y) {
 __host__ __device__ constexpr int timeout_code(int site) { return 4 | (site << 8); }
 enum WaitSite {
   kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteOFull,
-  kSiteDrain, kSiteBadLen, kSiteXch
+  kSiteDrain, kSiteBadLen
 };
 
 template <int D>
@@ -98,12 +97,18 @@ struct Layout {
   static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE;
   // barrier indices
   static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_OFULL = 6,
-                       B_DRAIN = 8, B_XCH = 9, B_KVFULL = 17, B_KVEMPTY = 17 + NSTAGE;
-  static constexpr int NBARS = 17 + 2 * NSTAGE;
+                       B_DRAIN = 8, B_KVFULL = 9, B_KVEMPTY = 9 + NSTAGE;
+  static constexpr int NBARS = 9 + 2 * NSTAGE;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-  static constexpr int EXCH_OFF = MISC_OFF + 64;          // float [2][2][128][2]
-  static constexpr int TABLE_OFF = EXCH_OFF + 2 * 2 * 128 * 2 * 4;
+  static constexpr int TABLE_OFF = MISC_OFF + 64;
   static constexpr int TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
+};
+
+// A work item: query rows [row_base, row_base + 256) of one (sequence, head) as
+// two 128-row sub-tiles, or only the first sub-tile when `two` is false.
+struct Item {
+  int b, h, seq_start, L, row_base;
+  bool two;
 };
 
 // Work-item decoding shared by every role (all roles walk the same list).
@@ -112,6 +117,8 @@ struct Sched {
   int B, H, N, T;
   const int* order;  // varlen: sequences sorted by tile-pair count, descending
   const int* start;  // varlen: first pair index of bucket t (buckets by t descending)
+  int pairs;         // 256-row items before any split
+  int split;         // dense non-causal: the last `split` pairs become 2*split half items
   int count;         // number of items
 
   __device__ __forceinline__ int item(int k) const {
@@ -119,16 +126,25 @@ struct Sched {
     const int idx = k * G + ((k & 1) ? (G - 1 - c) : c);
     return idx < count ? idx : -1;
   }
-  __device__ __forceinline__ void decode(int idx, int& b, int& t, int& h, int& seq_start,
-                                         int& L) const {
+  // SPLIT: the launch may hold half items (dense non-causal only).
+  template <bool SPLIT>
+  __device__ __forceinline__ Item decode(int idx) const {
+    Item it;
+    int sub = -1;  // >= 0: a half item made of sub-tile `sub` of its pair
+    if (SPLIT && idx >= pairs - split) {
+      const int u = idx - (pairs - split);
+      idx = pairs - split + (u >> 1);
+      sub = u & 1;
+    }
     const int pr = idx / H;
-    h = idx - pr * H;
+    it.h = idx - pr * H;
+    int t;
     if (cu == nullptr) {
       const int tt = pr / B;
       t = T - 1 - tt;
-      b = pr - tt * B;
-      seq_start = b * N;
-      L = N;
+      it.b = pr - tt * B;
+      it.seq_start = it.b * N;
+      it.L = N;
     } else {
       int lo = 0, hi = T - 1;  // smallest t with start[t] <= pr
       while (lo < hi) {
@@ -136,21 +152,26 @@ struct Sched {
         if (start[mid] <= pr) hi = mid; else lo = mid + 1;
       }
       t = lo;
-      b = order[pr - start[lo]];
-      seq_start = __ldg(cu + b);
-      L = __ldg(cu + b + 1) - seq_start;
+      it.b = order[pr - start[lo]];
+      it.seq_start = __ldg(cu + it.b);
+      it.L = __ldg(cu + it.b + 1) - it.seq_start;
     }
+    it.row_base = t * 2 * kBM + ((SPLIT && sub > 0) ? kBM : 0);
+    it.two = !SPLIT || sub < 0;
+    return it;
   }
 };
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// Key tiles sub-tile s of pair t processes (0 when its rows are all past L).
+// Key tiles sub-tile s of an item processes (0 when its rows are all past L, or
+// for the missing second sub-tile of a half item).
 template <bool CAUSAL>
-__device__ __forceinline__ int num_kv_tiles(int t, int s, int L) {
-  const int row0 = t * 2 * kBM + s * kBM;
-  if (row0 >= L) return 0;
-  const int all = ceil_div(L, kBN);
+__device__ __forceinline__ int num_kv_tiles(const Item& it, int s) {
+  if (!CAUSAL && s == 1 && !it.two) return 0;
+  const int row0 = it.row_base + s * kBM;
+  if (row0 >= it.L) return 0;
+  const int all = ceil_div(it.L, kBN);
   if (!CAUSAL) return all;
   const int diag = row0 / kBN + 1;  // tiles up to and including the diagonal
   return diag < all ? diag : all;
@@ -246,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
-  // misc[0] TMEM base, misc[1] abort flag, misc[2] item count
+  // misc[0] TMEM base, misc[1] abort flag, misc[2] number of 256-row items
   int* tab = reinterpret_cast<int*>(smem + Lay::TABLE_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -256,11 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(Lay::B_QEMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Lay::B_SFULL + s), 1);
-      mbar_init(bar(Lay::B_PFULL + s), 8);
+      mbar_init(bar(Lay::B_PFULL + s), 4);
       mbar_init(bar(Lay::B_OFULL + s), 1);
     }
     mbar_init(bar(Lay::B_DRAIN), 1);
-    for (int i = 0; i < 8; ++i) mbar_init(bar(Lay::B_XCH + i), 2);
     for (int i = 0; i < NS; ++i) {
       mbar_init(bar(Lay::B_KVFULL + i), 1);
       mbar_init(bar(Lay::B_KVEMPTY + i), 1);
@@ -268,11 +288,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     misc[1] = 0u;
     fence_barrier_init();
   }
-  if (warp == 17) {
+  if (warp == 9) {
     tmem_alloc(sb + Lay::MISC_OFF, 512);
     tmem_relinquish();
   }
-  if (warp == 16) {
+  if (warp == 8) {
     int count;
     if (p.cu_seqlens == nullptr) {
       count = p.B * p.T * p.H;
@@ -297,56 +317,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   sch.B = p.B; sch.H = p.H; sch.N = p.N; sch.T = p.T;
   sch.order = tab;
   sch.start = tab + p.B + 2 * p.T + 1;
-  sch.count = static_cast<int>(misc[2]);
+  sch.pairs = static_cast<int>(misc[2]);
+  // Dense non-causal items all cost the same: when the last wave would leave
+  // CTAs idle, its pairs are split into 128-row half items so it spreads over
+  // more SMs (a half item runs without a ping-pong partner, but the wave is
+  // shorter).  Causal and varlen items are already longest-first.
+  sch.split = 0;
+  if (!CAUSAL && p.cu_seqlens == nullptr) {
+    const int rem = sch.pairs % static_cast<int>(gridDim.x);
+    if (rem > 0 && 2 * rem <= static_cast<int>(gridDim.x)) sch.split = rem;
+  }
+  sch.count = sch.pairs + sch.split;
   WaitCtl wc;
   wc.abort = reinterpret_cast<volatile uint32_t*>(misc + 1);
   wc.err = p.err;
   wc.limit_ns = p.timeout_ns;
 
-  if (warp < 16) {
+  if (warp < 8) {
     // ------------------------------------------------------------ softmax
-    // Sub-tile s, TMEM lane quarter q (rows 32q..32q+31), column half hf: the two
-    // warps of a (s, q) pair share the rows and split each row's 128 key columns,
-    // exchanging partial row maxima (and, at the end, partial row sums) through
-    // shared memory with a 64-thread named barrier.
-    const int s = warp >> 3, hf = (warp >> 2) & 1, wq = warp & 3;
+    // Sub-tile s = warp / 4; warp w owns TMEM lanes 32(w%4)..+31: one query row per
+    // thread, all 128 key columns of each tile.
+    const int s = warp >> 2, wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t t_s = tmem + lane_bits + (s ? Lay::TM_S1 : Lay::TM_S0);
-    // This half's packed bf16 P columns.  Half 1 writes columns 32..63, which hold
-    // half 0's scores; that is safe because half 1 passes the pair's max exchange
-    // of the tile only after half 0 arrived there, i.e. after half 0's TMEM load.
-    const uint32_t t_p = t_s + 32 * hf;
-    const uint32_t t_o = tmem + lane_bits + (s ? Lay::TM_O1 : Lay::TM_O0) + (D / 2) * hf;
-    // Pair exchange: write a value, arrive (one arrival per warp), wait for the
-    // partner's arrival, read its value.  Slots alternate with the exchange count,
-    // so a slot is rewritten only after the partner has passed the next exchange.
-    const uint32_t xbar = bar(Lay::B_XCH + s * 4 + wq);
-    float* xch = reinterpret_cast<float*>(smem + Lay::EXCH_OFF);
-    uint32_t n_x = 0;
-    auto exchange = [&](float mine, float& theirs) -> bool {
-      float* slot = xch + (((n_x & 1) * 2 + s) * 128 + r) * 2;
-      slot[hf] = mine;
-      __threadfence_block();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xbar);
-      bool okx = mbar_wait(xbar, n_x & 1, wc, timeout_code(kSiteXch));
-      okx = __all_sync(0xffffffffu, okx);
-      theirs = slot[hf ^ 1];
-      ++n_x;
-      return okx;
-    };
+    const uint32_t t_o = tmem + lane_bits + (s ? Lay::TM_O1 : Lay::TM_O0);
     const float sl = p.scale_log2;
     uint32_t s_phase = 0, o_phase = 0;
     unsigned long long n_rescale = 0, n_rowtiles = 0;
     for (int k = 0;; ++k) {
       const int idx = sch.item(k);
       if (idx < 0) break;
-      int b, t, h, seq_start, L;
-      sch.decode(idx, b, t, h, seq_start, L);
-      const int nkv = num_kv_tiles<CAUSAL>(t, s, L);
+      const Item it = sch.template decode<!CAUSAL>(idx);
+      const int b = it.b, h = it.h, seq_start = it.seq_start, L = it.L;
+      const int nkv = num_kv_tiles<CAUSAL>(it, s);
       if (nkv == 0) continue;
-      const int row0 = t * 2 * kBM + s * kBM;
+      const int row0 = it.row_base + s * kBM;
       const int q_row = row0 + r;
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
@@ -356,56 +362,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         s_phase ^= 1u;
         tc_fence_after();
-        uint32_t sv[64];
-        tmem_ld_x64(t_s + 64 * hf, sv);
-        const int kb = j * kBN + 64 * hf;  // key index of this thread's first column
-        if ((CAUSAL && j * kBN + kBN - 1 > row0) || kb + 64 > L) {
-          int lim = L - kb;  // columns [0, lim) hold visible keys for this row
+        uint32_t sv[128];
+        tmem_ld_x128(t_s, sv);
+        const int kb = j * kBN;
+        if ((CAUSAL && kb + kBN - 1 > row0) || kb + kBN > L) {
+          int lim = L - kb;  // keys [kb, kb+lim) are visible to this row
           if (CAUSAL && q_row - kb + 1 < lim) lim = q_row - kb + 1;
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < 128; ++c)
             if (c >= lim) sv[c] = __float_as_uint(-INFINITY);
         }
-        // Partial row maximum over this half: four 3-input max chains and a tree.
+        // Row maximum: four independent 3-input max chains, then a small tree.
         float m4[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           m4[i] = fmax3(__uint_as_float(sv[i]), __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 8]));
 #pragma unroll
-        for (int c = 12; c < 60; c += 8)
+        for (int c = 12; c < 124; c += 8)
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             m4[i] = fmax3(m4[i], __uint_as_float(sv[c + i]), __uint_as_float(sv[c + 4 + i]));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], __uint_as_float(sv[60 + i]));
-        const float mx_half = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-        float mx_other;
-        ok = exchange(mx_half, mx_other);
-        if (!ok) break;
-        const float mx = fmaxf(mx_half, mx_other);
-        const float m_tile = mx * sl;
+        for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], __uint_as_float(sv[124 + i]));
+        const float m_tile = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sl;
         bool need = false;
         float alpha = 1.f;
         if (j == 0) {
           m_ref = m_tile;
         } else {
-          if (hf == 0) ++n_rowtiles;
+          ++n_rowtiles;
           if (m_tile - m_ref > p.tau) {
             need = true;
             alpha = fast_exp2(m_ref - m_tile);
             m_ref = m_tile;
             l *= alpha;
-            if (hf == 0) ++n_rescale;
+            ++n_rescale;
           }
         }
         // P~ = 2^(s*scale*log2e - m_ref): one FMA for the argument, MUFU ex2 or the
-        // FMA-pipe polynomial for the exponential, four partial row sums, then
-        // bf16 packing.
+        // FMA-pipe polynomial for the exponential, partial row sums, bf16 packing.
         const float nm = -m_ref;
-        uint32_t pk[32];
+        uint32_t pk[64];
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < 64; ++c) {
           float a = fmaf(__uint_as_float(sv[2 * c]), sl, nm);
           float e = fmaf(__uint_as_float(sv[2 * c + 1]), sl, nm);
           if ((c & 7) >= 8 - kPolyPairsPer8) {
@@ -420,11 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[c] = pack_bf16x2(a, e);
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        tmem_st_x32(t_p, pk);
+        tmem_st_x64(t_s, pk);
         // O_s is stable here: the commit that signalled S(s, j) also covers PV(s, j-1).
         if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t ov[32];
             tmem_ld_x32(t_o + 32 * c, ov);
 #pragma unroll
@@ -441,21 +441,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      float l_other;
-      ok = exchange(l, l_other);
-      if (!ok) break;
       ok = mbar_wait(bar(Lay::B_OFULL + s), o_phase, wc, timeout_code(kSiteOFull));
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       o_phase ^= 1u;
       tc_fence_after();
-      l += l_other;
       const float inv = 1.f / l;
       const bool store = q_row < L;
-      __nv_bfloat16* dst = p.o + (static_cast<int64_t>(seq_start + q_row) * p.H + h) *
-                                     static_cast<int64_t>(D) + (D / 2) * hf;
+      __nv_bfloat16* dst =
+          p.o + (static_cast<int64_t>(seq_start + q_row) * p.H + h) * static_cast<int64_t>(D);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
         tmem_ld_x32(t_o + 32 * c, ov);
         uint32_t w[16];
@@ -468,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (store && hf == 0) {
+      if (store) {
         const float lse = (m_ref + __log2f(l)) * kLn2;
         int64_t li;
         if (p.cu_seqlens == nullptr)
@@ -482,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       atomicAdd(p.stats, n_rescale);
       atomicAdd(p.stats + 1, n_rowtiles);
     }
-  } else if (warp == 16) {
+  } else if (warp == 8) {
     // ----------------------------------------------------------- producer
     // Whole warp walks the loop and waits; one elected lane issues the copies.
     if (elect_one()) {
@@ -499,9 +495,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int idx = sch.item(k);
       if (idx < 0) break;
-      int b, t, h, seq_start, L;
-      sch.decode(idx, b, t, h, seq_start, L);
-      const int nkv0 = num_kv_tiles<CAUSAL>(t, 0, L), nkv1 = num_kv_tiles<CAUSAL>(t, 1, L);
+      const Item it = sch.template decode<!CAUSAL>(idx);
+      const int h = it.h, seq_start = it.seq_start;
+      const int nkv0 = num_kv_tiles<CAUSAL>(it, 0), nkv1 = num_kv_tiles<CAUSAL>(it, 1);
       const int nkv = nkv0 > nkv1 ? nkv0 : nkv1;
       if (k > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QEMPTY), qe_phase, wc, timeout_code(kSiteQEmpty)));
@@ -515,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(sb + Lay::Q_OFF + s * Lay::TILE + c * Lay::CHUNK, &tm_q, bar(Lay::B_QFULL),
-                        c * 64, h, seq_start + t * 2 * kBM + s * kBM, pol_q);
+                        c * 64, h, seq_start + it.row_base + s * kBM, pol_q);
       }
       __syncwarp();
       ++n_items;
@@ -534,12 +530,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < D / 64; ++c)
               tma_load_3d(sb + Lay::KV_OFF + slot * Lay::TILE + c * Lay::CHUNK, which ? &tm_v : &tm_k,
                           bar(Lay::B_KVFULL + slot), c * 64, h, seq_start + j * kBN, pol_kv);
-            // Warm L2 with the same operand two tiles ahead: when its ring slot frees
-            // up, the copy then hits L2 instead of HBM.
-            if (j + 2 < nkv)
-#pragma unroll
-              for (int c = 0; c < D / 64; ++c)
-                tma_prefetch_l2_3d(which ? &tm_v : &tm_k, c * 64, h, seq_start + (j + 2) * kBN);
           }
           __syncwarp();
           ++n_ld;
@@ -567,9 +557,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int idx = sch.item(k);
       if (idx < 0) break;
-      int b, t, h, seq_start, L;
-      sch.decode(idx, b, t, h, seq_start, L);
-      const int nk0 = num_kv_tiles<CAUSAL>(t, 0, L), nk1 = num_kv_tiles<CAUSAL>(t, 1, L);
+      const Item it = sch.template decode<!CAUSAL>(idx);
+      const int nk0 = num_kv_tiles<CAUSAL>(it, 0), nk1 = num_kv_tiles<CAUSAL>(it, 1);
       const int nkv = nk0 > nk1 ? nk0 : nk1;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QFULL), q_phase, wc, timeout_code(kSiteQFull)));
       if (!ok) break;
@@ -646,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 17) tmem_dealloc(tmem, 512);
+  if (warp == 9) tmem_dealloc(tmem, 512);
 }
 
 template <int D>
