@@ -38,7 +38,8 @@ class FwdOpts(ctypes.Structure):
     _fields_ = [("rescale_threshold", ctypes.c_float),
                 ("stats", ctypes.c_void_p),
                 ("timeout_ns", ctypes.c_uint64),
-                ("total_tokens", ctypes.c_int64)]
+                ("total_tokens", ctypes.c_int64),
+                ("test_fault", ctypes.c_int)]
 
 
 _lib = None
@@ -111,7 +112,8 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         max_seqlen: Optional[int] = None, out: Optional[torch.Tensor] = None,
         lse: Optional[torch.Tensor] = None, rescale_threshold: Optional[float] = None,
         stats: Optional[torch.Tensor] = None, timeout_ns: int = 0,
-        stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+        stream: Optional[torch.cuda.Stream] = None,
+        test_fault: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
     """Exact attention forward on the GPU.
 
     Dense: q, k, v are bf16 ``[B, N, H, d]``; returns O ``[B, N, H, d]`` and LSE
@@ -128,7 +130,7 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     opts = FwdOpts(-1.0 if rescale_threshold is None else float(rescale_threshold),
-                   None if stats is None else stats.data_ptr(), int(timeout_ns), 0)
+                   None if stats is None else stats.data_ptr(), int(timeout_ns), 0, int(test_fault))
     if stats is not None:
         _need(stats, "stats", torch.int64)
     if cu_seqlens is None:

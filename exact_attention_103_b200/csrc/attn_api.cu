@@ -126,7 +126,11 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   float tau = kDefaultTau;
   uint64_t timeout = kDefaultTimeoutNs;
   unsigned long long* stats = nullptr;
+  int test_fault = 0;
   if (opts) {
+    if (opts->test_fault != 0 && opts->test_fault != 1)
+      return fail(ATTN_ERR_INVALID_ARG, "test_fault must be 0 or 1");
+    test_fault = opts->test_fault;
     if (opts->rescale_threshold >= 0.f) tau = opts->rescale_threshold;
     if (!(tau <= 64.f)) return fail(ATTN_ERR_INVALID_ARG, "rescale_threshold must be <= 64");
     if (opts->timeout_ns) timeout = opts->timeout_ns;
@@ -174,6 +178,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   a.p.err = dev->err;
   a.p.stats = stats;
   a.p.timeout_ns = timeout;
+  a.p.test_fault = test_fault;
   // Dense non-causal launches may split their last wave into half items (see the
   // kernel), so up to twice as many CTAs can be useful there.
   const int64_t useful = (!varlen && !causal) ? 2 * items_bound : items_bound;

@@ -335,9 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     }
     // Drain: copies still in flight must land before the CTA exits.
-    drain_wait(bar(Lay::B_RES), 0u, p.timeout_ns);
+    drain_wait(bar(Lay::B_RES), 0u, kDrainLimitNs);
     for (int n = (nq > Lay::NSTAGE ? nq - Lay::NSTAGE : 0); n < nq; ++n)
-      drain_wait(bar(Lay::B_FULL + (n & 1)), (n >> 1) & 1u, p.timeout_ns);
+      drain_wait(bar(Lay::B_FULL + (n & 1)), (n >> 1) & 1u, kDrainLimitNs);
   } else {
     // ---------------------------------------------------------------- MMA
     constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0, 0);
@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(bar(Lay::B_DRAIN));
     }
     __syncwarp();
-    if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, p.timeout_ns)) && lane == 0 && p.err)
+    if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, kDrainLimitNs)) && lane == 0 && p.err)
       atomicCAS(p.err, 0, timeout_code(kSiteDrain));
   }
   tc_fence_before();
@@ -530,9 +530,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
-    drain_wait(bar(Lay::B_RES), 0u, p.timeout_ns);
+    drain_wait(bar(Lay::B_RES), 0u, kDrainLimitNs);
     for (int j = (nk > Lay::NSTAGE ? nk - Lay::NSTAGE : 0); j < nk; ++j)
-      drain_wait(bar(Lay::B_FULL + (j & 1)), (j >> 1) & 1u, p.timeout_ns);
+      drain_wait(bar(Lay::B_FULL + (j & 1)), (j >> 1) & 1u, kDrainLimitNs);
   } else {
     constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0, 0);
     constexpr uint32_t idesc_acc = idesc_bf16_f32(kTile, D, 0, 1);
@@ -584,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(bar(Lay::B_DRAIN));
     }
     __syncwarp();
-    if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, p.timeout_ns)) && lane == 0 && p.err)
+    if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, kDrainLimitNs)) && lane == 0 && p.err)
       atomicCAS(p.err, 0, timeout_code(kSiteDrain));
   }
   tc_fence_before();

@@ -504,7 +504,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         qe_phase ^= 1u;
       }
-      if (elect_one()) {
+      // Failure-path test: the first query tile's copy is never issued, so its
+      // consumers' waits run out.
+      const bool withhold = p.test_fault == 1 && k == 0;
+      if (!withhold && elect_one()) {
         mbar_arrive_expect_tx(bar(Lay::B_QFULL), 2 * Lay::TILE);
 #pragma unroll
         for (int s = 0; s < 2; ++s)
@@ -514,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         c * 64, h, seq_start + it.row_base + s * kBM, pol_q);
       }
       __syncwarp();
-      ++n_items;
+      if (!withhold) ++n_items;
       for (int j = 0; j < nkv && ok; ++j) {
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
@@ -539,8 +542,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Drain: every issued copy must have landed before the CTA may exit.
     const uint32_t first = n_ld > static_cast<uint32_t>(NS) ? n_ld - NS : 0u;
     for (uint32_t n = first; n < n_ld; ++n)
-      drain_wait(bar(Lay::B_KVFULL + n % NS), (n / NS) & 1u, p.timeout_ns);
-    if (n_items > 0) drain_wait(bar(Lay::B_QFULL), (n_items - 1) & 1u, p.timeout_ns);
+      drain_wait(bar(Lay::B_KVFULL + n % NS), (n / NS) & 1u, kDrainLimitNs);
+    if (n_items > 0) drain_wait(bar(Lay::B_QFULL), (n_items - 1) & 1u, kDrainLimitNs);
   } else {
     // ---------------------------------------------------------------- MMA
     // The whole warp walks the loop and waits; one elected lane issues each MMA
@@ -628,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Drain: every MMA issued by this warp completes before TMEM is freed.
     if (elect_one()) tc_commit(bar(Lay::B_DRAIN));
     __syncwarp();
-    if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, p.timeout_ns)) && lane == 0 && p.err)
+    if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, kDrainLimitNs)) && lane == 0 && p.err)
       atomicCAS(p.err, 0, timeout_code(kSiteDrain));
   }
 

@@ -20,6 +20,7 @@ struct FwdParams {
   int* err;              // device error word
   unsigned long long* stats;  // optional [rescaled rows, row-tiles]
   uint64_t timeout_ns;   // limit of every internal wait
+  int test_fault;        // 1: withhold the first Q copy (failure-path tests only)
 };
 
 struct FwdLaunch {

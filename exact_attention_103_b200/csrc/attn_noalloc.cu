@@ -132,6 +132,7 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
   a.p.err = dev->scratch;
   a.p.stats = nullptr;
   a.p.timeout_ns = 2000000000ull;
+  a.p.test_fault = 0;
   const int64_t useful = (!varlen && !causal) ? 2 * items_bound : items_bound;
   a.grid = static_cast<int>(useful < dev->sms ? useful : dev->sms);
   a.smem = attn::fwd_smem_bytes(d, B, static_cast<int>(T256), varlen ? 1 : 0);

@@ -86,6 +86,12 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// Limit of the waits with which a CTA drains its own in-flight copies and MMAs
+// before freeing TMEM and exiting.  It is independent of the (caller-settable)
+// limit of ordinary waits: hardware work already issued finishes in microseconds,
+// and exiting earlier would free memory that copies or MMAs still write.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -110,6 +116,11 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0,
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {

@@ -88,12 +88,17 @@ ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, voi
  *  total_tokens: varlen only; if > 0 it must equal cu_seqlens[B] (checked on the
  *      device).  When 0, attn_fwd_ex (like attn_fwd) reads cu_seqlens[B] back
  *      to the host with a 4-byte copy and a stream synchronisation, because the
- *      TMA views of Q/K/V must not extend past the packed tensors. */
+ *      TMA views of Q/K/V must not extend past the packed tensors.
+ *  test_fault: for tests of the failure path only, 0 otherwise.  1 makes every
+ *      CTA withhold the copy of its first query tile, so the wait for it expires
+ *      after timeout_ns: the kernel records ATTN_ERR_TIMEOUT, drains its other
+ *      copies, frees its tensor memory and returns (outputs undefined). */
 typedef struct {
   float rescale_threshold;
   unsigned long long* stats;
   uint64_t timeout_ns;
   int64_t total_tokens;
+  int test_fault;
 } attn_fwd_opts_t;
 
 /* attn_fwd with options (opts may be NULL = defaults). */

@@ -85,10 +85,11 @@ def test_varlen_limits(lib):
 
 
 def test_bad_options(lib):
-    opts = ea.FwdOpts(float("inf"), None, 0, 0)
-    st = lib.attn_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0, 0.1, None,
-                         ctypes.byref(opts), None)
-    assert st == ea.ATTN_ERR_INVALID_ARG
+    for opts in (ea.FwdOpts(float("inf"), None, 0, 0, 0), ea.FwdOpts(65.0, None, 0, 0, 0),
+                 ea.FwdOpts(-1.0, None, 0, 0, 2)):
+        st = lib.attn_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0, 0.1, None,
+                             ctypes.byref(opts), None)
+        assert st == ea.ATTN_ERR_INVALID_ARG
 
 
 def test_backward_argument_checks(lib):

@@ -227,3 +227,25 @@ def test_fwd_full_workload_sampled(name):
     o_ref, l_ref = oracle.fwd_rows(qp, kp, vp, cu, w.causal, scale, rows, heads)
     compare_o(o[rows, heads], o_ref, name)
     compare_lse(lse[heads, rows], l_ref, name)
+
+
+def test_wait_timeout_is_reported_and_the_context_stays_usable():
+    """With the test-only fault option every CTA withholds its first query-tile
+    copy, so the MMA warp's wait for it runs out (20 ms limit).  Each CTA records
+    ATTN_ERR_TIMEOUT, the other roles see the CTA's abort flag, in-flight copies
+    and MMAs drain, TMEM is freed, and the host reads the status; the next
+    ordinary call still computes the right answer."""
+    ea = _lib()
+    B, N, H, d = 2, 1024, 4, 128
+    q, k, v = ai.make_custom(B, N, H, d, seed=41)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    ea.fwd(qd, kd, vd, causal=True, timeout_ns=20_000_000, test_fault=1)
+    with pytest.raises(ea.AttnError) as e:
+        ea.get_device_status()
+    assert e.value.status == ea.ATTN_ERR_TIMEOUT
+    ea.get_device_status()  # cleared
+    o, lse = ea.fwd(qd, kd, vd, causal=True)
+    ea.get_device_status()
+    o_ref, l_ref = _dense_ref(q, k, v, True, 1 / math.sqrt(d))
+    compare_o(o.cpu(), o_ref, "after timeout")
+    compare_lse(lse.cpu(), l_ref)
