@@ -57,6 +57,13 @@ def _load():
         lib.oracle_fwd_rows.restype = ci
         lib.oracle_probs.argtypes = [dp, dp, ci, i64p, ci, ci, ci, cd, ci, ci, dp]
         lib.oracle_probs.restype = ci
+        lib.oracle_fwd_masked.argtypes = [dp, dp, dp, dp, dp, ci, i64p, ci, ci, ci, ci, ci, cd, ci]
+        lib.oracle_fwd_masked.restype = ci
+        lib.oracle_fwd_rows_masked.argtypes = [dp, dp, dp, ci, i64p, ci, ci, ci, ci, ci, cd, i64p,
+                                               ip, ci, dp, dp, ci]
+        lib.oracle_fwd_rows_masked.restype = ci
+        lib.oracle_probs_masked.argtypes = [dp, dp, ci, i64p, ci, ci, ci, ci, ci, cd, ci, ci, dp]
+        lib.oracle_probs_masked.restype = ci
         lib.oracle_online_fwd.argtypes = [dp, dp, dp, dp, dp, ci, i64p, ci, ci, ci, cd, ci, ci, cd]
         lib.oracle_online_fwd.restype = ctypes.c_int64
         lib.oracle_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, ci, i64p, ci, ci, ci, cd, ci]
@@ -90,22 +97,32 @@ def dense_cu(B: int, N: int) -> np.ndarray:
     return np.arange(B + 1, dtype=np.int64) * N
 
 
-def fwd(q, k, v, cu, causal: bool, scale: float, nthreads: int = 0):
-    """Exact forward: returns (o [T,H,d] fp64, lse [H,T] fp64, threads used)."""
+def _window(window):
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    return wl, wr
+
+
+def fwd(q, k, v, cu, causal: bool, scale: float, nthreads: int = 0, window=None):
+    """Exact forward: returns (o [T,H,d] fp64, lse [H,T] fp64, threads used).
+
+    ``window = (wl, wr)`` adds the sliding-window mask: key j is visible to query i
+    only if ``i - wl <= j <= i + wr`` (a negative bound is unbounded)."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     T, H, d = q.shape
     cu = _cu(cu, T)
     o = np.zeros_like(q)
     lse = np.zeros((H, T), dtype=np.float64)
-    used = _load().oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), cu.size - 1,
-                              _ptr(cu, ctypes.c_int64), H, d, int(causal), float(scale),
-                              int(nthreads))
+    wl, wr = _window(window)
+    used = _load().oracle_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), cu.size - 1,
+                                     _ptr(cu, ctypes.c_int64), H, d, int(causal), wl, wr,
+                                     float(scale), int(nthreads))
     if used < 0:
         raise ValueError("oracle_fwd rejected its arguments")
     return o, lse, used
 
 
-def fwd_rows(q, k, v, cu, causal: bool, scale: float, rows, heads, nthreads: int = 0):
+def fwd_rows(q, k, v, cu, causal: bool, scale: float, rows, heads, nthreads: int = 0,
+             window=None):
     """Exact forward for selected (token, head) rows: returns (o [R,d], lse [R])."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     T, H, d = q.shape
@@ -116,24 +133,27 @@ def fwd_rows(q, k, v, cu, causal: bool, scale: float, rows, heads, nthreads: int
         raise ValueError("rows and heads must be 1-D of equal length")
     o = np.zeros((rows.size, d), dtype=np.float64)
     lse = np.zeros(rows.size, dtype=np.float64)
-    rc = _load().oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), cu.size - 1,
-                                 _ptr(cu, ctypes.c_int64), H, d, int(causal), float(scale),
-                                 _ptr(rows, ctypes.c_int64), _ptr(heads, ctypes.c_int),
-                                 rows.size, _ptr(o), _ptr(lse), int(nthreads))
+    wl, wr = _window(window)
+    rc = _load().oracle_fwd_rows_masked(_ptr(q), _ptr(k), _ptr(v), cu.size - 1,
+                                        _ptr(cu, ctypes.c_int64), H, d, int(causal), wl, wr,
+                                        float(scale), _ptr(rows, ctypes.c_int64),
+                                        _ptr(heads, ctypes.c_int), rows.size, _ptr(o), _ptr(lse),
+                                        int(nthreads))
     if rc < 0:
         raise ValueError("oracle_fwd_rows rejected its arguments")
     return o, lse
 
 
-def probs(q, k, cu, causal: bool, scale: float, b: int, h: int) -> np.ndarray:
+def probs(q, k, cu, causal: bool, scale: float, b: int, h: int, window=None) -> np.ndarray:
     """Probability matrix P [L, L] of sequence b, head h."""
     q, k = _f64(q), _f64(k)
     T, H, d = q.shape
     cu = _cu(cu, T)
     L = int(cu[b + 1] - cu[b])
     P = np.zeros((L, L), dtype=np.float64)
-    rc = _load().oracle_probs(_ptr(q), _ptr(k), cu.size - 1, _ptr(cu, ctypes.c_int64), H, d,
-                              int(causal), float(scale), int(b), int(h), _ptr(P))
+    wl, wr = _window(window)
+    rc = _load().oracle_probs_masked(_ptr(q), _ptr(k), cu.size - 1, _ptr(cu, ctypes.c_int64), H,
+                                     d, int(causal), wl, wr, float(scale), int(b), int(h), _ptr(P))
     if rc < 0:
         raise ValueError("oracle_probs rejected its arguments")
     return P

@@ -20,6 +20,8 @@
  *   oracle_fwd         explicit score row, two-pass softmax, P.V, LSE (definition)
  *   oracle_fwd_rows    the same for a list of (token, head) rows only
  *   oracle_probs       the full probability matrix P of one (sequence, head)
+ *   *_masked           the three above with a sliding-window mask added to the
+ *                      causal option (see visible_range)
  *   oracle_online_fwd  the tiled online-softmax algorithm in the pages' steps
  *                      (FlashAttention 1 recurrences, FlashAttention 2 deferred
  *                      normalisation, FlashAttention 4 conditional rescale)
@@ -28,7 +30,8 @@
  *                      rows (dK, dV) of one (sequence, head), for full-size checks
  *
  * Empty rows cannot occur: a causal row always sees its own key, a non-causal row
- * sees every key of a non-empty sequence.  Zero-length sequences are skipped.
+ * sees every key of a non-empty sequence, and a window never excludes the row's
+ * own key.  Zero-length sequences are skipped.
  */
 #include <math.h>
 #include <stdint.h>
@@ -41,22 +44,39 @@
 /* Number of keys visible to local query row i of a sequence of length L. */
 static int visible_keys(int i, int L, int causal) { return causal ? i + 1 : L; }
 
-/* One query row of one head: scores, two-pass softmax, output row and LSE.
+/* Keys visible to local query row i, as the half-open range [*lo, *hi).
+ * Causal ("FlashAttention 1-4 详解", 其他优化, lower triangle): j <= i.
+ * Sliding window, the mask added beside causal (the pages name FlexAttention's
+ * masks as the interface FA4 serves -- "FlashAttention V4 deep-dive" section 5,
+ * FA-4 summary item [27] -- but print no mask other than causal; reading:
+ * local attention): j >= i - wl when wl >= 0 and j <= i + wr when wr >= 0; a
+ * negative bound means that side is unbounded.  With wl, wr >= 0 the range always
+ * holds j = i. */
+static void visible_range(int i, int L, int causal, int wl, int wr, int* lo, int* hi) {
+  int a = 0, b = L;
+  if (wl >= 0 && i - wl > a) a = i - wl;
+  if (causal && i + 1 < b) b = i + 1;
+  if (wr >= 0 && i + wr + 1 < b) b = i + wr + 1;
+  *lo = a;
+  *hi = b;
+}
+
+/* One query row of one head: scores, two-pass softmax, output row and LSE over the
+ * visible keys [lo, hi).
  * "FlashAttention 1-4 详解", 原算法 (S = Q K^T, P = softmax(S scaled), O = P V) and
  * Online Softmax 数学推导 (two-pass stable softmax: subtract the row max m, divide
  * by the sum of e^{x_j - m}).  srow is caller scratch of length >= L. */
-static void attend_row(const double* q, const double* k, const double* v, double* o_row,
-                       double* lse_out, const double* q_row, int64_t seq_base, int L,
-                       int i, int H, int d, int h, int causal, double scale, double* srow) {
-  (void)q;
-  const int nvis = visible_keys(i, L, causal);
+static void attend_row(const double* k, const double* v, double* o_row, double* lse_out,
+                       const double* q_row, int64_t seq_base, int lo, int hi, int H, int d,
+                       int h, double scale, double* srow) {
   /* Pass 0: scores s_j = scale * <q_i, k_j>. */
-  for (int j = 0; j < nvis; ++j) {
+  for (int j = lo; j < hi; ++j) {
     const double* k_row = k + ((seq_base + j) * H + h) * (int64_t)d;
     double acc = 0.0;
     for (int c = 0; c < d; ++c) acc += q_row[c] * k_row[c];
-    srow[j] = scale * acc;
+    srow[j - lo] = scale * acc;
   }
+  const int nvis = hi - lo;
   /* Pass 1: row max. */
   double m = -INFINITY;
   for (int j = 0; j < nvis; ++j) if (srow[j] > m) m = srow[j];
@@ -67,7 +87,7 @@ static void attend_row(const double* q, const double* k, const double* v, double
   for (int c = 0; c < d; ++c) o_row[c] = 0.0;
   for (int j = 0; j < nvis; ++j) {
     const double p = srow[j] / l;
-    const double* v_row = v + ((seq_base + j) * H + h) * (int64_t)d;
+    const double* v_row = v + ((seq_base + lo + j) * H + h) * (int64_t)d;
     for (int c = 0; c < d; ++c) o_row[c] += p * v_row[c];
   }
   *lse_out = m + log(l);
@@ -84,10 +104,11 @@ static int set_threads(int nthreads) {
 }
 
 /* Exact forward pass over every row.  Returns the number of threads used, or -1 on
- * bad arguments.  cu has nseq+1 entries (token offsets, cu[0] = 0). */
-int oracle_fwd(const double* q, const double* k, const double* v, double* o, double* lse,
-               int nseq, const int64_t* cu, int H, int d, int causal, double scale,
-               int nthreads) {
+ * bad arguments.  cu has nseq+1 entries (token offsets, cu[0] = 0).  wl / wr are
+ * the sliding-window bounds of visible_range (negative: unbounded). */
+int oracle_fwd_masked(const double* q, const double* k, const double* v, double* o,
+                      double* lse, int nseq, const int64_t* cu, int H, int d, int causal,
+                      int wl, int wr, double scale, int nthreads) {
   if (nseq < 0 || H <= 0 || d <= 0 || !cu) return -1;
   const int used = set_threads(nthreads);
   const int64_t T = cu[nseq];
@@ -108,8 +129,10 @@ int oracle_fwd(const double* q, const double* k, const double* v, double* o, dou
       const int L = (int)(cu[b + 1] - cu[b]);
       for (int i = 0; i < L; ++i) {
         const int64_t tok = base + i;
-        attend_row(q, k, v, o + (tok * H + h) * (int64_t)d, lse + (int64_t)h * T + tok,
-                   q + (tok * H + h) * (int64_t)d, base, L, i, H, d, h, causal, scale, srow);
+        int lo, hi;
+        visible_range(i, L, causal, wl, wr, &lo, &hi);
+        attend_row(k, v, o + (tok * H + h) * (int64_t)d, lse + (int64_t)h * T + tok,
+                   q + (tok * H + h) * (int64_t)d, base, lo, hi, H, d, h, scale, srow);
       }
     }
     free(srow);
@@ -117,12 +140,18 @@ int oracle_fwd(const double* q, const double* k, const double* v, double* o, dou
   return used;
 }
 
+int oracle_fwd(const double* q, const double* k, const double* v, double* o, double* lse,
+               int nseq, const int64_t* cu, int H, int d, int causal, double scale,
+               int nthreads) {
+  return oracle_fwd_masked(q, k, v, o, lse, nseq, cu, H, d, causal, -1, -1, scale, nthreads);
+}
+
 /* Exact forward pass for selected rows only: rows[r] is a packed token index and
  * heads[r] its head.  o_rows is [nrows][d], lse_rows [nrows]. */
-int oracle_fwd_rows(const double* q, const double* k, const double* v, int nseq,
-                    const int64_t* cu, int H, int d, int causal, double scale,
-                    const int64_t* rows, const int* heads, int nrows, double* o_rows,
-                    double* lse_rows, int nthreads) {
+int oracle_fwd_rows_masked(const double* q, const double* k, const double* v, int nseq,
+                           const int64_t* cu, int H, int d, int causal, int wl, int wr,
+                           double scale, const int64_t* rows, const int* heads, int nrows,
+                           double* o_rows, double* lse_rows, int nthreads) {
   if (nseq <= 0 || H <= 0 || d <= 0 || !cu) return -1;
   const int used = set_threads(nthreads);
   const int64_t T = cu[nseq];
@@ -136,28 +165,40 @@ int oracle_fwd_rows(const double* q, const double* k, const double* v, int nseq,
     while (cu[b + 1] <= tok) ++b;
     const int64_t base = cu[b];
     const int L = (int)(cu[b + 1] - cu[b]);
+    int lo, hi;
+    visible_range((int)(tok - base), L, causal, wl, wr, &lo, &hi);
     double* srow = (double*)malloc(sizeof(double) * L);
-    attend_row(q, k, v, o_rows + (int64_t)r * d, lse_rows + r, q + (tok * H + h) * (int64_t)d,
-               base, L, (int)(tok - base), H, d, h, causal, scale, srow);
+    attend_row(k, v, o_rows + (int64_t)r * d, lse_rows + r, q + (tok * H + h) * (int64_t)d,
+               base, lo, hi, H, d, h, scale, srow);
     free(srow);
   }
   return bad ? -1 : used;
 }
 
+int oracle_fwd_rows(const double* q, const double* k, const double* v, int nseq,
+                    const int64_t* cu, int H, int d, int causal, double scale,
+                    const int64_t* rows, const int* heads, int nrows, double* o_rows,
+                    double* lse_rows, int nthreads) {
+  return oracle_fwd_rows_masked(q, k, v, nseq, cu, H, d, causal, -1, -1, scale, rows, heads,
+                                nrows, o_rows, lse_rows, nthreads);
+}
+
 /* Probability matrix P[L][L] of sequence b, head h (zeros where masked).
  * "FlashAttention 1-4 详解", 原算法: P = softmax(S / sqrt(d)), row-wise. */
-int oracle_probs(const double* q, const double* k, int nseq, const int64_t* cu, int H, int d,
-                 int causal, double scale, int b, int h, double* P) {
+int oracle_probs_masked(const double* q, const double* k, int nseq, const int64_t* cu, int H,
+                        int d, int causal, int wl, int wr, double scale, int b, int h,
+                        double* P) {
   if (b < 0 || b >= nseq || h < 0 || h >= H) return -1;
   const int64_t base = cu[b];
   const int L = (int)(cu[b + 1] - cu[b]);
   for (int i = 0; i < L; ++i) {
     double* prow = P + (int64_t)i * L;
     const double* q_row = q + ((base + i) * H + h) * (int64_t)d;
-    const int nvis = visible_keys(i, L, causal);
+    int lo, hi;
+    visible_range(i, L, causal, wl, wr, &lo, &hi);
     double m = -INFINITY;
     for (int j = 0; j < L; ++j) {
-      if (j >= nvis) { prow[j] = 0.0; continue; }
+      if (j < lo || j >= hi) { prow[j] = 0.0; continue; }
       const double* k_row = k + ((base + j) * H + h) * (int64_t)d;
       double acc = 0.0;
       for (int c = 0; c < d; ++c) acc += q_row[c] * k_row[c];
@@ -165,10 +206,15 @@ int oracle_probs(const double* q, const double* k, int nseq, const int64_t* cu, 
       if (prow[j] > m) m = prow[j];
     }
     double l = 0.0;
-    for (int j = 0; j < nvis; ++j) { prow[j] = exp(prow[j] - m); l += prow[j]; }
-    for (int j = 0; j < nvis; ++j) prow[j] /= l;
+    for (int j = lo; j < hi; ++j) { prow[j] = exp(prow[j] - m); l += prow[j]; }
+    for (int j = lo; j < hi; ++j) prow[j] /= l;
   }
   return 0;
+}
+
+int oracle_probs(const double* q, const double* k, int nseq, const int64_t* cu, int H, int d,
+                 int causal, double scale, int b, int h, double* P) {
+  return oracle_probs_masked(q, k, nseq, cu, H, d, causal, -1, -1, scale, b, h, P);
 }
 
 /* Tiled online softmax, in the order the pages give the steps.

@@ -302,3 +302,110 @@ def test_bwd_sampled_matches_torch_autograd(causal):
     np.testing.assert_allclose(dq, ref[0][0][rows, h], rtol=0, atol=1e-11)
     np.testing.assert_allclose(dk, ref[1][0][rows, h], rtol=0, atol=1e-11)
     np.testing.assert_allclose(dv, ref[2][0][rows, h], rtol=0, atol=1e-11)
+
+
+# ------------------------------------------------------ sliding-window masks
+# Reading of the mask hook: key j is visible to query i iff i - wl <= j <= i + wr
+# (a negative bound is unbounded), on top of the causal rule when that is set.
+
+def _window_bool_mask(N, wl, wr, causal):
+    """The visibility rule written as a dense boolean matrix [i, j] (True = visible)."""
+    i = torch.arange(N)[:, None]
+    j = torch.arange(N)[None, :]
+    vis = torch.ones(N, N, dtype=torch.bool)
+    if wl >= 0:
+        vis &= j >= i - wl
+    if wr >= 0:
+        vis &= j <= i + wr
+    if causal:
+        vis &= j <= i
+    return vis
+
+
+@pytest.mark.parametrize("wl,wr,causal", [(0, 0, False), (3, 0, True), (5, 2, False),
+                                          (-1, 4, False), (7, -1, False), (16, 16, True),
+                                          (200, 200, False)])
+def test_window_matches_torch_sdpa_with_boolean_mask(wl, wr, causal):
+    """Library special case: PyTorch fp64 SDPA given the visibility matrix as attn_mask."""
+    B, N, H, d = 2, 37, 2, 16
+    scale = 0.3
+    q, k, v = make_custom(B, N, H, d, seed=21)
+    o, lse, _ = oracle.fwd(_packed(q), _packed(k), _packed(v), oracle.dense_cu(B, N), causal,
+                           scale, window=(wl, wr))
+    mask = _window_bool_mask(N, wl, wr, causal)
+    qt, kt, vt = (x.double().permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale)
+    np.testing.assert_allclose(o.reshape(B, N, H, d), ref.permute(0, 2, 1, 3).numpy(), rtol=0,
+                               atol=1e-12)
+    s = torch.einsum("bihc,bjhc->bhij", q.double(), k.double()) * scale
+    ref_lse = torch.logsumexp(s.masked_fill(~mask, float("-inf")), dim=-1).numpy()
+    np.testing.assert_allclose(oracle.lse_to_dense(lse, B, N), ref_lse, rtol=0, atol=1e-12)
+
+
+def test_window_zero_returns_own_value_exactly():
+    """wl = wr = 0: each query sees only its own key, so O_i = V_i exactly and
+    LSE_i = scale * <q_i, k_i>."""
+    q, k, v = make_custom(1, 19, 2, 8, seed=22)
+    qp, kp, vp = _packed(q), _packed(k), _packed(v)
+    o, lse, _ = oracle.fwd(qp, kp, vp, [0, 19], False, 0.7, window=(0, 0))
+    np.testing.assert_array_equal(o, vp)
+    np.testing.assert_allclose(lse, 0.7 * np.einsum("thc,thc->ht", qp, kp), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("wl,wr", [(2, 3), (0, 5), (4, 0), (-1, 1), (3, -1)])
+def test_window_zero_q_returns_mean_of_window(wl, wr):
+    """Q = 0 gives uniform weights: O_i is the mean of V over
+    [max(0, i - wl), min(L - 1, i + wr)] and LSE_i = ln(count) -- an off-by-one at
+    either edge of the window changes both."""
+    L = 23
+    _, k, v = make_custom(1, L, 1, 4, seed=23)
+    vp = _packed(v)
+    o, lse, _ = oracle.fwd(np.zeros((L, 1, 4)), _packed(k), vp, [0, L], False, 1.0,
+                           window=(wl, wr))
+    for i in range(L):
+        lo = 0 if wl < 0 else max(0, i - wl)
+        hi = L - 1 if wr < 0 else min(L - 1, i + wr)
+        np.testing.assert_allclose(o[i, 0], vp[lo:hi + 1, 0].mean(axis=0), rtol=0, atol=1e-12)
+        assert abs(lse[0, i] - math.log(hi - lo + 1)) < 1e-12
+
+
+def test_window_two_key_closed_form():
+    """Causal window of one key back: query i sees keys i-1 and i only.  With
+    q_i = (x), k_{i-1} = (0), k_i = (1), v_{i-1} = 0, v_i = 1 and x = ln 3, the
+    weight of key i is 3/4 (the two-key logistic closed form), whatever lies further back."""
+    x = math.log(3.0)
+    L = 6
+    q = np.full((L, 1, 1), x)
+    k = np.array([[[1.0 if t % 2 else 0.0]] for t in range(L)])
+    v = k.copy()
+    o, lse, _ = oracle.fwd(q, k, v, [0, L], True, 1.0, window=(1, 0))
+    for i in range(1, L, 2):  # odd i: key i has k = 1, key i-1 has k = 0
+        assert abs(o[i, 0, 0] - 0.75) < 1e-15
+        assert abs(lse[0, i] - math.log(4.0)) < 1e-15
+
+
+@pytest.mark.parametrize("wl,wr,causal", [(4, 1, False), (6, 0, True)])
+def test_window_probs_zero_outside_and_rows_sum_to_one(wl, wr, causal):
+    q, k, _ = make_custom(1, 31, 1, 8, seed=24)
+    P = oracle.probs(_packed(q), _packed(k), [0, 31], causal, 0.5, 0, 0, window=(wl, wr))
+    mask = _window_bool_mask(31, wl, wr, causal).numpy()
+    assert np.all(P[~mask] == 0.0)
+    assert np.all(P[mask] > 0.0)
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+
+
+def test_window_rows_equal_full_and_wide_window_is_unmasked():
+    """fwd_rows honours the window, and a window wider than the sequence masks nothing."""
+    lengths = [50, 7, 90]
+    q, k, v = make_custom(0, 0, 2, 16, seed=25, lengths=lengths)
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    qp, kp, vp = _packed(q), _packed(k), _packed(v)
+    o, lse, _ = oracle.fwd(qp, kp, vp, cu, False, 0.25, window=(9, 4))
+    rows = np.array([0, 5, 49, 50, 56, 57, 100, 146])
+    heads = np.array([0, 1, 1, 0, 1, 0, 1, 0])
+    o_r, l_r = oracle.fwd_rows(qp, kp, vp, cu, False, 0.25, rows, heads, window=(9, 4))
+    np.testing.assert_allclose(o_r, o[rows, heads], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l_r, lse[heads, rows], rtol=0, atol=1e-13)
+    o_w, _, _ = oracle.fwd(qp, kp, vp, cu, True, 0.25, window=(1000, 1000))
+    o_c, _, _ = oracle.fwd(qp, kp, vp, cu, True, 0.25)
+    np.testing.assert_array_equal(o_w, o_c)
