@@ -14,7 +14,7 @@ own generator (seed 1).
 from __future__ import annotations
 
 from dataclasses import dataclass, field
-from typing import List, Optional
+from typing import List, Optional, Tuple
 
 import torch
 
@@ -30,6 +30,8 @@ class Workload:
     causal: bool
     q_mult: float = 1.0  # exact power-of-two multiplier applied to the bf16 Q
     lengths: Optional[List[int]] = field(default=None)  # varlen sequence lengths
+    # sliding window (left, right): key j visible to query i iff i-left <= j <= i+right
+    window: Optional[Tuple[int, int]] = None
 
     @property
     def varlen(self) -> bool:
@@ -55,19 +57,21 @@ def varlen_lengths(n: int = 16, lo: int = 512, hi: int = 16384, seed: int = 1) -
     return [int(x) for x in torch.randint(lo, hi + 1, (n,), generator=g)]
 
 
-# The five benchmark problems: tiny latency case, dense non-causal (and a variant
-# with Q scaled by 4 so the running maximum moves often), long causal, packed
-# causal varlen, and the causal backward problem.
+# The benchmark problems: tiny latency case, dense non-causal (and a variant with
+# Q scaled by 4 so the running maximum moves often), long causal, packed causal
+# varlen, the long causal problem under a 1024-key sliding window, and the causal
+# backward problem.
 TINY = Workload("B1-H1-N256-d64", 1, 1, 256, 64, False)
 DENSE = Workload("B4-H16-N2048-d128", 4, 16, 2048, 128, False)
 DENSE_X4 = Workload("B4-H16-N2048-d128-qx4", 4, 16, 2048, 128, False, q_mult=4.0)
 CAUSAL = Workload("B2-H16-N8192-d128-causal", 2, 16, 8192, 128, True)
 _VL = varlen_lengths()
 VARLEN = Workload("varlen16-H16-d128-causal", len(_VL), 16, max(_VL), 128, True, lengths=_VL)
+WINDOW = Workload("B2-H16-N8192-d128-causal-win1024", 2, 16, 8192, 128, True, window=(1024, 0))
 BWD_CAUSAL = CAUSAL  # the backward problem uses the causal forward's shapes
 BWD_NAME = CAUSAL.name + "-bwd"
 
-ALL = {w.name: w for w in (TINY, DENSE, DENSE_X4, CAUSAL, VARLEN)}
+ALL = {w.name: w for w in (TINY, DENSE, DENSE_X4, CAUSAL, VARLEN, WINDOW)}
 
 
 def make_qkv(w: Workload, seed: int = 0, with_dout: bool = False):

@@ -38,10 +38,26 @@ FLUSH_BYTES = 256 << 20
 MUFU_EX2_PER_CLK_PER_SM = 16  # 4 SFU lanes per SM sub-partition, 4 sub-partitions
 
 
+def visible_pairs(L: int, causal: bool, window=None) -> float:
+    """(query, key) pairs a sequence of length L attends to.  Causal without a
+    window counts L^2/2 (the convention of the published causal TFLOP/s figures);
+    under a sliding window the exact count."""
+    if window is None:
+        return L * L / 2.0 if causal else float(L * L)
+    import numpy as np
+    i = np.arange(L, dtype=np.int64)
+    wl, wr = window
+    lo = np.maximum(i - wl, 0) if wl >= 0 else np.zeros_like(i)
+    hi = np.full_like(i, L - 1)
+    if wr >= 0:
+        hi = np.minimum(hi, i + wr)
+    if causal:
+        hi = np.minimum(hi, i)
+    return float((hi - lo + 1).sum())
+
+
 def workload_flops(w: ai.Workload) -> float:
-    per_seq = [4.0 * w.H * L * L * w.d for L in w.seq_lengths()]
-    total = sum(per_seq)
-    return total / 2.0 if w.causal else total
+    return sum(4.0 * w.H * w.d * visible_pairs(L, w.causal, w.window) for L in w.seq_lengths())
 
 
 def workload_exps(w: ai.Workload) -> float:
@@ -79,19 +95,6 @@ def profiled_traffic(workload: str):
         return float(fields["dram_bytes_per_launch"])
     except (KeyError, ValueError):
         return None
-
-
-def poly_pairs_per_8() -> int:
-    """Column pairs of every 8 the kernel exponentiates on the FMA pipe (compiled-in
-    default, or the override passed to the build through ATTN_NVCC_EXTRA)."""
-    import re
-    m = re.search(r"-DATTN_POLY_PAIRS_PER_8=(\d+)", os.environ.get("ATTN_NVCC_EXTRA", ""))
-    if m:
-        return int(m.group(1))
-    src = os.path.join(ROOT, "exact_attention_103_b200", "csrc", "attn_fwd_sm100.cu")
-    with open(src) as f:
-        m = re.search(r"#define ATTN_POLY_PAIRS_PER_8 (\d+)", f.read())
-    return int(m.group(1)) if m else 0
 
 
 def load_peaks():
@@ -221,9 +224,9 @@ def cpu_oracle_sample(w: ai.Workload, q, k, v, budget_s: float):
             rows = np.arange(cu[b], cu[b + 1])
             heads = np.full(L, h)
             t0 = time.perf_counter()
-            oracle.fwd_rows(qp, kp, vp, cu, w.causal, scale, rows, heads)
+            oracle.fwd_rows(qp, kp, vp, cu, w.causal, scale, rows, heads, window=w.window)
             spent += time.perf_counter() - t0
-            f = 4.0 * L * L * w.d * (0.5 if w.causal else 1.0)
+            f = 4.0 * w.d * visible_pairs(L, w.causal, w.window)
             done_flops += f
             units += 1
             if spent >= budget_s:
@@ -238,7 +241,7 @@ def cpu_oracle_sample(w: ai.Workload, q, k, v, budget_s: float):
 
 def bench_config(w: ai.Workload, world: int) -> dict:
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-            "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"replicas{world}",
+            "window": w.window, "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"replicas{world}",
             "l2": "flushed (256 MiB write) before every timed step"}
 
 
@@ -292,7 +295,7 @@ def run_ours(args, rank, world, local):
 
     def step():
         ea.fwd(q, k, v, causal=w.causal, scale=scale, cu_seqlens=cu, max_seqlen=max_len,
-               out=out, lse=lse)
+               out=out, lse=lse, window=w.window, exp_poly_per8=args.exp_poly_per8)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -321,7 +324,7 @@ def run_ours(args, rank, world, local):
     mhz = clk["sm_mhz"] or peaks["sm_max_mhz"]
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     mufu_peak = sms * MUFU_EX2_PER_CLK_PER_SM * mhz * 1e6
-    mufu_share = 1.0 - poly_pairs_per_8() / 8.0
+    mufu_share = 1.0 - args.exp_poly_per8 / 8.0
     mufu_achieved = mufu_share * workload_exps(w) / (statistics.mean(times) / 1e3)
 
     # End to end through the public API from pinned host buffers: H2D of Q/K/V
@@ -333,7 +336,8 @@ def run_ours(args, rank, world, local):
     l_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     for _ in range(2):
         ea.fwd_from_host(q_p, k_p, v_p, causal=w.causal, scale=scale, cu_seqlens_host=cu_p,
-                         max_seqlen=max_len, out_host=o_host, lse_host=l_host)
+                         max_seqlen=max_len, out_host=o_host, lse_host=l_host, window=w.window,
+                         exp_poly_per8=args.exp_poly_per8)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -341,7 +345,8 @@ def run_ours(args, rank, world, local):
     for _ in range(e2e_steps):
         o_h, l_h = ea.fwd_from_host(q_p, k_p, v_p, causal=w.causal, scale=scale,
                                     cu_seqlens_host=cu_p, max_seqlen=max_len,
-                                    out_host=o_host, lse_host=l_host)
+                                    out_host=o_host, lse_host=l_host, window=w.window,
+                                    exp_poly_per8=args.exp_poly_per8)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
@@ -359,7 +364,7 @@ def run_ours(args, rank, world, local):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": bench_config(w, world),
+                "config": dict(bench_config(w, world), exp_poly_per8=args.exp_poly_per8),
                 "pct_of_peak": 100.0 * achieved / peak,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                              "unit": "TFLOP/s", "frac": achieved / peak,
@@ -438,6 +443,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--exp-poly-per8", type=int, default=0, choices=[0, 2, 8],
+                    help="exponential pairs of every 8 computed by the FMA-pipe polynomial")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -39,7 +39,11 @@ class FwdOpts(ctypes.Structure):
                 ("stats", ctypes.c_void_p),
                 ("timeout_ns", ctypes.c_uint64),
                 ("total_tokens", ctypes.c_int64),
-                ("test_fault", ctypes.c_int)]
+                ("test_fault", ctypes.c_int),
+                ("has_window", ctypes.c_int),
+                ("window_left", ctypes.c_int),
+                ("window_right", ctypes.c_int),
+                ("exp_poly_per8", ctypes.c_int)]
 
 
 _lib = None
@@ -113,13 +117,17 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         lse: Optional[torch.Tensor] = None, rescale_threshold: Optional[float] = None,
         stats: Optional[torch.Tensor] = None, timeout_ns: int = 0,
         stream: Optional[torch.cuda.Stream] = None,
-        test_fault: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+        test_fault: int = 0, window: Optional[Tuple[int, int]] = None,
+        exp_poly_per8: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
     """Exact attention forward on the GPU.
 
     Dense: q, k, v are bf16 ``[B, N, H, d]``; returns O ``[B, N, H, d]`` and LSE
     ``[B, H, N]`` (fp32, natural log).  Varlen: q, k, v are packed ``[T, H, d]``,
     ``cu_seqlens`` is int32 ``[B+1]`` on the device and ``max_seqlen`` the longest
     sequence; LSE is ``[H, T]``.  ``scale`` defaults to ``1/sqrt(d)``.
+    ``window = (left, right)`` keeps key j for query i only if
+    ``i - left <= j <= i + right`` (negative = open side).  ``exp_poly_per8``
+    (0, 2 or 8) moves that many of every 8 exponential pairs to the FMA pipe.
     """
     lib = load_library()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -130,7 +138,9 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     opts = FwdOpts(-1.0 if rescale_threshold is None else float(rescale_threshold),
-                   None if stats is None else stats.data_ptr(), int(timeout_ns), 0, int(test_fault))
+                   None if stats is None else stats.data_ptr(), int(timeout_ns), 0, int(test_fault),
+                   0 if window is None else 1, -1 if window is None else int(window[0]),
+                   -1 if window is None else int(window[1]), int(exp_poly_per8))
     if stats is not None:
         _need(stats, "stats", torch.int64)
     if cu_seqlens is None:
@@ -186,7 +196,8 @@ def fwd_from_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tens
                   max_seqlen: Optional[int] = None, device: str = "cuda",
                   stream: Optional[torch.cuda.Stream] = None,
                   out_host: Optional[torch.Tensor] = None,
-                  lse_host: Optional[torch.Tensor] = None):
+                  lse_host: Optional[torch.Tensor] = None,
+                  window: Optional[Tuple[int, int]] = None, exp_poly_per8: int = 0):
     """End-to-end call from host tensors: copies Q/K/V (and cu_seqlens) to the
     device, runs the forward, copies O and LSE back into host tensors (``out_host``
     / ``lse_host`` if given, ideally pinned; else new pinned tensors).  Returns
@@ -198,7 +209,7 @@ def fwd_from_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tens
         v = v_host.to(device, non_blocking=True)
         cu = None if cu_seqlens_host is None else cu_seqlens_host.to(device, non_blocking=True)
         o, lse = fwd(q, k, v, causal=causal, scale=scale, cu_seqlens=cu, max_seqlen=max_seqlen,
-                     stream=s)
+                     stream=s, window=window, exp_poly_per8=exp_poly_per8)
         o_h = out_host if out_host is not None else torch.empty(o.shape, dtype=o.dtype,
                                                                 pin_memory=True)
         l_h = lse_host if lse_host is not None else torch.empty(lse.shape, dtype=lse.dtype,

@@ -126,7 +126,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   float tau = kDefaultTau;
   uint64_t timeout = kDefaultTimeoutNs;
   unsigned long long* stats = nullptr;
-  int test_fault = 0;
+  int test_fault = 0, poly = 0, has_window = 0, wl = -1, wr = -1;
   if (opts) {
     if (opts->test_fault != 0 && opts->test_fault != 1)
       return fail(ATTN_ERR_INVALID_ARG, "test_fault must be 0 or 1");
@@ -136,6 +136,28 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
     if (opts->timeout_ns) timeout = opts->timeout_ns;
     stats = opts->stats;
     if (stats && !aligned(stats, 8)) return fail(ATTN_ERR_INVALID_ARG, "stats misaligned");
+    poly = opts->exp_poly_per8;
+    if (poly != 0 && poly != 2 && poly != 8)
+      return fail(ATTN_ERR_INVALID_ARG, "exp_poly_per8 must be 0, 2 or 8");
+    if (opts->has_window) {
+      has_window = 1;
+      wl = opts->window_left;
+      wr = opts->window_right;
+    }
+  }
+  // The mask: a window bound of N - 1 or more hides nothing on that side, so the
+  // window collapses to the causal or the unmasked kernel where it can.
+  attn::MaskKind mask = causal ? attn::kMaskCausal : attn::kMaskNone;
+  int win_l = 0, win_r = 0;
+  if (has_window) {
+    if (N >= (1 << 30)) return fail(ATTN_ERR_UNSUPPORTED, "sliding window needs N < 2^30");
+    win_l = (wl < 0 || wl > N) ? N : wl;
+    win_r = causal ? 0 : ((wr < 0 || wr > N) ? N : wr);
+    const bool left_open = win_l >= N - 1, right_open = win_r >= N - 1;
+    if (left_open && right_open) mask = attn::kMaskNone;
+    else if (left_open && win_r == 0) mask = attn::kMaskCausal;
+    else mask = attn::kMaskWindow;
+    if (mask == attn::kMaskWindow) stats = nullptr;  // counters are not kept under a window
   }
 
   DeviceState* dev = nullptr;
@@ -179,12 +201,14 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   a.p.stats = stats;
   a.p.timeout_ns = timeout;
   a.p.test_fault = test_fault;
-  // Dense non-causal launches may split their last wave into half items (see the
+  a.p.wl = win_l;
+  a.p.wr = win_r;
+  // Dense unmasked launches may split their last wave into half items (see the
   // kernel), so up to twice as many CTAs can be useful there.
-  const int64_t useful = (!varlen && !causal) ? 2 * items_bound : items_bound;
+  const int64_t useful = (!varlen && mask == attn::kMaskNone) ? 2 * items_bound : items_bound;
   a.grid = static_cast<int>(useful < dev->sms ? useful : dev->sms);
   a.smem = attn::fwd_smem_bytes(d, B, static_cast<int>(T256), varlen ? 1 : 0);
-  const cudaError_t e = attn::launch_fwd(a, d, causal ? 1 : 0, cs);
+  const cudaError_t e = attn::launch_fwd(a, d, mask, poly, cs);
   if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
   return ATTN_OK;
 }

@@ -53,15 +53,6 @@ constexpr int kBM = 128;  // query rows per sub-tile
 constexpr int kBN = 128;  // keys per key tile
 constexpr float kLn2 = 0.693147180559945309f;
 
-// Of every 8 consecutive (even, odd) column pairs of a score row, this many are
-// exponentiated on the FMA pipe by the polynomial below; the rest use MUFU ex2.
-// Measured on B200 (same-box A/B, this kernel): 0 is fastest; 1 costs ~1%, 2 ~4%.
-#ifndef ATTN_POLY_PAIRS_PER_8
-#define ATTN_POLY_PAIRS_PER_8 0
-#endif
-constexpr int kPolyPairsPer8 = ATTN_POLY_PAIRS_PER_8;
-static_assert(kPolyPairsPer8 >= 0 && kPolyPairsPer8 <= 8, "pairs per 8");
-
 // 2^y without MUFU: j = round(y) by the 1.5*2^23 trick, f = y - j in [-1/2, 1/2],
 // p(f) ~ 2^f (minimax, exp2_poly.h), then 2^j is added to the exponent field as an
 // integer.  y is clamped below at -125 so the result stays a normal float (the
@@ -164,17 +155,68 @@ struct Sched {
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// Key tiles sub-tile s of an item processes (0 when its rows are all past L, or
-// for the missing second sub-tile of a half item).
-template <bool CAUSAL>
-__device__ __forceinline__ int num_kv_tiles(const Item& it, int s) {
-  if (!CAUSAL && s == 1 && !it.two) return 0;
+// The mask hook, one compile-time functor per MaskKind.  For the 128 query rows
+// [row0, row0 + 128) of a sequence of length L:
+//   tiles()   the key tiles [lo, hi) holding a key visible to some row; the tiles
+//             outside are skipped, not loaded;
+//   partial() whether key tile kb (its first key) may hide a key from some row;
+//   cols()    the visible columns [c_lo, c_hi) of that tile for query row q.
+// Causal is the lower triangle of "FlashAttention 1-4 详解", 其他优化 (tiles above
+// the diagonal skipped).  The window is this library's instance of the
+// FlexAttention mask interface ("FlashAttention V4 deep-dive", section 5):
+// q - wl <= key <= q + wr.  A new mask is a new MaskKind with these three members.
+template <int MASK>
+struct MaskFn {
+  int wl, wr;  // kMaskWindow only; both >= 0 and below 2^30
+  __device__ __forceinline__ void tiles(int row0, int L, int& lo, int& hi) const {
+    const int all = ceil_div(L, kBN);
+    lo = 0;
+    hi = all;
+    if (MASK == kMaskCausal) {
+      hi = min(row0 / kBN + 1, all);  // up to and including the diagonal tile
+    } else if (MASK == kMaskWindow) {
+      lo = max(row0 - wl, 0) / kBN;
+      hi = ceil_div(min(row0 + kBM + wr, L), kBN);
+    }
+  }
+  __device__ __forceinline__ bool partial(int kb, int row0, int L) const {
+    if (kb + kBN > L) return true;
+    if (MASK == kMaskCausal) return kb + kBN - 1 > row0;
+    if (MASK == kMaskWindow) return kb < row0 + kBM - 1 - wl || kb + kBN - 1 > row0 + wr;
+    return false;
+  }
+  __device__ __forceinline__ void cols(int q, int kb, int L, int& c_lo, int& c_hi) const {
+    c_lo = 0;
+    c_hi = L - kb;
+    if (MASK == kMaskCausal) c_hi = min(c_hi, q - kb + 1);
+    if (MASK == kMaskWindow) {
+      c_lo = q - wl - kb;
+      c_hi = min(c_hi, q + wr + 1 - kb);
+    }
+  }
+};
+
+// Key tiles [lo, hi) that sub-tile s of an item processes (empty when its rows are
+// all past L, or for the missing second sub-tile of a half item).
+template <int MASK>
+__device__ __forceinline__ void kv_range(const Item& it, int s, const MaskFn<MASK>& mk, int& lo,
+                                         int& hi) {
+  lo = hi = 0;
+  if (s == 1 && !it.two) return;
   const int row0 = it.row_base + s * kBM;
-  if (row0 >= it.L) return 0;
-  const int all = ceil_div(it.L, kBN);
-  if (!CAUSAL) return all;
-  const int diag = row0 / kBN + 1;  // tiles up to and including the diagonal
-  return diag < all ? diag : all;
+  if (row0 >= it.L) return;
+  mk.tiles(row0, it.L, lo, hi);
+}
+
+// Key tiles of the whole item: the union of its sub-tiles' ranges (sub-tile 0 is
+// never empty and its range starts no later than sub-tile 1's).
+template <int MASK>
+__device__ __forceinline__ void item_range(const Item& it, const MaskFn<MASK>& mk, int& lo, int& n) {
+  int lo0, hi0, lo1, hi1;
+  kv_range<MASK>(it, 0, mk, lo0, hi0);
+  kv_range<MASK>(it, 1, mk, lo1, hi1);
+  lo = lo0;
+  n = (hi1 > hi0 ? hi1 : hi0) - lo0;
 }
 
 // Inclusive warp scan (sum) of one value per lane.
@@ -255,12 +297,16 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64
   return true;
 }
 
-template <int D, bool CAUSAL>
+// POLY: of every 8 consecutive (even, odd) column pairs of a score row, this many
+// are exponentiated on the FMA pipe by exp2_poly; the rest use MUFU ex2.
+template <int D, int MASK, int POLY>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using Lay = Layout<D>;
   constexpr int NS = Lay::NSTAGE;
+  constexpr bool SPLIT = MASK == kMaskNone;  // the launch may hold half items
+  static_assert(POLY >= 0 && POLY <= 8, "pairs per 8");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -323,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // more SMs (a half item runs without a ping-pong partner, but the wave is
   // shorter).  Causal and varlen items are already longest-first.
   sch.split = 0;
-  if (!CAUSAL && p.cu_seqlens == nullptr) {
+  if (SPLIT && p.cu_seqlens == nullptr) {
     const int rem = sch.pairs % static_cast<int>(gridDim.x);
     if (rem > 0 && 2 * rem <= static_cast<int>(gridDim.x)) sch.split = rem;
   }
@@ -332,6 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   wc.abort = reinterpret_cast<volatile uint32_t*>(misc + 1);
   wc.err = p.err;
   wc.limit_ns = p.timeout_ns;
+  MaskFn<MASK> mk;
+  mk.wl = p.wl;
+  mk.wr = p.wr;
 
   if (warp < 8) {
     // ------------------------------------------------------------ softmax
@@ -348,15 +397,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0;; ++k) {
       const int idx = sch.item(k);
       if (idx < 0) break;
-      const Item it = sch.template decode<!CAUSAL>(idx);
+      const Item it = sch.template decode<SPLIT>(idx);
       const int b = it.b, h = it.h, seq_start = it.seq_start, L = it.L;
-      const int nkv = num_kv_tiles<CAUSAL>(it, s);
-      if (nkv == 0) continue;
+      int jlo, jhi;
+      kv_range<MASK>(it, s, mk, jlo, jhi);
+      if (jhi <= jlo) continue;
       const int row0 = it.row_base + s * kBM;
       const int q_row = row0 + r;
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < nkv; ++j) {
+      for (int j = jlo; j < jhi; ++j) {
         ok = mbar_wait(bar(Lay::B_SFULL + s), s_phase, wc, timeout_code(kSiteSFull));
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -365,12 +415,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sv[128];
         tmem_ld_x128(t_s, sv);
         const int kb = j * kBN;
-        if ((CAUSAL && kb + kBN - 1 > row0) || kb + kBN > L) {
-          int lim = L - kb;  // keys [kb, kb+lim) are visible to this row
-          if (CAUSAL && q_row - kb + 1 < lim) lim = q_row - kb + 1;
+        if (mk.partial(kb, row0, L)) {
+          int c_lo, c_hi;  // keys [kb + c_lo, kb + c_hi) are visible to this row
+          mk.cols(q_row, kb, L, c_lo, c_hi);
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (c >= lim) sv[c] = __float_as_uint(-INFINITY);
+            if (c < c_lo || c >= c_hi) sv[c] = __float_as_uint(-INFINITY);
         }
         // Row maximum: four independent 3-input max chains, then a small tree.
         float m4[4];
@@ -387,7 +437,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_tile = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sl;
         bool need = false;
         float alpha = 1.f;
-        if (j == 0) {
+        // A window can hide every key of a tile from a row (m_tile = -inf): the
+        // row's reference is then set by its first tile with a visible key.
+        if (MASK == kMaskWindow ? m_ref == -INFINITY : j == jlo) {
           m_ref = m_tile;
         } else {
           ++n_rowtiles;
@@ -401,14 +453,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // P~ = 2^(s*scale*log2e - m_ref): one FMA for the argument, MUFU ex2 or the
         // FMA-pipe polynomial for the exponential, partial row sums, bf16 packing.
-        const float nm = -m_ref;
+        const float nm = (MASK == kMaskWindow && m_ref == -INFINITY) ? 0.f : -m_ref;
         uint32_t pk[64];
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           float a = fmaf(__uint_as_float(sv[2 * c]), sl, nm);
           float e = fmaf(__uint_as_float(sv[2 * c + 1]), sl, nm);
-          if ((c & 7) >= 8 - kPolyPairsPer8) {
+          if ((c & 7) >= 8 - POLY) {
             a = exp2_poly(a);
             e = exp2_poly(e);
           } else {
@@ -495,10 +547,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int idx = sch.item(k);
       if (idx < 0) break;
-      const Item it = sch.template decode<!CAUSAL>(idx);
+      const Item it = sch.template decode<SPLIT>(idx);
       const int h = it.h, seq_start = it.seq_start;
-      const int nkv0 = num_kv_tiles<CAUSAL>(it, 0), nkv1 = num_kv_tiles<CAUSAL>(it, 1);
-      const int nkv = nkv0 > nkv1 ? nkv0 : nkv1;
+      int jlo, nkv;
+      item_range<MASK>(it, mk, jlo, nkv);
       if (k > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QEMPTY), qe_phase, wc, timeout_code(kSiteQEmpty)));
         if (!ok) break;
@@ -532,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
               tma_load_3d(sb + Lay::KV_OFF + slot * Lay::TILE + c * Lay::CHUNK, which ? &tm_v : &tm_k,
-                          bar(Lay::B_KVFULL + slot), c * 64, h, seq_start + j * kBN, pol_kv);
+                          bar(Lay::B_KVFULL + slot), c * 64, h, seq_start + (jlo + j) * kBN, pol_kv);
           }
           __syncwarp();
           ++n_ld;
@@ -549,6 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // The whole warp walks the loop and waits; one elected lane issues each MMA
     // and commit.  Issue order per key tile j (ping-pong of the two sub-tiles):
     //   PV(0, j-1), S(0, j), PV(1, j-1), S(1, j)
+    // each only where tile j (j-1) lies in that sub-tile's key range.
     // S(s, j) overwrites P(s, j-1) in TMEM, which PV(s, j-1) read just before; the
     // tensor pipe executes one thread's MMAs in issue order.
     constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0, 0);
@@ -560,21 +613,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int idx = sch.item(k);
       if (idx < 0) break;
-      const Item it = sch.template decode<!CAUSAL>(idx);
-      const int nk0 = num_kv_tiles<CAUSAL>(it, 0), nk1 = num_kv_tiles<CAUSAL>(it, 1);
-      const int nkv = nk0 > nk1 ? nk0 : nk1;
+      const Item it = sch.template decode<SPLIT>(idx);
+      int jlo, nkv, lo0, hi0, lo1, hi1;
+      item_range<MASK>(it, mk, jlo, nkv);
+      kv_range<MASK>(it, 0, mk, lo0, hi0);
+      kv_range<MASK>(it, 1, mk, lo1, hi1);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QFULL), q_phase, wc, timeout_code(kSiteQFull)));
       if (!ok) break;
       q_phase ^= 1u;
       tc_fence_after();
-      for (int j = 0; j <= nkv && ok; ++j) {
-        const uint32_t nK = n_ld + 2u * j;  // load sequence number of K_j
+      for (int jj = 0; jj <= nkv && ok; ++jj) {
+        const int j = jlo + jj;              // key tile
+        const uint32_t nK = n_ld + 2u * jj;  // load sequence number of K_j
         const uint32_t nV = nK - 1u;        // ... and of V_{j-1}
         const uint32_t slotK = nK % NS, slotV = nV % NS;
-        if (j < nkv)
+        if (jj < nkv)
           ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KVFULL + slotK), (nK / NS) & 1u, wc,
                                                  timeout_code(kSiteKvFull)));
-        if (ok && j > 0)
+        if (ok && jj > 0)
           ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KVFULL + slotV), (nV / NS) & 1u, wc,
                                                  timeout_code(kSiteKvFull)));
         if (!ok) break;
@@ -582,8 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
           const uint32_t tS = s ? tS1 : tS0, tO = s ? tO1 : tO0;
-          const int nks = s ? nk1 : nk0;
-          if (ok && j > 0 && j - 1 < nks) {
+          const int los = s ? lo1 : lo0, his = s ? hi1 : hi0;
+          if (ok && jj > 0 && j - 1 >= los && j - 1 < his) {
             uint32_t& ph = s ? p_phase1 : p_phase0;
             ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_PFULL + s), ph, wc, timeout_code(kSitePFull)));
             if (ok) {
@@ -594,16 +650,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int kk = 0; kk < kBN / 16; ++kk) {
                 if (elect_one())
                   mma_ts(tO, tS + kk * 8, sdesc_sw128(vbase + kk * 2048, Lay::CHUNK, 1024), idesc_o,
-                         (j > 1 || kk > 0) ? 1u : 0u);
+                         (j - 1 > los || kk > 0) ? 1u : 0u);
                 __syncwarp();
               }
-              if (j == nks) {
+              if (j == his) {
                 if (elect_one()) tc_commit(bar(Lay::B_OFULL + s));
                 __syncwarp();
               }
             }
           }
-          if (ok && j < nks) {
+          if (ok && j >= los && j < his) {
             const uint32_t qbase = sb + Lay::Q_OFF + s * Lay::TILE;
             const uint32_t kbase = sb + Lay::KV_OFF + slotK * Lay::TILE;
 #pragma unroll
@@ -620,9 +676,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         if (elect_one()) {
-          if (j < nkv) tc_commit(bar(Lay::B_KVEMPTY + slotK));
-          if (j > 0) tc_commit(bar(Lay::B_KVEMPTY + slotV));
-          if (j == nkv - 1) tc_commit(bar(Lay::B_QEMPTY));
+          if (jj < nkv) tc_commit(bar(Lay::B_KVEMPTY + slotK));
+          if (jj > 0) tc_commit(bar(Lay::B_KVEMPTY + slotV));
+          if (jj == nkv - 1) tc_commit(bar(Lay::B_QEMPTY));
         }
         __syncwarp();
       }
@@ -651,18 +707,31 @@ int fwd_smem_bytes(int D, int B, int T, int varlen) {
   return fixed + (varlen ? (B + 3 * T + 1) * 4 : 0);
 }
 
-template <int D, bool CAUSAL>
+template <int D, int MASK, int POLY>
 static cudaError_t launch_t(const FwdLaunch& a, cudaStream_t st) {
-  auto kern = fwd_kernel<D, CAUSAL>;
+  auto kern = fwd_kernel<D, MASK, POLY>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem);
   if (e != cudaSuccess) return e;
   kern<<<a.grid, kThreads, a.smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_fwd(const FwdLaunch& a, int D, int causal, cudaStream_t st) {
-  if (D == 128) return causal ? launch_t<128, true>(a, st) : launch_t<128, false>(a, st);
-  return causal ? launch_t<64, true>(a, st) : launch_t<64, false>(a, st);
+template <int D, int MASK>
+static cudaError_t launch_p(const FwdLaunch& a, int poly, cudaStream_t st) {
+  if (poly == 2) return launch_t<D, MASK, 2>(a, st);
+  if (poly == 8) return launch_t<D, MASK, 8>(a, st);
+  return launch_t<D, MASK, 0>(a, st);
+}
+
+template <int D>
+static cudaError_t launch_m(const FwdLaunch& a, MaskKind mask, int poly, cudaStream_t st) {
+  if (mask == kMaskCausal) return launch_p<D, kMaskCausal>(a, poly, st);
+  if (mask == kMaskWindow) return launch_p<D, kMaskWindow>(a, poly, st);
+  return launch_p<D, kMaskNone>(a, poly, st);
+}
+
+cudaError_t launch_fwd(const FwdLaunch& a, int D, MaskKind mask, int poly, cudaStream_t st) {
+  return D == 128 ? launch_m<128>(a, mask, poly, st) : launch_m<64>(a, mask, poly, st);
 }
 
 }  // namespace attn

@@ -8,6 +8,14 @@
 
 namespace attn {
 
+// The mask hook: which (query, key) pairs are visible.  Each kind is a
+// compile-time functor of the kernel (attn_fwd_sm100.cu, struct MaskFn).
+enum MaskKind : int {
+  kMaskNone = 0,    // every key of the sequence
+  kMaskCausal = 1,  // key <= query
+  kMaskWindow = 2,  // query - wl <= key <= query + wr
+};
+
 struct FwdParams {
   __nv_bfloat16* o;      // [T, H, D] bf16 (dense T = B*N)
   float* lse;            // dense [B, H, N]; varlen [H, total]
@@ -21,6 +29,7 @@ struct FwdParams {
   unsigned long long* stats;  // optional [rescaled rows, row-tiles]
   uint64_t timeout_ns;   // limit of every internal wait
   int test_fault;        // 1: withhold the first Q copy (failure-path tests only)
+  int wl, wr;            // kMaskWindow bounds, both >= 0 (an open side holds a large value)
 };
 
 struct FwdLaunch {
@@ -31,6 +40,7 @@ struct FwdLaunch {
 };
 
 int fwd_smem_bytes(int D, int B, int T, int varlen);
-cudaError_t launch_fwd(const FwdLaunch& a, int D, int causal, cudaStream_t st);
+// poly: exponentials per 8 column pairs on the FMA-pipe polynomial (0, 2 or 8).
+cudaError_t launch_fwd(const FwdLaunch& a, int D, MaskKind mask, int poly, cudaStream_t st);
 
 }  // namespace attn

@@ -140,7 +140,7 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
   // The status word must start at zero; it keeps the previous call's value otherwise.
   cudaError_t e = cudaMemsetAsync(dev->scratch, 0, kFwdScratchNeeded, cs);
   if (e != cudaSuccess) return report(ATTN_ERR_CUDA, "attn_fwd_noalloc: clearing the status word failed");
-  e = attn::launch_fwd(a, d, causal ? 1 : 0, cs);
+  e = attn::launch_fwd(a, d, causal ? attn::kMaskCausal : attn::kMaskNone, 0, cs);
   if (e != cudaSuccess) return report(ATTN_ERR_CUDA, cudaGetErrorString(e));
   if (!check) return ATTN_OK;
   int word = 0;

@@ -92,13 +92,35 @@ ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, voi
  *  test_fault: for tests of the failure path only, 0 otherwise.  1 makes every
  *      CTA withhold the copy of its first query tile, so the wait for it expires
  *      after timeout_ns: the kernel records ATTN_ERR_TIMEOUT, drains its other
- *      copies, frees its tensor memory and returns (outputs undefined). */
+ *      copies, frees its tensor memory and returns (outputs undefined).
+ *  has_window, window_left, window_right: the mask hook.  When has_window is
+ *      nonzero, key j is visible to query i (indices local to the sequence) only
+ *      if i - window_left <= j <= i + window_right; a negative bound leaves that
+ *      side open, and the causal flag still applies on top (it forces
+ *      window_right to 0).  Key tiles that no row of a query tile can see are
+ *      skipped, not masked.  Every row keeps its own key visible, so no row is
+ *      empty.  The pages name FlexAttention's masks as the interface FA4 serves
+ *      ("FlashAttention V4 deep-dive", section 5; FA-4 summary [27]) but define
+ *      no mask beyond causal: the sliding window (local attention) is this
+ *      library's instance of that interface.  The stats counters are not kept
+ *      under a window.
+ *  exp_poly_per8: how many of every 8 (even, odd) column pairs of a score row are
+ *      exponentiated by the FMA-pipe polynomial instead of MUFU ex2
+ *      ("FlashAttention V4 deep-dive", section 3.2: software exp on the FMA
+ *      units).  0 (the default, all MUFU), 2 or 8; other values are rejected
+ *      (ATTN_ERR_INVALID_ARG).  The polynomial has a relative error below 7.5e-5,
+ *      under half a bf16 ulp, so the results differ from the MUFU path only by
+ *      the rounding of P~. */
 typedef struct {
   float rescale_threshold;
   unsigned long long* stats;
   uint64_t timeout_ns;
   int64_t total_tokens;
   int test_fault;
+  int has_window;
+  int window_left;
+  int window_right;
+  int exp_poly_per8;
 } attn_fwd_opts_t;
 
 /* attn_fwd with options (opts may be NULL = defaults). */

@@ -203,10 +203,12 @@ def _sample_rows(lengths, H, n, seed):
     return np.array(rows), np.array(heads), cu
 
 
-@pytest.mark.parametrize("name", ["B1-H1-N256-d64", "B4-H16-N2048-d128",
-                                  "B4-H16-N2048-d128-qx4", "B2-H16-N8192-d128-causal",
-                                  "varlen16-H16-d128-causal"])
-def test_fwd_full_workload_sampled(name):
+@pytest.mark.parametrize("name,poly", [("B1-H1-N256-d64", 0), ("B4-H16-N2048-d128", 0),
+                                       ("B4-H16-N2048-d128", 2), ("B4-H16-N2048-d128-qx4", 0),
+                                       ("B2-H16-N8192-d128-causal", 0),
+                                       ("varlen16-H16-d128-causal", 0),
+                                       ("B2-H16-N8192-d128-causal-win1024", 0)])
+def test_fwd_full_workload_sampled(name, poly):
     ea = _lib()
     w = ai.ALL[name]
     q, k, v = ai.make_qkv(w)
@@ -215,7 +217,8 @@ def test_fwd_full_workload_sampled(name):
     if w.varlen:
         cu_t = torch.tensor(w.cu_seqlens(), dtype=torch.int32, device=DEV)
     o, lse = ea.fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=w.causal, scale=scale,
-                    cu_seqlens=cu_t, max_seqlen=w.N if w.varlen else None)
+                    cu_seqlens=cu_t, max_seqlen=w.N if w.varlen else None, window=w.window,
+                    exp_poly_per8=poly)
     ea.get_device_status()
     o = o.cpu().reshape(-1, w.H, w.d)
     lse = lse.cpu()
@@ -224,7 +227,7 @@ def test_fwd_full_workload_sampled(name):
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
     rows, heads, cu = _sample_rows(w.seq_lengths(), w.H, 192, seed=len(name))
     qp, kp, vp = (t.reshape(-1, w.H, w.d) for t in (q, k, v))
-    o_ref, l_ref = oracle.fwd_rows(qp, kp, vp, cu, w.causal, scale, rows, heads)
+    o_ref, l_ref = oracle.fwd_rows(qp, kp, vp, cu, w.causal, scale, rows, heads, window=w.window)
     compare_o(o[rows, heads], o_ref, name)
     compare_lse(lse[heads, rows], l_ref, name)
 
