@@ -20,13 +20,17 @@
 //   conditional rescale: only when m exceeds the reference maximum by > tau
 //       ("FlashAttention V4 deep-dive", section 3.2; "FlashAttention 1-4 详解",
 //        FlashAttention 4 / 三项核心技术 (2)): O_s, l scaled by 2^(m_ref - m)
-//   P~  = 2^(scale*S*log2e - m_ref)    MUFU ex2; l += sum P~ (fp32, before rounding)
+//   P~  = 2^(scale*S*log2e - m_ref)    MUFU ex2, or for POLY of every 8 column pairs
+//       the FMA-pipe polynomial ("FlashAttention V4 deep-dive", section 3.2);
+//       l += sum P~ (fp32, before rounding)
 //   P~ -> bf16, written back over S_s in TMEM
 //   O_s += P~ V_j                      tcgen05.mma, A = P~ from TMEM, B = V from smem
 // after the last key tile: O = O_s / l -> bf16 -> global; LSE = ln2*(m_ref + log2 l).
-// Causal items skip key tiles above the diagonal ("FlashAttention 1-4 详解",
-// 其他优化 / FlashAttention 2 的工程优化) and mask the diagonal tile; packed
-// variable-length batches mask keys past the sequence end.
+// The mask hook (MaskFn below) decides which key tiles an item visits and which
+// keys of a tile are hidden: causal items skip key tiles above the diagonal
+// ("FlashAttention 1-4 详解", 其他优化 / FlashAttention 2 的工程优化) and mask the
+// diagonal tile; sliding-window items skip tiles outside the window and mask its
+// edges; packed variable-length batches mask keys past the sequence end.
 //
 // Scheduling ("FlashAttention V4 deep-dive", section 3.4 dynamic tile scheduling;
 // FlashAttention-4 summary (reportify.cn) item [14], the new tile scheduler):
