@@ -32,6 +32,7 @@ class Workload:
     lengths: Optional[List[int]] = field(default=None)  # varlen sequence lengths
     # sliding window (left, right): key j visible to query i iff i-left <= j <= i+right
     window: Optional[Tuple[int, int]] = None
+    e4m3: bool = False  # inputs quantised per tensor to E4M3 (see to_e4m3)
 
     @property
     def varlen(self) -> bool:
@@ -59,8 +60,8 @@ def varlen_lengths(n: int = 16, lo: int = 512, hi: int = 16384, seed: int = 1) -
 
 # The benchmark problems: tiny latency case, dense non-causal (and a variant with
 # Q scaled by 4 so the running maximum moves often), long causal, packed causal
-# varlen, the long causal problem under a 1024-key sliding window, and the causal
-# backward problem.
+# varlen, the long causal problem under a 1024-key sliding window, the dense and
+# long causal problems with E4M3 inputs, and the causal backward problem.
 TINY = Workload("B1-H1-N256-d64", 1, 1, 256, 64, False)
 DENSE = Workload("B4-H16-N2048-d128", 4, 16, 2048, 128, False)
 DENSE_X4 = Workload("B4-H16-N2048-d128-qx4", 4, 16, 2048, 128, False, q_mult=4.0)
@@ -68,10 +69,13 @@ CAUSAL = Workload("B2-H16-N8192-d128-causal", 2, 16, 8192, 128, True)
 _VL = varlen_lengths()
 VARLEN = Workload("varlen16-H16-d128-causal", len(_VL), 16, max(_VL), 128, True, lengths=_VL)
 WINDOW = Workload("B2-H16-N8192-d128-causal-win1024", 2, 16, 8192, 128, True, window=(1024, 0))
+DENSE_E4M3 = Workload("B4-H16-N2048-d128-e4m3", 4, 16, 2048, 128, False, e4m3=True)
+CAUSAL_E4M3 = Workload("B2-H16-N8192-d128-causal-e4m3", 2, 16, 8192, 128, True, e4m3=True)
 BWD_CAUSAL = CAUSAL  # the backward problem uses the causal forward's shapes
 BWD_NAME = CAUSAL.name + "-bwd"
 
-ALL = {w.name: w for w in (TINY, DENSE, DENSE_X4, CAUSAL, VARLEN, WINDOW)}
+ALL = {w.name: w for w in (TINY, DENSE, DENSE_X4, CAUSAL, VARLEN, WINDOW, DENSE_E4M3,
+                           CAUSAL_E4M3)}
 
 
 def make_qkv(w: Workload, seed: int = 0, with_dout: bool = False):
@@ -87,6 +91,27 @@ def make_qkv(w: Workload, seed: int = 0, with_dout: bool = False):
     if w.q_mult != 1.0:
         out[0] = (out[0].float() * w.q_mult).to(torch.bfloat16)
     return tuple(out)
+
+
+def to_e4m3(x: torch.Tensor):
+    """Per-tensor 8-bit copy of a CPU tensor for the E4M3 entry point: returns
+    (x8, scale) with x8 = e4m3(x / scale) (torch's float8_e4m3fn rounding) and
+    scale the power of two that puts max|x| just below 448, so x8 * scale is the
+    8-bit input the kernel sees (exactly representable in fp32 and fp64)."""
+    import math
+    amax = float(x.abs().max())
+    scale = 2.0 ** math.ceil(math.log2(amax / 448.0)) if amax > 0 else 1.0
+    return (x.float() / scale).to(torch.float8_e4m3fn), scale
+
+
+def make_qkv_e4m3(w: Workload, seed: int = 0):
+    """The bf16 draws of ``make_qkv`` quantised per tensor: (q8, k8, v8, scales)."""
+    out, scales = [], []
+    for t in make_qkv(w, seed):
+        t8, sc = to_e4m3(t)
+        out.append(t8)
+        scales.append(sc)
+    return out[0], out[1], out[2], tuple(scales)
 
 
 def make_custom(B: int, N: int, H: int, d: int, seed: int = 0, lengths=None, n: int = 3,

@@ -34,6 +34,11 @@ sys.path.insert(0, ROOT)
 import attn_inputs as ai  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s (bf16, d=128, 1 B200) and % of dense-BF16 tensor peak"
+METRIC_E4M3 = "attention fwd TFLOP/s (e4m3 inputs, d=128, 1 B200) and % of dense-FP8 tensor peak"
+
+
+def metric_for(w: ai.Workload) -> str:
+    return METRIC_E4M3 if w.e4m3 else METRIC
 FLUSH_BYTES = 256 << 20
 MUFU_EX2_PER_CLK_PER_SM = 16  # 4 SFU lanes per SM sub-partition, 4 sub-partitions
 
@@ -199,20 +204,33 @@ def whole_job_tflops(flops_per_step: float, steps: int, world: int, max_total_ms
 
 
 def make_inputs(w: ai.Workload, device):
-    q, k, v = ai.make_qkv(w)
+    """CPU inputs of a workload: (q, k, v, cu_seqlens); E4M3 workloads give the
+    8-bit tensors (their per-tensor scales come from e4m3_scales)."""
+    if w.e4m3:
+        q, k, v, _ = ai.make_qkv_e4m3(w)
+    else:
+        q, k, v = ai.make_qkv(w)
     cu = None
     if w.varlen:
         cu = torch.tensor(w.cu_seqlens(), dtype=torch.int32)
     return q, k, v, cu
 
 
+def e4m3_scales(w: ai.Workload):
+    return ai.make_qkv_e4m3(w)[3] if w.e4m3 else None
+
+
 def cpu_oracle_sample(w: ai.Workload, q, k, v, budget_s: float):
     """Times the fp64 oracle on whole (sequence, head) units of the workload until
-    about budget_s of CPU time is spent; returns (TFLOP/s, threads, description)."""
+    about budget_s of CPU time is spent; returns (TFLOP/s, threads, description).
+    E4M3 inputs are dequantised (x8 * scale) first, outside the timing."""
     import numpy as np
     import oracle
     lengths = w.seq_lengths()
     cu = np.concatenate([[0], np.cumsum(lengths)])
+    if w.e4m3:
+        scales = e4m3_scales(w)
+        q, k, v = (t.double() * sc for t, sc in zip((q, k, v), scales))
     qp, kp, vp = (t.reshape(-1, w.H, w.d) for t in (q, k, v))
     scale = 1.0 / math.sqrt(w.d)
     done_flops, spent, units, threads = 0.0, 0.0, 0, 0
@@ -262,7 +280,7 @@ def run_reference(args, rank, world):
             vals.append(tf)
     value = statistics.median(vals)
     ms = flops / (value * 1e12) * 1e3
-    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+    line = {"metric": metric_for(w), "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
@@ -286,7 +304,8 @@ def run_ours(args, rank, world, local):
     cu = None if cu_h is None else cu_h.to(dev)
     max_len = w.N if w.varlen else None
     scale = 1.0 / math.sqrt(w.d)
-    out = torch.empty_like(q)
+    f8 = e4m3_scales(w)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
     lse_shape = (w.H, w.total_tokens) if w.varlen else (w.B, w.H, w.N)
     lse = torch.empty(lse_shape, dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -295,7 +314,8 @@ def run_ours(args, rank, world, local):
 
     def step():
         ea.fwd(q, k, v, causal=w.causal, scale=scale, cu_seqlens=cu, max_seqlen=max_len,
-               out=out, lse=lse, window=w.window, exp_poly_per8=args.exp_poly_per8)
+               out=out, lse=lse, window=w.window, exp_poly_per8=args.exp_poly_per8,
+               e4m3_scales=f8)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -319,7 +339,11 @@ def run_ours(args, rank, world, local):
     ms_per_step = total_ms / args.steps
     value = whole_job_tflops(flops, args.steps, world, total_ms)
     achieved = flops / (statistics.mean(times) / 1e3) / 1e12  # per launch, this rank
-    peak = peaks["bf16_tflops"]
+    # An E4M3 contraction's peak: the measured bf16 burst peak x the nominal 2x
+    # ratio of dense FP8 to BF16 tensor throughput.
+    peak = peaks["bf16_tflops"] * (2.0 if w.e4m3 else 1.0)
+    peak_source = (f"bf16_tflops (burst) x 2 (nominal e4m3/bf16), {peaks['source']}" if w.e4m3
+                   else f"bf16_tflops (burst), {peaks['source']}")
     clk = clocks.summary()
     mhz = clk["sm_mhz"] or peaks["sm_max_mhz"]
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -337,7 +361,7 @@ def run_ours(args, rank, world, local):
     for _ in range(2):
         ea.fwd_from_host(q_p, k_p, v_p, causal=w.causal, scale=scale, cu_seqlens_host=cu_p,
                          max_seqlen=max_len, out_host=o_host, lse_host=l_host, window=w.window,
-                         exp_poly_per8=args.exp_poly_per8)
+                         exp_poly_per8=args.exp_poly_per8, e4m3_scales=f8)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -346,11 +370,11 @@ def run_ours(args, rank, world, local):
         o_h, l_h = ea.fwd_from_host(q_p, k_p, v_p, causal=w.causal, scale=scale,
                                     cu_seqlens_host=cu_p, max_seqlen=max_len,
                                     out_host=o_host, lse_host=l_host, window=w.window,
-                                    exp_poly_per8=args.exp_poly_per8)
+                                    exp_poly_per8=args.exp_poly_per8, e4m3_scales=f8)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
-    h2d = 3 * q_h.numel() * 2 + (0 if cu_h is None else cu_h.numel() * 4)
+    h2d = 3 * q_h.numel() * q_h.element_size() + (0 if cu_h is None else cu_h.numel() * 4)
     d2h = o_h.numel() * 2 + l_h.numel() * 4
     barrier(world)
 
@@ -360,15 +384,15 @@ def run_ours(args, rank, world, local):
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        line = {"metric": metric_for(w), "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16", "data": "synthetic",
+                "dtype": "e4m3" if w.e4m3 else "bf16", "data": "synthetic",
                 "config": dict(bench_config(w, world), exp_poly_per8=args.exp_poly_per8),
                 "pct_of_peak": 100.0 * achieved / peak,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                              "unit": "TFLOP/s", "frac": achieved / peak,
-                             "peak_source": f"bf16_tflops (burst), {peaks['source']}",
+                             "peak_source": peak_source,
                              "traffic": profiled_traffic(w.name),
                              "traffic_unit": "bytes per launch (ncu dram read+write)"},
                 "mufu": {"achieved_ex2_per_s": mufu_achieved, "peak_ex2_per_s": mufu_peak,

@@ -25,7 +25,8 @@ ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_WORKSPACE = 3, 4, 5
 # Every symbol include/attn.h and include/attn_selftest.h declare.
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_ex", "attn_bwd", "attn_bwd_workspace_size",
                     "attn_get_device_status", "attn_status_string", "attn_last_error",
-                    "attn_selftest_umma", "attn_fwd_noalloc")
+                    "attn_selftest_umma", "attn_fwd_noalloc", "attn_fwd_e4m3",
+                    "attn_selftest_umma_e4m3")
 
 
 class AttnError(RuntimeError):
@@ -77,6 +78,11 @@ def load_library(path: str = LIB_PATH):
     lib.attn_last_error.restype = ctypes.c_char_p
     lib.attn_selftest_umma.argtypes = [vp, vp, vp, vp, vp, ci, vp]
     lib.attn_selftest_umma.restype = ci
+    lib.attn_selftest_umma_e4m3.argtypes = [vp, vp, vp, vp, vp, vp]
+    lib.attn_selftest_umma_e4m3.restype = ci
+    lib.attn_fwd_e4m3.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, cf, cf, cf, vp,
+                                  ctypes.POINTER(FwdOpts), vp]
+    lib.attn_fwd_e4m3.restype = ci
     lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp,
                                      ctypes.c_int64, ci, vp]
     lib.attn_fwd_noalloc.restype = ci
@@ -118,7 +124,9 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         stats: Optional[torch.Tensor] = None, timeout_ns: int = 0,
         stream: Optional[torch.cuda.Stream] = None,
         test_fault: int = 0, window: Optional[Tuple[int, int]] = None,
-        exp_poly_per8: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+        exp_poly_per8: int = 0,
+        e4m3_scales: Optional[Tuple[float, float, float]] = None
+        ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Exact attention forward on the GPU.
 
     Dense: q, k, v are bf16 ``[B, N, H, d]``; returns O ``[B, N, H, d]`` and LSE
@@ -128,10 +136,14 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     ``window = (left, right)`` keeps key j for query i only if
     ``i - left <= j <= i + right`` (negative = open side).  ``exp_poly_per8``
     (0, 2 or 8) moves that many of every 8 exponential pairs to the FMA pipe.
+    ``e4m3_scales = (q_scale, k_scale, v_scale)`` selects the 8-bit entry point
+    ``attn_fwd_e4m3``: q, k, v are then ``torch.float8_e4m3fn`` holding the real
+    inputs divided by those per-tensor scales; O is still bf16.
     """
     lib = load_library()
+    in_dtype = torch.bfloat16 if e4m3_scales is None else torch.float8_e4m3fn
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n)
+        _need(t, n, in_dtype)
     if k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must have the same shape")
     d = q.shape[-1]
@@ -160,7 +172,7 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         lse_shape = (H, q.shape[0])
         opts.total_tokens = q.shape[0]
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     else:
         _need(out, "out")
         if out.shape != q.shape:
@@ -173,11 +185,17 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
             raise ValueError("lse has the wrong shape")
     if cu_seqlens is not None and q.shape[0] == 0:
         return out, lse
+    cu_ptr = None if cu_seqlens is None else cu_seqlens.data_ptr()
     with torch.cuda.device(q.device):
-        st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                             lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
-                             None if cu_seqlens is None else cu_seqlens.data_ptr(),
-                             ctypes.byref(opts), _stream_ptr(stream))
+        if e4m3_scales is None:
+            st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                 cu_ptr, ctypes.byref(opts), _stream_ptr(stream))
+        else:
+            qs, ks, vs = (float(x) for x in e4m3_scales)
+            st = lib.attn_fwd_e4m3(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                   qs, ks, vs, cu_ptr, ctypes.byref(opts), _stream_ptr(stream))
     _check(st)
     return out, lse
 
@@ -197,7 +215,8 @@ def fwd_from_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tens
                   stream: Optional[torch.cuda.Stream] = None,
                   out_host: Optional[torch.Tensor] = None,
                   lse_host: Optional[torch.Tensor] = None,
-                  window: Optional[Tuple[int, int]] = None, exp_poly_per8: int = 0):
+                  window: Optional[Tuple[int, int]] = None, exp_poly_per8: int = 0,
+                  e4m3_scales: Optional[Tuple[float, float, float]] = None):
     """End-to-end call from host tensors: copies Q/K/V (and cu_seqlens) to the
     device, runs the forward, copies O and LSE back into host tensors (``out_host``
     / ``lse_host`` if given, ideally pinned; else new pinned tensors).  Returns
@@ -209,7 +228,8 @@ def fwd_from_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tens
         v = v_host.to(device, non_blocking=True)
         cu = None if cu_seqlens_host is None else cu_seqlens_host.to(device, non_blocking=True)
         o, lse = fwd(q, k, v, causal=causal, scale=scale, cu_seqlens=cu, max_seqlen=max_seqlen,
-                     stream=s, window=window, exp_poly_per8=exp_poly_per8)
+                     stream=s, window=window, exp_poly_per8=exp_poly_per8,
+                     e4m3_scales=e4m3_scales)
         o_h = out_host if out_host is not None else torch.empty(o.shape, dtype=o.dtype,
                                                                 pin_memory=True)
         l_h = lse_host if lse_host is not None else torch.empty(lse.shape, dtype=lse.dtype,
@@ -284,6 +304,21 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse:
 def get_device_status(stream: Optional[torch.cuda.Stream] = None) -> None:
     """Synchronises the stream; raises AttnError if a kernel recorded an error."""
     _check(load_library().attn_get_device_status(_stream_ptr(stream)))
+
+
+def selftest_umma_e4m3(a: torch.Tensor, b: torch.Tensor, v: torch.Tensor):
+    """The one-tile check of the 8-bit path: a, b, v are float8_e4m3fn [128, 128];
+    returns (S = A B^T, O = e4m3(S) V), fp32."""
+    for t, n in ((a, "a"), (b, "b"), (v, "v")):
+        _need(t, n, torch.float8_e4m3fn)
+        if tuple(t.shape) != (128, 128):
+            raise ValueError(f"{n} must be [128, 128]")
+    s_out = torch.empty((128, 128), dtype=torch.float32, device=a.device)
+    o_out = torch.empty((128, 128), dtype=torch.float32, device=a.device)
+    _check(load_library().attn_selftest_umma_e4m3(a.data_ptr(), b.data_ptr(), v.data_ptr(),
+                                                  s_out.data_ptr(), o_out.data_ptr(),
+                                                  _stream_ptr(None)))
+    return s_out, o_out
 
 
 def selftest_umma(a: torch.Tensor, b: torch.Tensor, v: torch.Tensor):

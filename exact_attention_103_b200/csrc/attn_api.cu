@@ -83,18 +83,25 @@ attn_status_t device_state(DeviceState** out) {
 
 // 3-D bf16 view {d, H, total} of a token-major [total, H, d] tensor; box
 // {64, 1, 128} (one 128-byte swizzle chunk by 128 rows), 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, int64_t total, int H, int d) {
+// A 3-D view {d, H, total} of a token-major [total, H, d] tensor of esz-byte
+// elements (2: bf16, 1: E4M3 moved as bytes); box = one 128-byte-wide chunk of
+// 128 rows, 128-byte swizzle.
+bool make_map_esz(CUtensorMap* m, const void* ptr, int64_t total, int H, int d, int esz) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(total)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(H) * d * 2};
-  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esz,
+                                 static_cast<cuuint64_t>(H) * d * esz};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz), 1, 128};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
-                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = g_encode(m, esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                              3, const_cast<void*>(ptr), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_map(CUtensorMap* m, const void* ptr, int64_t total, int H, int d) {
+  return make_map_esz(m, ptr, total, H, d, 2);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -104,12 +111,22 @@ constexpr float kDefaultTau = 8.0f;
 constexpr int kMaxVarlenB = 1024;
 constexpr int kMaxVarlenN = 131072;
 
+// Per-tensor scales of the E4M3 entry point (real value = stored value * scale).
+struct E4m3Scales {
+  float q, k, v;
+};
+
 attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                        int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
-                       int64_t total_hint, const attn_fwd_opts_t* opts, attn_stream_t stream) {
+                       int64_t total_hint, const attn_fwd_opts_t* opts, attn_stream_t stream,
+                       const E4m3Scales* f8 = nullptr) {
   if (B < 0 || H <= 0 || N < 0) return fail(ATTN_ERR_INVALID_ARG, "B=%d H=%d N=%d", B, H, N);
+  if (f8 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "E4M3 path: head dim %d (supported: 128)", d);
   if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
   if (!(std::isfinite(scale) && scale > 0.f)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (f8 && !(std::isfinite(f8->q) && f8->q > 0.f && std::isfinite(f8->k) && f8->k > 0.f &&
+              std::isfinite(f8->v) && f8->v > 0.f))
+    return fail(ATTN_ERR_INVALID_ARG, "E4M3 scales must be finite and > 0");
   if (B == 0 || N == 0) return ATTN_OK;
   if (!q || !k || !v || !o || !lse) return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
@@ -139,6 +156,9 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
     poly = opts->exp_poly_per8;
     if (poly != 0 && poly != 2 && poly != 8)
       return fail(ATTN_ERR_INVALID_ARG, "exp_poly_per8 must be 0, 2 or 8");
+    if (f8 && poly != 0) return fail(ATTN_ERR_UNSUPPORTED, "E4M3 path: exp_poly_per8 must be 0");
+    if (f8 && !(tau <= 8.f))
+      return fail(ATTN_ERR_INVALID_ARG, "E4M3 path: rescale_threshold must be <= 8 (P~ <= 256 < 448)");
     if (opts->has_window) {
       has_window = 1;
       wl = opts->window_left;
@@ -184,8 +204,9 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
 
   attn::FwdLaunch a;
   std::memset(&a, 0, sizeof(a));
-  if (!make_map(&a.tm_q, q, total, H, d) || !make_map(&a.tm_k, k, total, H, d) ||
-      !make_map(&a.tm_v, v, total, H, d))
+  const int esz = f8 ? 1 : 2;
+  if (!make_map_esz(&a.tm_q, q, total, H, d, esz) || !make_map_esz(&a.tm_k, k, total, H, d, esz) ||
+      !make_map_esz(&a.tm_v, v, total, H, d, esz))
     return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled rejected the Q/K/V views");
   a.p.o = static_cast<__nv_bfloat16*>(o);
   a.p.lse = lse;
@@ -195,7 +216,10 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   a.p.N = N;
   a.p.T = static_cast<int>(T256);
   a.p.total = static_cast<int>(total);
-  a.p.scale_log2 = scale * 1.4426950408889634f;
+  // The E4M3 scales of Q and K fold into the score scale; V's into 1/l.
+  a.p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634 *
+                                      (f8 ? static_cast<double>(f8->q) * f8->k : 1.0));
+  a.p.o_scale = f8 ? f8->v : 1.f;
   a.p.tau = tau;
   a.p.err = dev->err;
   a.p.stats = stats;
@@ -207,8 +231,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   // kernel), so up to twice as many CTAs can be useful there.
   const int64_t useful = (!varlen && mask == attn::kMaskNone) ? 2 * items_bound : items_bound;
   a.grid = static_cast<int>(useful < dev->sms ? useful : dev->sms);
-  a.smem = attn::fwd_smem_bytes(d, B, static_cast<int>(T256), varlen ? 1 : 0);
-  const cudaError_t e = attn::launch_fwd(a, d, mask, poly, cs);
+  a.smem = attn::fwd_smem_bytes(d, B, static_cast<int>(T256), varlen ? 1 : 0, f8 ? 1 : 0);
+  const cudaError_t e = attn::launch_fwd(a, d, mask, poly, f8 ? 1 : 0, cs);
   if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
   return ATTN_OK;
 }
@@ -241,6 +265,9 @@ attn_status_t load_tensor_map_encoder() {
 bool make_tensor_map(CUtensorMap* m, const void* ptr, int64_t total, int H, int d) {
   return make_map(m, ptr, total, H, d);
 }
+bool make_tensor_map_e4m3(CUtensorMap* m, const void* ptr, int64_t total, int H, int d) {
+  return make_map_esz(m, ptr, total, H, d, 1);
+}
 attn_status_t report(attn_status_t s, const char* message) { return fail(s, "%s", message); }
 }  // namespace attn_internal
 
@@ -257,6 +284,15 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
                           const attn_fwd_opts_t* opts, attn_stream_t stream) {
   const int64_t hint = (opts && opts->total_tokens > 0) ? opts->total_tokens : -1;
   return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, hint, opts, stream);
+}
+
+attn_status_t attn_fwd_e4m3(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int H, int N, int d, int causal, float scale, float q_scale,
+                            float k_scale, float v_scale, const int32_t* cu_seqlens,
+                            const attn_fwd_opts_t* opts, attn_stream_t stream) {
+  const int64_t hint = (opts && opts->total_tokens > 0) ? opts->total_tokens : -1;
+  const E4m3Scales f8{q_scale, k_scale, v_scale};
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, hint, opts, stream, &f8);
 }
 
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,

@@ -82,11 +82,14 @@ enum WaitSite {
   kSiteDrain, kSiteBadLen
 };
 
-template <int D>
+template <int D, bool F8>
 struct Layout {
-  static constexpr int TILE = kBM * D * 2;            // bytes of one 128 x D bf16 tile
-  static constexpr int CHUNK = kBM * 128;             // one 64-column swizzle chunk
-  static constexpr int NSTAGE = (D == 128) ? 4 : 8;   // K/V ring slots
+  static constexpr int ESZ = F8 ? 1 : 2;              // bytes per element (E4M3 / bf16)
+  static constexpr int TILE = kBM * D * ESZ;          // bytes of one 128 x D tile
+  static constexpr int CHUNK = kBM * 128;             // one 128-byte-wide swizzle chunk
+  static constexpr int NCHUNK = TILE / CHUNK;
+  static constexpr int KSTEP = 32 / ESZ;              // elements per MMA K step (32 bytes)
+  static constexpr int NSTAGE = (TILE <= 16384) ? 8 : 4;  // K/V ring slots
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE;
   static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE;
@@ -303,11 +306,15 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64
 
 // POLY: of every 8 consecutive (even, odd) column pairs of a score row, this many
 // are exponentiated on the FMA pipe by exp2_poly; the rest use MUFU ex2.
-template <int D, int MASK, int POLY>
+// F8: Q, K, V are E4M3 with per-tensor scales (S = Q K^T and O += P~ V with
+// tcgen05.mma kind::f8f6f4, P~ rounded to E4M3; "FlashAttention 1-4 详解", 其他优化:
+// FP8 tensor cores for the forward's matrix products).
+template <int D, int MASK, int POLY, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Lay = Layout<D>;
+  using Lay = Layout<D, F8>;
+  static_assert(!F8 || D == 128, "E4M3 path: one 128-byte row per head");
   constexpr int NS = Lay::NSTAGE;
   constexpr bool SPLIT = MASK == kMaskNone;  // the launch may hold half items
   static_assert(POLY >= 0 && POLY <= 8, "pairs per 8");
@@ -458,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P~ = 2^(s*scale*log2e - m_ref): one FMA for the argument, MUFU ex2 or the
         // FMA-pipe polynomial for the exponential, partial row sums, bf16 packing.
         const float nm = (MASK == kMaskWindow && m_ref == -INFINITY) ? 0.f : -m_ref;
-        uint32_t pk[64];
+        uint32_t pk[F8 ? 32 : 64];
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -473,10 +480,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ls[2 * (c & 1)] += a;
           ls[2 * (c & 1) + 1] += e;
-          pk[c] = pack_bf16x2(a, e);
+          if constexpr (F8) {
+            const uint32_t h = pack_e4m3x2(a, e);  // keys 2c, 2c+1: bytes 2(c&1), +1 of word c/2
+            if (c & 1) pk[c >> 1] |= h << 16; else pk[c >> 1] = h;
+          } else {
+            pk[c] = pack_bf16x2(a, e);
+          }
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        tmem_st_x64(t_s, pk);
+        if constexpr (F8) tmem_st_x32(t_s, pk); else tmem_st_x64(t_s, pk);
         // O_s is stable here: the commit that signalled S(s, j) also covers PV(s, j-1).
         if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
@@ -502,7 +514,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       o_phase ^= 1u;
       tc_fence_after();
-      const float inv = 1.f / l;
+      float inv = 1.f / l;
+      if constexpr (F8) inv *= p.o_scale;  // V's per-tensor scale
       const bool store = q_row < L;
       __nv_bfloat16* dst =
           p.o + (static_cast<int64_t>(seq_start + q_row) * p.H + h) * static_cast<int64_t>(D);
@@ -568,9 +581,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int s = 0; s < 2; ++s)
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
+          for (int c = 0; c < Lay::NCHUNK; ++c)
             tma_load_3d(sb + Lay::Q_OFF + s * Lay::TILE + c * Lay::CHUNK, &tm_q, bar(Lay::B_QFULL),
-                        c * 64, h, seq_start + it.row_base + s * kBM, pol_q);
+                        c * (128 / Lay::ESZ), h, seq_start + it.row_base + s * kBM, pol_q);
       }
       __syncwarp();
       if (!withhold) ++n_items;
@@ -586,9 +599,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (elect_one()) {
             mbar_arrive_expect_tx(bar(Lay::B_KVFULL + slot), Lay::TILE);
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c)
+            for (int c = 0; c < Lay::NCHUNK; ++c)
               tma_load_3d(sb + Lay::KV_OFF + slot * Lay::TILE + c * Lay::CHUNK, which ? &tm_v : &tm_k,
-                          bar(Lay::B_KVFULL + slot), c * 64, h, seq_start + (jlo + j) * kBN, pol_kv);
+                          bar(Lay::B_KVFULL + slot), c * (128 / Lay::ESZ), h,
+                          seq_start + (jlo + j) * kBN, pol_kv);
           }
           __syncwarp();
           ++n_ld;
@@ -608,8 +622,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // each only where tile j (j-1) lies in that sub-tile's key range.
     // S(s, j) overwrites P(s, j-1) in TMEM, which PV(s, j-1) read just before; the
     // tensor pipe executes one thread's MMAs in issue order.
-    constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0, 0);
-    constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 0, 1);
+    constexpr uint32_t idesc_s = F8 ? idesc_e4m3_f32(kBM, kBN, 0, 0) : idesc_bf16_f32(kBM, kBN, 0, 0);
+    constexpr uint32_t idesc_o = F8 ? idesc_e4m3_f32(kBM, D, 0, 1) : idesc_bf16_f32(kBM, D, 0, 1);
     const uint32_t tS0 = tmem + Lay::TM_S0, tS1 = tmem + Lay::TM_S1;
     const uint32_t tO0 = tmem + Lay::TM_O0, tO1 = tmem + Lay::TM_O1;
     uint32_t n_ld = 0, q_phase = 0, p_phase0 = 0, p_phase1 = 0;
@@ -650,11 +664,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               ph ^= 1u;
               tc_fence_after();
               const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::TILE;
+              // One K step: KSTEP keys = 32 bytes of a P~ row (8 TMEM columns) and
+              // KSTEP rows of V (128 bytes each).
 #pragma unroll
-              for (int kk = 0; kk < kBN / 16; ++kk) {
-                if (elect_one())
-                  mma_ts(tO, tS + kk * 8, sdesc_sw128(vbase + kk * 2048, Lay::CHUNK, 1024), idesc_o,
-                         (j - 1 > los || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < kBN / Lay::KSTEP; ++kk) {
+                if (elect_one()) {
+                  const uint64_t dv = sdesc_sw128(vbase + kk * Lay::KSTEP * 128, Lay::CHUNK, 1024);
+                  const uint32_t acc = (j - 1 > los || kk > 0) ? 1u : 0u;
+                  if constexpr (F8) mma_ts_f8(tO, tS + kk * 8, dv, idesc_o, acc);
+                  else mma_ts(tO, tS + kk * 8, dv, idesc_o, acc);
+                }
                 __syncwarp();
               }
               if (j == his) {
@@ -667,11 +686,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t qbase = sb + Lay::Q_OFF + s * Lay::TILE;
             const uint32_t kbase = sb + Lay::KV_OFF + slotK * Lay::TILE;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
+            for (int kk = 0; kk < D / Lay::KSTEP; ++kk) {
               const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-              if (elect_one())
-                mma_ss(tS, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
-                       idesc_s, kk > 0 ? 1u : 0u);
+              if (elect_one()) {
+                const uint64_t da = sdesc_sw128(qbase + off, 16, 1024);
+                const uint64_t db = sdesc_sw128(kbase + off, 16, 1024);
+                if constexpr (F8) mma_ss_f8(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
+                else mma_ss(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
+              }
               __syncwarp();
             }
             if (elect_one()) tc_commit(bar(Lay::B_SFULL + s));
@@ -701,19 +723,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 9) tmem_dealloc(tmem, 512);
 }
 
-template <int D>
-constexpr int smem_bytes_fixed() { return 1024 + Layout<D>::TABLE_OFF; }
+template <int D, bool F8>
+constexpr int smem_bytes_fixed() { return 1024 + Layout<D, F8>::TABLE_OFF; }
 
 }  // namespace
 
-int fwd_smem_bytes(int D, int B, int T, int varlen) {
-  const int fixed = D == 128 ? smem_bytes_fixed<128>() : smem_bytes_fixed<64>();
+int fwd_smem_bytes(int D, int B, int T, int varlen, int fp8) {
+  const int fixed = fp8 ? smem_bytes_fixed<128, true>()
+                        : (D == 128 ? smem_bytes_fixed<128, false>() : smem_bytes_fixed<64, false>());
   return fixed + (varlen ? (B + 3 * T + 1) * 4 : 0);
 }
 
-template <int D, int MASK, int POLY>
+template <int D, int MASK, int POLY, bool F8 = false>
 static cudaError_t launch_t(const FwdLaunch& a, cudaStream_t st) {
-  auto kern = fwd_kernel<D, MASK, POLY>;
+  auto kern = fwd_kernel<D, MASK, POLY, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem);
   if (e != cudaSuccess) return e;
   kern<<<a.grid, kThreads, a.smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.p);
@@ -734,7 +757,12 @@ static cudaError_t launch_m(const FwdLaunch& a, MaskKind mask, int poly, cudaStr
   return launch_p<D, kMaskNone>(a, poly, st);
 }
 
-cudaError_t launch_fwd(const FwdLaunch& a, int D, MaskKind mask, int poly, cudaStream_t st) {
+cudaError_t launch_fwd(const FwdLaunch& a, int D, MaskKind mask, int poly, int fp8, cudaStream_t st) {
+  if (fp8) {  // E4M3: d = 128, all-MUFU exponentials
+    if (mask == kMaskCausal) return launch_t<128, kMaskCausal, 0, true>(a, st);
+    if (mask == kMaskWindow) return launch_t<128, kMaskWindow, 0, true>(a, st);
+    return launch_t<128, kMaskNone, 0, true>(a, st);
+  }
   return D == 128 ? launch_m<128>(a, mask, poly, st) : launch_m<64>(a, mask, poly, st);
 }
 

@@ -30,17 +30,21 @@ struct FwdParams {
   uint64_t timeout_ns;   // limit of every internal wait
   int test_fault;        // 1: withhold the first Q copy (failure-path tests only)
   int wl, wr;            // kMaskWindow bounds, both >= 0 (an open side holds a large value)
+  float o_scale;         // E4M3 path: V's per-tensor scale, applied with 1/l
 };
 
 struct FwdLaunch {
-  CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps {D, H, total}, box {64, 1, 128}, 128B swizzle
+  // 3-D maps {D, H, total} with 128-byte swizzle; box {64, 1, 128} for bf16 and
+  // {128, 1, 128} for E4M3 (one 128-byte row either way)
+  CUtensorMap tm_q, tm_k, tm_v;
   FwdParams p;
   int grid;
   int smem;
 };
 
-int fwd_smem_bytes(int D, int B, int T, int varlen);
+int fwd_smem_bytes(int D, int B, int T, int varlen, int fp8);
 // poly: exponentials per 8 column pairs on the FMA-pipe polynomial (0, 2 or 8).
-cudaError_t launch_fwd(const FwdLaunch& a, int D, MaskKind mask, int poly, cudaStream_t st);
+// fp8: E4M3 inputs (D = 128, poly = 0 only).
+cudaError_t launch_fwd(const FwdLaunch& a, int D, MaskKind mask, int poly, int fp8, cudaStream_t st);
 
 }  // namespace attn

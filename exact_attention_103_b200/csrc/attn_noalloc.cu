@@ -135,12 +135,13 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
   a.p.test_fault = 0;
   const int64_t useful = (!varlen && !causal) ? 2 * items_bound : items_bound;
   a.grid = static_cast<int>(useful < dev->sms ? useful : dev->sms);
-  a.smem = attn::fwd_smem_bytes(d, B, static_cast<int>(T256), varlen ? 1 : 0);
+  a.p.o_scale = 1.f;
+  a.smem = attn::fwd_smem_bytes(d, B, static_cast<int>(T256), varlen ? 1 : 0, 0);
 
   // The status word must start at zero; it keeps the previous call's value otherwise.
   cudaError_t e = cudaMemsetAsync(dev->scratch, 0, kFwdScratchNeeded, cs);
   if (e != cudaSuccess) return report(ATTN_ERR_CUDA, "attn_fwd_noalloc: clearing the status word failed");
-  e = attn::launch_fwd(a, d, causal ? attn::kMaskCausal : attn::kMaskNone, 0, cs);
+  e = attn::launch_fwd(a, d, causal ? attn::kMaskCausal : attn::kMaskNone, 0, 0, cs);
   if (e != cudaSuccess) return report(ATTN_ERR_CUDA, cudaGetErrorString(e));
   if (!check) return ATTN_OK;
   int word = 0;

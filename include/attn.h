@@ -130,6 +130,27 @@ ATTN_API attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, 
                           attn_stream_t stream);
 
 /*
+ * Forward pass with 8-bit inputs ("FlashAttention 1-4 详解", section 其他优化: the
+ * forward runs its matrix products on FP8 tensor cores, the backward stays in
+ * BF16).  q, k, v: DEVICE E4M3 (1 sign, 4 exponent, 3 mantissa bits, bias 7,
+ * largest finite 448, no infinities; the encoding of torch.float8_e4m3fn), one
+ * byte per element, same layouts as attn_fwd, 16-byte aligned.  The real inputs
+ * are q * q_scale, k * k_scale, v * v_scale (per-tensor scales, finite and > 0).
+ * O is bf16 and LSE fp32 exactly as in attn_fwd (LSE of the scaled scores of the
+ * real inputs).  S = Q K^T and O += P~ V run on tcgen05.mma kind::f8f6f4; P~
+ * (<= 2^tau) is rounded to E4M3 (nearest even, saturating) for the PV product,
+ * while the row sum l adds the unrounded fp32 P~.  d must be 128
+ * (ATTN_ERR_UNSUPPORTED otherwise); opts as for attn_fwd_ex, except that
+ * exp_poly_per8 must be 0 and rescale_threshold at most 8, so that P~ <= 256 stays
+ * inside the E4M3 range.  Errors as for attn_fwd_ex.
+ */
+ATTN_API attn_status_t attn_fwd_e4m3(const void* q, const void* k, const void* v, void* o,
+                                     float* lse, int B, int H, int N, int d, int causal,
+                                     float scale, float q_scale, float k_scale, float v_scale,
+                                     const int32_t* cu_seqlens, const attn_fwd_opts_t* opts,
+                                     attn_stream_t stream);
+
+/*
  * Backward pass (dQ, dK, dV) from Q, K, V, O, LSE and dO, recomputing P from LSE
  * ("FlashAttention 1-4 详解", 总结 table: 反向传播重计算; "FlashAttention V4
  * deep-dive", section 3.3).  Same layouts as the forward; dq/dk/dv are bf16.

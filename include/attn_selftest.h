@@ -8,6 +8,11 @@
  *   O = P V with tcgen05.mma, A = P from TMEM, B = V from shared memory (MN-major).
  * a, b, v: DEVICE bf16 [128, d] (16-byte aligned); s_out: DEVICE fp32 [128, 128];
  * o_out: DEVICE fp32 [128, d]; d in {64, 128}.  Asynchronous on `stream`.
+ *
+ * attn_selftest_umma_e4m3 is the same check for the 8-bit path of attn_fwd_e4m3:
+ * a, b, v are DEVICE E4M3 [128, 128] (one byte per element), S = A B^T with
+ * tcgen05.mma kind::f8f6f4, P = e4m3(S) (round to nearest even, saturating) in
+ * TMEM, O = P V; s_out fp32 [128, 128], o_out fp32 [128, 128].
  */
 #ifndef LIBATTN_ATTN_SELFTEST_H
 #define LIBATTN_ATTN_SELFTEST_H
@@ -17,6 +22,8 @@ extern "C" {
 #endif
 ATTN_API attn_status_t attn_selftest_umma(const void* a, const void* b, const void* v, float* s_out,
                                  float* o_out, int d, attn_stream_t stream);
+ATTN_API attn_status_t attn_selftest_umma_e4m3(const void* a, const void* b, const void* v,
+                                               float* s_out, float* o_out, attn_stream_t stream);
 #ifdef __cplusplus
 }
 #endif

@@ -49,3 +49,33 @@ def compare_lse(lse_gpu, lse_ref, label: str = ""):
     err = np.abs(l - r)
     assert np.all(err <= LSE_ABS), f"{label}: LSE error {err.max():.3e} > {LSE_ABS}"
     return float(err.max())
+
+
+# E4M3 forward (attn_fwd_e4m3), against the exact attention of the dequantised
+# inputs.  The pages give no FP8 tolerance.  Reading: the 8-bit path adds one
+# rounding, P~ -> E4M3 (3 mantissa bits, nearest even), so |P8 - P~| <= 2^-4 P~
+# for P~ >= 2^-6 (normal E4M3) and the output error of row i, column c is at most
+# 2^-4 * sum_j p_ij |v_jc| = 2^-4 * A_ic, where A is the attention output with |V|
+# as values.  Added: half a bf16 ulp (O is bf16) and 2e-3 for subnormal P~ and
+# fp32 accumulation.  Relative L2: E4M3's rounding error has a relative standard
+# deviation of about 2.6% per element, which carries over to O for random V, so the
+# bar is 4e-2.  LSE comes from the fp32 scores: the bf16 bar applies.
+E4M3_REL = 2.0 ** -4
+E4M3_ABS = 2e-3
+E4M3_REL_L2 = 4e-2
+
+
+def compare_o_e4m3(o_gpu, o_ref, a_ref, label: str = ""):
+    """Asserts the E4M3 bar; a_ref is the oracle output with |V| (same shape)."""
+    o, r, a = to_np(o_gpu), to_np(o_ref), to_np(a_ref)
+    assert o.shape == r.shape == a.shape, (o.shape, r.shape, a.shape)
+    assert np.all(np.isfinite(o)), f"{label}: non-finite output"
+    err = np.abs(o - r)
+    bound = E4M3_REL * a + bf16_half_ulp(r) + E4M3_ABS
+    worst = np.argmax(err - bound)
+    assert np.all(err <= bound), (
+        f"{label}: |O-O_ref| = {err.flat[worst]:.3e} at {np.unravel_index(worst, err.shape)} "
+        f"exceeds {bound.flat[worst]:.3e} (ref {r.flat[worst]:.4f}, got {o.flat[worst]:.4f})")
+    rel = float(np.linalg.norm(o - r) / max(np.linalg.norm(r), 1e-30))
+    assert rel <= E4M3_REL_L2, f"{label}: rel-L2 {rel:.3e} > {E4M3_REL_L2}"
+    return float(err.max()), rel

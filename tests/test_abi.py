@@ -117,3 +117,15 @@ def test_backward_workspace_size(lib):
     assert lib.attn_bwd_workspace_size(2, 16, 8192, 128, 2 * 8192, 0) == 2 * 8192 * 16 * 4
     assert lib.attn_bwd_workspace_size(1, 3, 5, 64, 5, 1) == 256
     assert lib.attn_bwd_workspace_size(0, 3, 5, 64, 0, 1) == 0
+
+
+def test_e4m3_argument_checks(lib):
+    def call(d=128, qs=1.0, opts=None, B=1):
+        return lib.attn_fwd_e4m3(FAKE, FAKE, FAKE, FAKE, FAKE, B, 1, 128, d, 0, 0.1, qs, 1.0, 1.0,
+                                 None, None if opts is None else ctypes.byref(opts), None)
+    assert call(d=64) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(qs=0.0) == ea.ATTN_ERR_INVALID_ARG
+    assert call(qs=float("nan")) == ea.ATTN_ERR_INVALID_ARG
+    assert call(opts=ea.FwdOpts(-1.0, None, 0, 0, 0, 0, 0, 0, 2)) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(opts=ea.FwdOpts(9.0, None, 0, 0, 0, 0, 0, 0, 0)) == ea.ATTN_ERR_INVALID_ARG
+    assert call(B=0) == ea.ATTN_OK
