@@ -94,9 +94,10 @@ struct Layout {
   static constexpr int KV_OFF = 2 * TILE;
   static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE;
   // barrier indices
-  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_OFULL = 6,
-                       B_DRAIN = 8, B_KVFULL = 9, B_KVEMPTY = 9 + NSTAGE;
-  static constexpr int NBARS = 9 + 2 * NSTAGE;
+  // B_PFULL + 2s + h: half h (keys 64h..64h+63) of P~ of sub-tile s is in TMEM
+  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_OFULL = 8,
+                       B_DRAIN = 10, B_KVFULL = 11, B_KVEMPTY = 11 + NSTAGE;
+  static constexpr int NBARS = 11 + 2 * NSTAGE;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int TABLE_OFF = MISC_OFF + 64;
   static constexpr int TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
@@ -334,7 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(Lay::B_QEMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Lay::B_SFULL + s), 1);
-      mbar_init(bar(Lay::B_PFULL + s), 4);
+      mbar_init(bar(Lay::B_PFULL + 2 * s), 4);
+      mbar_init(bar(Lay::B_PFULL + 2 * s + 1), 4);
       mbar_init(bar(Lay::B_OFULL + s), 1);
     }
     mbar_init(bar(Lay::B_DRAIN), 1);
@@ -463,49 +465,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // P~ = 2^(s*scale*log2e - m_ref): one FMA for the argument, MUFU ex2 or the
-        // FMA-pipe polynomial for the exponential, partial row sums, bf16 packing.
+        // FMA-pipe polynomial for the exponential, partial row sums, packing.  Two
+        // halves of 64 keys: the first is stored and released to the MMA warp (the
+        // PV K steps over keys 0-63) while the second is computed.
         const float nm = (MASK == kMaskWindow && m_ref == -INFINITY) ? 0.f : -m_ref;
-        uint32_t pk[F8 ? 32 : 64];
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          float a = fmaf(__uint_as_float(sv[2 * c]), sl, nm);
-          float e = fmaf(__uint_as_float(sv[2 * c + 1]), sl, nm);
-          if ((c & 7) >= 8 - POLY) {
-            a = exp2_poly(a);
-            e = exp2_poly(e);
-          } else {
-            a = fast_exp2(a);
-            e = fast_exp2(e);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[F8 ? 16 : 32];
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) {
+            const int c = 32 * half + cc;  // column pair (keys 2c, 2c+1)
+            float a = fmaf(__uint_as_float(sv[2 * c]), sl, nm);
+            float e = fmaf(__uint_as_float(sv[2 * c + 1]), sl, nm);
+            if ((c & 7) >= 8 - POLY) {
+              a = exp2_poly(a);
+              e = exp2_poly(e);
+            } else {
+              a = fast_exp2(a);
+              e = fast_exp2(e);
+            }
+            ls[2 * (c & 1)] += a;
+            ls[2 * (c & 1) + 1] += e;
+            if constexpr (F8) {
+              const uint32_t h = pack_e4m3x2(a, e);  // bytes 2(c&1), +1 of word c/2
+              if (cc & 1) pk[cc >> 1] |= h << 16; else pk[cc >> 1] = h;
+            } else {
+              pk[cc] = pack_bf16x2(a, e);
+            }
           }
-          ls[2 * (c & 1)] += a;
-          ls[2 * (c & 1) + 1] += e;
-          if constexpr (F8) {
-            const uint32_t h = pack_e4m3x2(a, e);  // keys 2c, 2c+1: bytes 2(c&1), +1 of word c/2
-            if (c & 1) pk[c >> 1] |= h << 16; else pk[c >> 1] = h;
-          } else {
-            pk[c] = pack_bf16x2(a, e);
+          if constexpr (F8) tmem_st_x16(t_s + 16 * half, pk); else tmem_st_x32(t_s + 32 * half, pk);
+          // O_s is stable here (the commit that signalled S(s, j) also covers
+          // PV(s, j-1)); the rare rescale must land before PV(s, j) starts, i.e.
+          // before the first half is released.
+          if (half == 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t ov[32];
+              tmem_ld_x32(t_o + 32 * c, ov);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tmem_st_x32(t_o + 32 * c, ov);
+            }
           }
+          tmem_st_wait();
+          // One arrival per warp: every lane's TMEM stores are complete (wait::st)
+          // and fenced before the warp converges; lane 0 then releases them.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(Lay::B_PFULL + 2 * s + half));
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        if constexpr (F8) tmem_st_x32(t_s, pk); else tmem_st_x64(t_s, pk);
-        // O_s is stable here: the commit that signalled S(s, j) also covers PV(s, j-1).
-        if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld_x32(t_o + 32 * c, ov);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st_x32(t_o + 32 * c, ov);
-          }
-        }
-        tmem_st_wait();
-        // One arrival per warp: every lane's TMEM stores are complete (wait::st) and
-        // fenced before the warp converges; lane 0 then releases them to the MMA warp.
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(Lay::B_PFULL + s));
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
@@ -659,15 +669,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int los = s ? lo1 : lo0, his = s ? hi1 : hi0;
           if (ok && jj > 0 && j - 1 >= los && j - 1 < his) {
             uint32_t& ph = s ? p_phase1 : p_phase0;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_PFULL + s), ph, wc, timeout_code(kSitePFull)));
-            if (ok) {
-              ph ^= 1u;
-              tc_fence_after();
-              const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::TILE;
-              // One K step: KSTEP keys = 32 bytes of a P~ row (8 TMEM columns) and
-              // KSTEP rows of V (128 bytes each).
+            const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::TILE;
+            constexpr int NK = kBN / Lay::KSTEP;  // PV K steps per key tile
+            // Each half of P~ (keys 0-63, then 64-127) is multiplied as soon as the
+            // softmax warps release it.  One K step: KSTEP keys = 32 bytes of a P~
+            // row (8 TMEM columns) and KSTEP rows of V (128 bytes each).
 #pragma unroll
-              for (int kk = 0; kk < kBN / Lay::KSTEP; ++kk) {
+            for (int half = 0; half < 2 && ok; ++half) {
+              ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_PFULL + 2 * s + half), ph, wc,
+                                                     timeout_code(kSitePFull)));
+              if (!ok) break;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = half * NK / 2; kk < (half + 1) * NK / 2; ++kk) {
                 if (elect_one()) {
                   const uint64_t dv = sdesc_sw128(vbase + kk * Lay::KSTEP * 128, Lay::CHUNK, 1024);
                   const uint32_t acc = (j - 1 > los || kk > 0) ? 1u : 0u;
@@ -676,6 +690,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
               }
+            }
+            if (ok) {
+              ph ^= 1u;
               if (j == his) {
                 if (elect_one()) tc_commit(bar(Lay::B_OFULL + s));
                 __syncwarp();
