@@ -56,6 +56,14 @@ constexpr int kThreads = 320;
 constexpr int kBM = 128;  // query rows per sub-tile
 constexpr int kBN = 128;  // keys per key tile
 constexpr float kLn2 = 0.693147180559945309f;
+// P~ of a key tile is handed to the PV product in this many parts of 128/kPSplit keys.
+// Measured on B200 (same-box A/B): 2 is fastest; against 1, dense +6% and causal +1%;
+// 4 costs 8% (four release round trips per tile outweigh the earlier start).
+#ifndef ATTN_P_SPLIT
+#define ATTN_P_SPLIT 2
+#endif
+constexpr int kPSplit = ATTN_P_SPLIT;
+static_assert(kPSplit == 1 || kPSplit == 2 || kPSplit == 4, "P~ split");
 
 // 2^y without MUFU: j = round(y) by the 1.5*2^23 trick, f = y - j in [-1/2, 1/2],
 // p(f) ~ 2^f (minimax, exp2_poly.h), then 2^j is added to the exponent field as an
@@ -94,10 +102,11 @@ struct Layout {
   static constexpr int KV_OFF = 2 * TILE;
   static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE;
   // barrier indices
-  // B_PFULL + 2s + h: half h (keys 64h..64h+63) of P~ of sub-tile s is in TMEM
-  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_OFULL = 8,
-                       B_DRAIN = 10, B_KVFULL = 11, B_KVEMPTY = 11 + NSTAGE;
-  static constexpr int NBARS = 11 + 2 * NSTAGE;
+  // B_PFULL + kPSplit*s + h: part h of P~ of sub-tile s is in TMEM
+  static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4,
+                       B_OFULL = 4 + 2 * kPSplit, B_DRAIN = B_OFULL + 2, B_KVFULL = B_DRAIN + 1,
+                       B_KVEMPTY = B_KVFULL + NSTAGE;
+  static constexpr int NBARS = B_KVEMPTY + NSTAGE;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int TABLE_OFF = MISC_OFF + 64;
   static constexpr int TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
@@ -335,8 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(Lay::B_QEMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Lay::B_SFULL + s), 1);
-      mbar_init(bar(Lay::B_PFULL + 2 * s), 4);
-      mbar_init(bar(Lay::B_PFULL + 2 * s + 1), 4);
+      for (int h = 0; h < kPSplit; ++h) mbar_init(bar(Lay::B_PFULL + kPSplit * s + h), 4);
       mbar_init(bar(Lay::B_OFULL + s), 1);
     }
     mbar_init(bar(Lay::B_DRAIN), 1);
@@ -465,17 +473,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // P~ = 2^(s*scale*log2e - m_ref): one FMA for the argument, MUFU ex2 or the
-        // FMA-pipe polynomial for the exponential, partial row sums, packing.  Two
-        // halves of 64 keys: the first is stored and released to the MMA warp (the
-        // PV K steps over keys 0-63) while the second is computed.
+        // FMA-pipe polynomial for the exponential, partial row sums, packing.  In
+        // kPSplit parts: each is stored and released to the MMA warp (the PV K steps
+        // over its keys) while the next is computed.
         const float nm = (MASK == kMaskWindow && m_ref == -INFINITY) ? 0.f : -m_ref;
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[F8 ? 16 : 32];
+        for (int half = 0; half < kPSplit; ++half) {
+          constexpr int PAIRS = 64 / kPSplit;  // column pairs per part
+          uint32_t pk[F8 ? PAIRS / 2 : PAIRS];
 #pragma unroll
-          for (int cc = 0; cc < 32; ++cc) {
-            const int c = 32 * half + cc;  // column pair (keys 2c, 2c+1)
+          for (int cc = 0; cc < PAIRS; ++cc) {
+            const int c = PAIRS * half + cc;  // column pair (keys 2c, 2c+1)
             float a = fmaf(__uint_as_float(sv[2 * c]), sl, nm);
             float e = fmaf(__uint_as_float(sv[2 * c + 1]), sl, nm);
             if ((c & 7) >= 8 - POLY) {
@@ -494,18 +503,37 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[cc] = pack_bf16x2(a, e);
             }
           }
-          if constexpr (F8) tmem_st_x16(t_s + 16 * half, pk); else tmem_st_x32(t_s + 32 * half, pk);
+          if constexpr (F8) {
+            if constexpr (PAIRS == 64) tmem_st_x32(t_s, pk);
+            else if constexpr (PAIRS == 32) tmem_st_x16(t_s + 16 * half, pk);
+            else tmem_st_x8(t_s + 8 * half, pk);
+          } else {
+            if constexpr (PAIRS == 64) tmem_st_x64(t_s, pk);
+            else if constexpr (PAIRS == 32) tmem_st_x32(t_s + 32 * half, pk);
+            else tmem_st_x16(t_s + 16 * half, pk);
+          }
           // O_s is stable here (the commit that signalled S(s, j) also covers
           // PV(s, j-1)); the rare rescale must land before PV(s, j) starts, i.e.
           // before the first half is released.
           if (half == 0 && __any_sync(0xffffffffu, need)) {
+            if constexpr (kPSplit <= 2) {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t ov[32];
-              tmem_ld_x32(t_o + 32 * c, ov);
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t ov[32];
+                tmem_ld_x32(t_o + 32 * c, ov);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-              tmem_st_x32(t_o + 32 * c, ov);
+                for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                tmem_st_x32(t_o + 32 * c, ov);
+              }
+            } else {  // most of the score row is still live: small chunks
+#pragma unroll 1
+              for (int c = 0; c < D / 8; ++c) {
+                uint32_t ov[8];
+                tmem_ld_x8(t_o + 8 * c, ov);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                tmem_st_x8(t_o + 8 * c, ov);
+              }
             }
           }
           tmem_st_wait();
@@ -513,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // and fenced before the warp converges; lane 0 then releases them.
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(Lay::B_PFULL + 2 * s + half));
+          if (lane == 0) mbar_arrive(bar(Lay::B_PFULL + kPSplit * s + half));
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       }
@@ -671,17 +699,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t& ph = s ? p_phase1 : p_phase0;
             const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::TILE;
             constexpr int NK = kBN / Lay::KSTEP;  // PV K steps per key tile
-            // Each half of P~ (keys 0-63, then 64-127) is multiplied as soon as the
-            // softmax warps release it.  One K step: KSTEP keys = 32 bytes of a P~
-            // row (8 TMEM columns) and KSTEP rows of V (128 bytes each).
+            // Each part of P~ is multiplied as soon as the softmax warps release it.
+            // One K step: KSTEP keys = 32 bytes of a P~ row (8 TMEM columns) and
+            // KSTEP rows of V (128 bytes each).
+            static_assert(NK % kPSplit == 0, "K steps per part");
 #pragma unroll
-            for (int half = 0; half < 2 && ok; ++half) {
-              ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_PFULL + 2 * s + half), ph, wc,
+            for (int half = 0; half < kPSplit && ok; ++half) {
+              ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_PFULL + kPSplit * s + half), ph, wc,
                                                      timeout_code(kSitePFull)));
               if (!ok) break;
               tc_fence_after();
 #pragma unroll
-              for (int kk = half * NK / 2; kk < (half + 1) * NK / 2; ++kk) {
+              for (int kk = half * NK / kPSplit; kk < (half + 1) * NK / kPSplit; ++kk) {
                 if (elect_one()) {
                   const uint64_t dv = sdesc_sw128(vbase + kk * Lay::KSTEP * 128, Lay::CHUNK, 1024);
                   const uint32_t acc = (j - 1 > los || kk > 0) ? 1u : 0u;
