@@ -48,8 +48,9 @@ struct BwdLayout {
   static constexpr int VEC_OFF = STAGE_OFF + NSTAGE * 2 * TILE;
   static constexpr int BAR_OFF = VEC_OFF + NSTAGE * 2 * kTile * 4;
   // barrier indices
+  // B_S: S (or S^T) is in TMEM region A; B_DP: dP (or dP^T) is in region B.
   static constexpr int B_RES = 0, B_FULL = 1, B_EMPTY = 3, B_S = 5, B_P = 6, B_DS = 7, B_ACC = 8,
-                       B_DRAIN = 9, NBARS = 10;
+                       B_DRAIN = 9, B_DP = 10, NBARS = 11;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM = MISC_OFF + 64;
   // TMEM columns: region A (S^T or S, then packed P^T), region B (dP^T or dP,
@@ -123,18 +124,20 @@ __device__ __forceinline__ void store_half_row(uint32_t t_acc, __nv_bfloat16* ds
 }
 
 // Shared set-up of both main kernels: barriers, TMEM (512 columns), abort flag.
+// full_arrivals: arrivals that complete a ring stage (besides its bytes).
 template <int D>
-__device__ __forceinline__ uint32_t bwd_setup(uint8_t* smem, uint32_t sb, int warp) {
+__device__ __forceinline__ uint32_t bwd_setup(uint8_t* smem, uint32_t sb, int warp, int full_arrivals) {
   using Lay = BwdLayout<D>;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
   if (threadIdx.x == 0) {
     auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
     mbar_init(bar(Lay::B_RES), 1);
     for (int s = 0; s < Lay::NSTAGE; ++s) {
-      mbar_init(bar(Lay::B_FULL + s), 1);
+      mbar_init(bar(Lay::B_FULL + s), full_arrivals);
       mbar_init(bar(Lay::B_EMPTY + s), 1);
     }
     mbar_init(bar(Lay::B_S), 1);
+    mbar_init(bar(Lay::B_DP), 1);
     mbar_init(bar(Lay::B_P), 8);
     mbar_init(bar(Lay::B_DS), 8);
     mbar_init(bar(Lay::B_ACC), 1);
@@ -213,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t tmem = bwd_setup<D>(smem, sb, warp);
+  const uint32_t tmem = bwd_setup<D>(smem, sb, warp, 2);  // copies + query vectors
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
   WaitCtl wc;
   wc.abort = reinterpret_cast<volatile uint32_t*>(misc + 1);
@@ -235,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tA = tmem + lane_bits + Lay::TM_A + 64 * hf;
     const uint32_t tB = tmem + lane_bits + Lay::TM_B + 64 * hf;
     const float sl = p.scale_log2;
-    uint32_t s_phase = 0;
+    uint32_t s_phase = 0, dp_phase = 0;
     bool ok = true;
     for (int n = 0; n < nq && ok; ++n) {
       const int i = i_first + n, st = n & 1;
@@ -261,6 +264,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
       tmem_st_x32(tA, pk);
       warp_release(bar(Lay::B_P), lane);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DP), dp_phase, wc, timeout_code(kSiteS)));
+      if (!ok) break;
+      dp_phase ^= 1u;
+      tc_fence_after();
       // dS^T = P^T o (dP^T - D), in two 32-column halves to bound registers.
 #pragma unroll
       for (int q2 = 0; q2 < 2; ++q2) {
@@ -304,23 +311,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int n = 0; n < nq && ok; ++n) {
       const int i = i_first + n, st = n & 1;
+      // Per-query vectors of this tile: LSE in log2 units (+inf past the
+      // sequence, so P = 0 there) and D.  Read into registers before the stage is
+      // free, so their latency overlaps the wait and the copies.
+      float lv[kTile / 32], dv[kTile / 32];
+#pragma unroll
+      for (int u = 0; u < kTile / 32; ++u) {
+        const int qrow = i * kTile + 32 * u + lane;
+        const bool in = qrow < it.L;
+        const int64_t vi = vec_index(p, it.b, it.h, it.seq_start, in ? qrow : 0);
+        lv[u] = in ? __ldg(p.lse + vi) * kLog2e : INFINITY;
+        dv[u] = in ? __ldg(p.dpre + vi) : 0.f;
+      }
       if (n >= Lay::NSTAGE) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_EMPTY + st), ((n >> 1) - 1) & 1u, wc,
                                                timeout_code(kSiteStageEmpty)));
         if (!ok) break;
       }
-      // Per-query vectors of this tile: LSE in log2 units (+inf past the
-      // sequence, so P = 0 there) and D.
-      float* v = vec + st * 2 * kTile;
-      for (int rr = lane; rr < kTile; rr += 32) {
-        const int qrow = i * kTile + rr;
-        const bool in = qrow < it.L;
-        const int64_t vi = vec_index(p, it.b, it.h, it.seq_start, in ? qrow : 0);
-        v[rr] = in ? __ldg(p.lse + vi) * kLog2e : INFINITY;
-        v[kTile + rr] = in ? __ldg(p.dpre + vi) : 0.f;
-      }
-      __threadfence_block();
-      __syncwarp();
+      // The stage's barrier counts two arrivals: the copies' (with their bytes)
+      // and the warp's, after it has written the vectors.
       if (elect_one()) {
         mbar_arrive_expect_tx(bar(Lay::B_FULL + st), 2 * Lay::TILE);
         const uint32_t base = sb + Lay::STAGE_OFF + st * 2 * Lay::TILE;
@@ -332,7 +341,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                       it.seq_start + i * kTile, pol_ring);
         }
       }
+      float* v = vec + st * 2 * kTile;
+#pragma unroll
+      for (int u = 0; u < kTile / 32; ++u) {
+        v[32 * u + lane] = lv[u];
+        v[kTile + 32 * u + lane] = dv[u];
+      }
       __syncwarp();
+      if (lane == 0) mbar_arrive(bar(Lay::B_FULL + st));
     }
     // Drain: copies still in flight must land before the CTA exits.
     drain_wait(bar(Lay::B_RES), 0u, kDrainLimitNs);
@@ -346,14 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tdV = tmem + Lay::TM_ACC0, tdK = tmem + Lay::TM_ACC1;
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_RES), 0, wc, timeout_code(kSiteKv)));
     uint32_t p_phase = 0, ds_phase = 0;
-    for (int n = 0; n < nq && ok; ++n) {
-      const int st = n & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL + st), (n >> 1) & 1u, wc,
-                                             timeout_code(kSiteStageFull)));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t qb = sb + Lay::STAGE_OFF + st * 2 * Lay::TILE, dob = qb + Lay::TILE;
-      // S^T = K Q^T and dP^T = V dO^T (A and B K-major from shared memory).
+    auto stage_q = [&](int n) -> uint32_t { return sb + Lay::STAGE_OFF + (n & 1) * 2 * Lay::TILE; };
+    // S^T = K Q_n^T into region A (A and B K-major from shared memory).
+    auto issue_st = [&](int n) {
+      const uint32_t qb = stage_q(n);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
@@ -362,6 +374,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                  idesc_s, kk > 0 ? 1u : 0u);
         __syncwarp();
       }
+      if (elect_one()) tc_commit(bar(Lay::B_S));
+      __syncwarp();
+    };
+    // dP^T = V dO_n^T into region B.
+    auto issue_dpt = [&](int n) {
+      const uint32_t dob = stage_q(n) + Lay::TILE;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
@@ -370,8 +388,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                  idesc_s, kk > 0 ? 1u : 0u);
         __syncwarp();
       }
-      if (elect_one()) tc_commit(bar(Lay::B_S));
+      if (elect_one()) tc_commit(bar(Lay::B_DP));
       __syncwarp();
+    };
+    // Software pipeline over query tiles: per tile n the tensor pipe runs
+    //   dV(n), S^T(n+1), dK(n), dP^T(n+1)
+    // so the elementwise work on tile n+1 (exponentials) overlaps dK(n) and
+    // dP^T(n+1), and dS of tile n overlaps dV(n) and S^T(n+1).  Region A is
+    // rewritten by S^T(n+1) only after dV(n) has read P^T(n) (one issuing thread:
+    // in order), region B by dP^T(n+1) only after dK(n) has read dS^T(n).
+    if (ok && nq > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL), 0u, wc, timeout_code(kSiteStageFull)));
+      if (ok) {
+        tc_fence_after();
+        issue_st(0);
+        issue_dpt(0);
+      }
+    }
+    for (int n = 0; n < nq && ok; ++n) {
+      const int st = n & 1;
+      const uint32_t qb = stage_q(n), dob = qb + Lay::TILE;
       // dV += P^T dO (A = P^T from TMEM, B = dO MN-major).
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_P), p_phase, wc, timeout_code(kSiteP)));
       if (!ok) break;
@@ -383,6 +419,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tdV, tA + packed_col(kk), sdesc_sw128(dob + kk * 2048, Lay::CHUNK, 1024), idesc_acc,
                  (n > 0 || kk > 0) ? 1u : 0u);
         __syncwarp();
+      }
+      if (n + 1 < nq) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL + ((n + 1) & 1)), ((n + 1) >> 1) & 1u, wc,
+                                               timeout_code(kSiteStageFull)));
+        if (!ok) break;
+        tc_fence_after();
+        issue_st(n + 1);
       }
       // dK += dS^T Q (A = dS^T from TMEM, B = Q MN-major); scale applied at the end.
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DS), ds_phase, wc, timeout_code(kSiteDs)));
@@ -398,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (elect_one()) tc_commit(bar(Lay::B_EMPTY + st));
       __syncwarp();
+      if (n + 1 < nq) issue_dpt(n + 1);
     }
     if (elect_one()) {
       if (ok) tc_commit(bar(Lay::B_ACC));
@@ -432,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t tmem = bwd_setup<D>(smem, sb, warp);
+  const uint32_t tmem = bwd_setup<D>(smem, sb, warp, 1);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
   WaitCtl wc;
   wc.abort = reinterpret_cast<volatile uint32_t*>(misc + 1);
@@ -455,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t vi = vec_index(p, it.b, it.h, it.seq_start, in ? q_row : 0);
     const float lse2 = in ? __ldg(p.lse + vi) * kLog2e : INFINITY;
     const float dd = in ? __ldg(p.dpre + vi) : 0.f;
-    uint32_t s_phase = 0;
+    uint32_t s_phase = 0, dp_phase = 0;
     bool ok = true;
     for (int j = 0; j < nk && ok; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_S), s_phase, wc, timeout_code(kSiteS)));
@@ -474,6 +518,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float e = fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lse2));
         pv[c] = (c < lim) ? e : 0.f;
       }
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DP), dp_phase, wc, timeout_code(kSiteS)));
+      if (!ok) break;
+      dp_phase ^= 1u;
+      tc_fence_after();
       uint32_t pk[32];
 #pragma unroll
       for (int q2 = 0; q2 < 2; ++q2) {
@@ -539,13 +587,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tA = tmem + Lay::TM_A, tB = tmem + Lay::TM_B, tdQ = tmem + Lay::TM_ACC0;
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_RES), 0, wc, timeout_code(kSiteKv)));
     uint32_t ds_phase = 0;
-    for (int j = 0; j < nk && ok; ++j) {
-      const int st = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL + st), (j >> 1) & 1u, wc,
-                                             timeout_code(kSiteStageFull)));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t kb = sb + Lay::STAGE_OFF + st * 2 * Lay::TILE, vb = kb + Lay::TILE;
+    auto stage_k = [&](int j) -> uint32_t { return sb + Lay::STAGE_OFF + (j & 1) * 2 * Lay::TILE; };
+    // S = Q K_j^T into region A, then dP = dO V_j^T into region B, each with its
+    // own commit so the exponentials start before dP is done.
+    auto issue_s_dp = [&](int j) {
+      const uint32_t kb = stage_k(j), vb = kb + Lay::TILE;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
@@ -554,6 +600,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                  idesc_s, kk > 0 ? 1u : 0u);
         __syncwarp();
       }
+      if (elect_one()) tc_commit(bar(Lay::B_S));
+      __syncwarp();
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
@@ -562,8 +610,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                  idesc_s, kk > 0 ? 1u : 0u);
         __syncwarp();
       }
-      if (elect_one()) tc_commit(bar(Lay::B_S));
+      if (elect_one()) tc_commit(bar(Lay::B_DP));
       __syncwarp();
+    };
+    // Per key tile j the tensor pipe runs dQ(j), then S(j+1) and dP(j+1): the
+    // elementwise warps read S(j) and dP(j) before releasing dS(j), and one thread
+    // issues every MMA, so S(j+1) and dP(j+1) overwrite regions A and B only after
+    // dQ(j) has read dS(j).
+    if (ok && nk > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL), 0u, wc, timeout_code(kSiteStageFull)));
+      if (ok) {
+        tc_fence_after();
+        issue_s_dp(0);
+      }
+    }
+    for (int j = 0; j < nk && ok; ++j) {
+      const int st = j & 1;
+      const uint32_t kb = stage_k(j);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DS), ds_phase, wc, timeout_code(kSiteDs)));
       if (!ok) break;
       ds_phase ^= 1u;
@@ -578,6 +641,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (elect_one()) tc_commit(bar(Lay::B_EMPTY + st));
       __syncwarp();
+      if (j + 1 < nk) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL + ((j + 1) & 1)), ((j + 1) >> 1) & 1u, wc,
+                                               timeout_code(kSiteStageFull)));
+        if (!ok) break;
+        tc_fence_after();
+        issue_s_dp(j + 1);
+      }
     }
     if (elect_one()) {
       if (ok) tc_commit(bar(Lay::B_ACC));
