@@ -252,3 +252,44 @@ def test_wait_timeout_is_reported_and_the_context_stays_usable():
     o_ref, l_ref = _dense_ref(q, k, v, True, 1 / math.sqrt(d))
     compare_o(o.cpu(), o_ref, "after timeout")
     compare_lse(lse.cpu(), l_ref)
+
+
+# ------------------------------------------------------------ size limits
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_max_sequences(causal):
+    """B = 1024 packed sequences (the varlen limit), lengths 0..9, compared in full."""
+    ea = _lib()
+    g = torch.Generator().manual_seed(71)
+    lengths = [int(x) for x in torch.randint(0, 10, (1024,), generator=g)]
+    H, d = 2, 64
+    q, k, v = ai.make_custom(0, 0, H, d, seed=72, lengths=lengths)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = ea.fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, scale=scale,
+                    cu_seqlens=torch.from_numpy(cu).to(DEV), max_seqlen=max(lengths))
+    ea.get_device_status()
+    o_ref, lse_ref, _ = oracle.fwd(q, k, v, cu, causal, scale)
+    compare_o(o.cpu(), o_ref, f"1024 sequences causal={causal}")
+    compare_lse(lse.cpu(), lse_ref)
+
+
+def test_varlen_max_length_sampled():
+    """N = 131072 (the varlen limit): one sequence of that length plus a short one,
+    causal, compared on sampled rows."""
+    ea = _lib()
+    lengths = [131072, 77]
+    H, d = 1, 64
+    q, k, v = ai.make_custom(0, 0, H, d, seed=73, lengths=lengths)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = ea.fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, scale=scale,
+                    cu_seqlens=torch.from_numpy(cu).to(DEV), max_seqlen=max(lengths))
+    ea.get_device_status()
+    o, lse = o.cpu(), lse.cpu()
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    rows, heads, cu64 = _sample_rows(lengths, H, 96, seed=74)
+    rows = np.concatenate([rows, [131071, 131071 - 128, 131072, 131072 + 76]])
+    heads = np.concatenate([heads, [0, 0, 0, 0]])
+    o_ref, l_ref = oracle.fwd_rows(q, k, v, cu64, True, scale, rows, heads)
+    compare_o(o[rows, heads], o_ref, "N=131072")
+    compare_lse(lse[heads, rows], l_ref, "N=131072")
