@@ -21,7 +21,7 @@ SOURCES = ["attn_api.cu", "attn_fwd_sm100.cu", "attn_bwd_sm100.cu", "selftest_sm
 HEADERS = ["attn_fwd_sm100.h", "attn_bwd_sm100.h", "sm100_ptx.cuh", "exp2_poly.h"]
 PUBLIC_HEADERS = [os.path.join(ROOT, "include", h) for h in ("attn.h", "attn_selftest.h")]
 NVCC = os.environ.get("NVCC", "nvcc")
-# Extra nvcc flags (e.g. -DATTN_POLY_PAIRS_PER_8=4 to change the MUFU/FMA exp split).
+# Extra nvcc flags (e.g. -DATTN_P_SPLIT=4 to change how P~ is handed to the PV product).
 EXTRA = os.environ.get("ATTN_NVCC_EXTRA", "").split()
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-Xptxas", "-v",
