@@ -351,29 +351,29 @@ def run_ours(args, rank, world, local):
     mufu_share = 1.0 - args.exp_poly_per8 / 8.0
     mufu_achieved = mufu_share * workload_exps(w) / (statistics.mean(times) / 1e3)
 
-    # End to end through the public API from pinned host buffers: H2D of Q/K/V
-    # (and cu_seqlens), the forward, D2H of O and LSE, every step.
+    # End to end through the public API from pinned host buffers: every call copies
+    # its Q/K/V (and cu_seqlens) to the device, runs the forward and copies O and
+    # LSE back; HostPipeline overlaps neighbouring calls' copies with compute.
     q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
     cu_p = None if cu_h is None else cu_h.pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
     o_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     l_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    pipe = ea.HostPipeline(q_h.shape, causal=w.causal, scale=scale, cu_seqlens_host=cu_p,
+                           max_seqlen=max_len, device=str(dev), window=w.window,
+                           exp_poly_per8=args.exp_poly_per8, e4m3_scales=f8)
     for _ in range(2):
-        ea.fwd_from_host(q_p, k_p, v_p, causal=w.causal, scale=scale, cu_seqlens_host=cu_p,
-                         max_seqlen=max_len, out_host=o_host, lse_host=l_host, window=w.window,
-                         exp_poly_per8=args.exp_poly_per8, e4m3_scales=f8)
-    torch.cuda.synchronize()
+        pipe.submit(q_p, k_p, v_p, o_host, l_host)
+    pipe.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(pipe.streams[0])
     for _ in range(e2e_steps):
-        o_h, l_h = ea.fwd_from_host(q_p, k_p, v_p, causal=w.causal, scale=scale,
-                                    cu_seqlens_host=cu_p, max_seqlen=max_len,
-                                    out_host=o_host, lse_host=l_host, window=w.window,
-                                    exp_poly_per8=args.exp_poly_per8, e4m3_scales=f8)
-    e1.record()
-    torch.cuda.synchronize()
+        pipe.submit(q_p, k_p, v_p, o_host, l_host)
+    e1.record(pipe.streams[2])
+    pipe.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    o_h, l_h = o_host, l_host
     h2d = 3 * q_h.numel() * q_h.element_size() + (0 if cu_h is None else cu_h.numel() * 4)
     d2h = o_h.numel() * 2 + l_h.numel() * 4
     barrier(world)
@@ -402,7 +402,9 @@ def run_ours(args, rank, world, local):
                                  "peak = SMs x 16 ex2/clk at the median sampled SM clock"},
                 "e2e": {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                        "ms_per_step": e2e_ms},
+                        "ms_per_step": e2e_ms,
+                        "api": "HostPipeline (2 device buffer sets, copy-in / compute / "
+                               "copy-out streams)"},
                 "gpu_launches": args.steps,
                 "clocks": clk,
                 "cpu_baseline": cpu}

@@ -239,6 +239,79 @@ def fwd_from_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tens
     return o_h, l_h
 
 
+class HostPipeline:
+    """End-to-end forward from pinned host memory with the copies of neighbouring
+    calls overlapped: call k's host-to-device copy runs while call k-1 computes and
+    call k-2's results travel back, on three streams (copy in, compute, copy out)
+    ordered by events.  ``depth`` device buffer sets rotate; every call still moves
+    its own inputs to the device and its own O and LSE back.  Only plumbing lives
+    here: the attention itself is ``fwd`` (the C ABI).
+
+    ``shape``: the q/k/v shape of every call (dense ``[B,N,H,d]`` or packed
+    ``[T,H,d]``); the other arguments are those of ``fwd``.
+    """
+
+    def __init__(self, shape, causal: bool = False, scale: Optional[float] = None,
+                 cu_seqlens_host: Optional[torch.Tensor] = None, max_seqlen: Optional[int] = None,
+                 device: str = "cuda", depth: int = 2,
+                 window: Optional[Tuple[int, int]] = None, exp_poly_per8: int = 0,
+                 e4m3_scales: Optional[Tuple[float, float, float]] = None):
+        if depth < 1:
+            raise ValueError("depth must be >= 1")
+        self.dev = torch.device(device)
+        self.kw = dict(causal=causal, scale=scale, max_seqlen=max_seqlen, window=window,
+                       exp_poly_per8=exp_poly_per8, e4m3_scales=e4m3_scales)
+        self.cu_host = cu_seqlens_host
+        in_dtype = torch.bfloat16 if e4m3_scales is None else torch.float8_e4m3fn
+        shape = tuple(shape)
+        if cu_seqlens_host is None:
+            B, N, H, _ = shape
+            lse_shape = (B, H, N)
+        else:
+            lse_shape = (shape[1], shape[0])
+        self.streams = [torch.cuda.Stream(self.dev) for _ in range(3)]
+        self.slots = []
+        for _ in range(depth):
+            slot = {n: torch.empty(shape, dtype=in_dtype, device=self.dev) for n in ("q", "k", "v")}
+            slot["o"] = torch.empty(shape, dtype=torch.bfloat16, device=self.dev)
+            slot["lse"] = torch.empty(lse_shape, dtype=torch.float32, device=self.dev)
+            slot["cu"] = (None if cu_seqlens_host is None else
+                          torch.empty(cu_seqlens_host.shape, dtype=torch.int32, device=self.dev))
+            for e in ("loaded", "computed", "drained"):
+                slot[e] = torch.cuda.Event()
+            self.slots.append(slot)
+        self.calls = 0
+
+    def submit(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
+               out_host: torch.Tensor, lse_host: torch.Tensor) -> torch.cuda.Event:
+        """Queues one call; returns the event after which out_host / lse_host hold it."""
+        h2d, comp, d2h = self.streams
+        slot = self.slots[self.calls % len(self.slots)]
+        self.calls += 1
+        h2d.wait_event(slot["computed"])  # the slot's previous inputs have been read
+        with torch.cuda.stream(h2d):
+            for n, t in (("q", q_host), ("k", k_host), ("v", v_host)):
+                slot[n].copy_(t, non_blocking=True)
+            if slot["cu"] is not None:
+                slot["cu"].copy_(self.cu_host, non_blocking=True)
+            slot["loaded"].record(h2d)
+        comp.wait_event(slot["loaded"])
+        comp.wait_event(slot["drained"])  # the slot's previous outputs have left
+        fwd(slot["q"], slot["k"], slot["v"], cu_seqlens=slot["cu"], out=slot["o"],
+            lse=slot["lse"], stream=comp, **self.kw)
+        slot["computed"].record(comp)
+        d2h.wait_event(slot["computed"])
+        with torch.cuda.stream(d2h):
+            out_host.copy_(slot["o"], non_blocking=True)
+            lse_host.copy_(slot["lse"], non_blocking=True)
+            slot["drained"].record(d2h)
+        return slot["drained"]
+
+    def synchronize(self) -> None:
+        for st in self.streams:
+            st.synchronize()
+
+
 def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                 lse: torch.Tensor, causal: bool = False, scale: Optional[float] = None,
                 cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: Optional[int] = None,

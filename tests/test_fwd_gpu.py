@@ -293,3 +293,34 @@ def test_varlen_max_length_sampled():
     o_ref, l_ref = oracle.fwd_rows(q, k, v, cu64, True, scale, rows, heads)
     compare_o(o[rows, heads], o_ref, "N=131072")
     compare_lse(lse[heads, rows], l_ref, "N=131072")
+
+
+@pytest.mark.parametrize("varlen", [False, True])
+def test_host_pipeline_matches_fwd(varlen):
+    """Four calls through the overlapped host pipeline (two device buffer sets, so
+    buffers are reused while neighbouring calls are in flight) give exactly the
+    results of plain device calls."""
+    ea = _lib()
+    H, d = 2, 128
+    lengths = [300, 5, 700] if varlen else None
+    cu = None if lengths is None else torch.tensor(np.concatenate([[0], np.cumsum(lengths)]),
+                                                   dtype=torch.int32)
+    inputs = [ai.make_custom(2, 640, H, d, seed=80 + i, lengths=lengths) for i in range(4)]
+    shape = inputs[0][0].shape
+    pipe = ea.HostPipeline(shape, causal=True, cu_seqlens_host=None if cu is None else cu.pin_memory(),
+                           max_seqlen=max(lengths) if varlen else None)
+    outs = []
+    for q, k, v in inputs:
+        o_h = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+        lse_shape = (H, shape[0]) if varlen else (shape[0], H, shape[1])
+        l_h = torch.empty(lse_shape, dtype=torch.float32, pin_memory=True)
+        pipe.submit(q.pin_memory(), k.pin_memory(), v.pin_memory(), o_h, l_h)
+        outs.append((o_h, l_h))
+    pipe.synchronize()
+    ea.get_device_status()
+    for (q, k, v), (o_h, l_h) in zip(inputs, outs):
+        o, lse = ea.fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=True,
+                        cu_seqlens=None if cu is None else cu.to(DEV),
+                        max_seqlen=max(lengths) if varlen else None)
+        ea.get_device_status()
+        assert torch.equal(o.cpu(), o_h) and torch.equal(lse.cpu(), l_h)
