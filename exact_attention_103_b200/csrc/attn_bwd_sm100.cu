@@ -48,14 +48,17 @@ struct BwdLayout {
   static constexpr int VEC_OFF = STAGE_OFF + NSTAGE * 2 * TILE;
   static constexpr int BAR_OFF = VEC_OFF + NSTAGE * 2 * kTile * 4;
   // barrier indices
-  // B_S: S (or S^T) is in TMEM region A; B_DP: dP (or dP^T) is in region B.
+  // B_S: S (or S^T) is in TMEM region A (B_S1: in region A', the dQ kernel's
+  // second score buffer); B_DP: dP (or dP^T) is in region B.
   static constexpr int B_RES = 0, B_FULL = 1, B_EMPTY = 3, B_S = 5, B_P = 6, B_DS = 7, B_ACC = 8,
-                       B_DRAIN = 9, B_DP = 10, NBARS = 11;
+                       B_DRAIN = 9, B_DP = 10, B_S1 = 11, NBARS = 12;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM = MISC_OFF + 64;
   // TMEM columns: region A (S^T or S, then packed P^T), region B (dP^T or dP,
-  // then packed dS), accumulators.
-  static constexpr int TM_A = 0, TM_B = 128, TM_ACC0 = 256, TM_ACC1 = 256 + D;
+  // then packed dS), accumulators.  The dQ kernel has one accumulator and uses
+  // the second one's columns as A', a second score buffer (128 columns).
+  static constexpr int TM_A = 0, TM_B = 128, TM_ACC0 = 256, TM_ACC1 = 256 + D, TM_A2 = 256 + D;
+  static_assert(TM_A2 + kTile <= 512, "A' fits in TMEM");
 };
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -137,6 +140,7 @@ __device__ __forceinline__ uint32_t bwd_setup(uint8_t* smem, uint32_t sb, int wa
       mbar_init(bar(Lay::B_EMPTY + s), 1);
     }
     mbar_init(bar(Lay::B_S), 1);
+    mbar_init(bar(Lay::B_S1), 1);
     mbar_init(bar(Lay::B_DP), 1);
     mbar_init(bar(Lay::B_P), 8);
     mbar_init(bar(Lay::B_DS), 8);
@@ -492,22 +496,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = wq * 32 + lane;
     const int q_row = i * kTile + r;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tA = tmem + lane_bits + Lay::TM_A + 64 * hf;
+    const uint32_t tA0 = tmem + lane_bits + Lay::TM_A + 64 * hf;
+    const uint32_t tA1 = tmem + lane_bits + Lay::TM_A2 + 64 * hf;
     const uint32_t tB = tmem + lane_bits + Lay::TM_B + 64 * hf;
     const float sl = p.scale_log2;
     const bool in = q_row < it.L;
     const int64_t vi = vec_index(p, it.b, it.h, it.seq_start, in ? q_row : 0);
     const float lse2 = in ? __ldg(p.lse + vi) * kLog2e : INFINITY;
     const float dd = in ? __ldg(p.dpre + vi) : 0.f;
-    uint32_t s_phase = 0, dp_phase = 0;
+    uint32_t dp_phase = 0;
     bool ok = true;
     for (int j = 0; j < nk && ok; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_S), s_phase, wc, timeout_code(kSiteS)));
+      // S of key tile j is in region A (j even) or A' (j odd); each buffer's
+      // barrier completes once per two tiles.
+      const int sb2 = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(sb2 ? Lay::B_S1 : Lay::B_S), (j >> 1) & 1u, wc,
+                                             timeout_code(kSiteS)));
       if (!ok) break;
-      s_phase ^= 1u;
       tc_fence_after();
       uint32_t sv[64];
-      tmem_ld_x64(tA, sv);
+      tmem_ld_x64(sb2 ? tA1 : tA0, sv);
       // keys visible to this row: key < L and (causal) key <= q_row
       const int kb = j * kTile + 64 * hf;
       int lim = it.L - kb;
@@ -584,24 +592,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0, 0);
     constexpr uint32_t idesc_acc = idesc_bf16_f32(kTile, D, 0, 1);
-    const uint32_t tA = tmem + Lay::TM_A, tB = tmem + Lay::TM_B, tdQ = tmem + Lay::TM_ACC0;
+    const uint32_t tB = tmem + Lay::TM_B, tdQ = tmem + Lay::TM_ACC0;
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_RES), 0, wc, timeout_code(kSiteKv)));
     uint32_t ds_phase = 0;
     auto stage_k = [&](int j) -> uint32_t { return sb + Lay::STAGE_OFF + (j & 1) * 2 * Lay::TILE; };
-    // S = Q K_j^T into region A, then dP = dO V_j^T into region B, each with its
-    // own commit so the exponentials start before dP is done.
-    auto issue_s_dp = [&](int j) {
-      const uint32_t kb = stage_k(j), vb = kb + Lay::TILE;
+    // S = Q K_j^T into region A (j even) or A' (j odd).
+    auto issue_s = [&](int j) {
+      const uint32_t kb = stage_k(j);
+      const uint32_t tS = tmem + ((j & 1) ? Lay::TM_A2 : Lay::TM_A);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
         if (elect_one())
-          mma_ss(tA, sdesc_sw128(sb + Lay::A0_OFF + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+          mma_ss(tS, sdesc_sw128(sb + Lay::A0_OFF + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
                  idesc_s, kk > 0 ? 1u : 0u);
         __syncwarp();
       }
-      if (elect_one()) tc_commit(bar(Lay::B_S));
+      if (elect_one()) tc_commit(bar((j & 1) ? Lay::B_S1 : Lay::B_S));
       __syncwarp();
+    };
+    // dP = dO V_j^T into region B, with its own commit.
+    auto issue_dp = [&](int j) {
+      const uint32_t vb = stage_k(j) + Lay::TILE;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
@@ -613,15 +625,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (elect_one()) tc_commit(bar(Lay::B_DP));
       __syncwarp();
     };
-    // Per key tile j the tensor pipe runs dQ(j), then S(j+1) and dP(j+1): the
-    // elementwise warps read S(j) and dP(j) before releasing dS(j), and one thread
-    // issues every MMA, so S(j+1) and dP(j+1) overwrite regions A and B only after
-    // dQ(j) has read dS(j).
+    // Per key tile j the tensor pipe runs dQ(j), dP(j+1), S(j+2): S(j+1) is
+    // already in the other score buffer, so the exponentials of tile j+1 start as
+    // soon as dS(j) is released.  The elementwise warps read S(j) and dP(j) before
+    // releasing dS(j), and one thread issues every MMA in order, so dP(j+1)
+    // overwrites region B only after dQ(j) has read dS(j), and S(j+2) reuses S(j)'s
+    // buffer only after that release.
+    auto wait_full = [&](int j) -> bool {
+      const bool r = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL + (j & 1)), (j >> 1) & 1u, wc,
+                                                       timeout_code(kSiteStageFull)));
+      if (r) tc_fence_after();
+      return r;
+    };
     if (ok && nk > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL), 0u, wc, timeout_code(kSiteStageFull)));
+      ok = wait_full(0);
       if (ok) {
-        tc_fence_after();
-        issue_s_dp(0);
+        issue_s(0);
+        issue_dp(0);
+      }
+      if (ok && nk > 1) {
+        ok = wait_full(1);
+        if (ok) issue_s(1);
       }
     }
     for (int j = 0; j < nk && ok; ++j) {
@@ -641,12 +665,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (elect_one()) tc_commit(bar(Lay::B_EMPTY + st));
       __syncwarp();
-      if (j + 1 < nk) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL + ((j + 1) & 1)), ((j + 1) >> 1) & 1u, wc,
-                                               timeout_code(kSiteStageFull)));
+      if (j + 1 < nk) issue_dp(j + 1);  // stage (j+1) was waited for before S(j+1)
+      if (j + 2 < nk) {
+        ok = wait_full(j + 2);
         if (!ok) break;
-        tc_fence_after();
-        issue_s_dp(j + 1);
+        issue_s(j + 2);
       }
     }
     if (elect_one()) {
