@@ -246,12 +246,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int n = 0; n < nq && ok; ++n) {
       const int i = i_first + n, st = n & 1;
-      const float* lse2 = vec + st * 2 * kTile + 64 * hf;
-      const float* dd = lse2 + kTile;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_S), s_phase, wc, timeout_code(kSiteS)));
       if (!ok) break;
       s_phase ^= 1u;
       tc_fence_after();
+      // The 64 query columns' LSE2 and D (written before S^T(n) was issued): lane l
+      // holds entries 2l, 2l+1 and the warp broadcasts them by shuffles.
+      const float2 my_l = reinterpret_cast<const float2*>(vec + st * 2 * kTile + 64 * hf)[lane];
+      const float2 my_d = reinterpret_cast<const float2*>(vec + st * 2 * kTile + kTile + 64 * hf)[lane];
       uint32_t sv[64];
       tmem_ld_x64(tA, sv);
       // P^T for this thread's 64 query columns (causal diagonal tile: a query
@@ -261,7 +263,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const float e = fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lse2[c]));
+        const float lc = __shfl_sync(0xffffffffu, (c & 1) ? my_l.y : my_l.x, c >> 1);
+        const float e = fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lc));
         pv[c] = (c < lim) ? 0.f : e;
       }
 #pragma unroll
@@ -280,8 +283,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int c0 = 32 * q2 + 2 * c;
-          pk[16 * q2 + c] = pack_bf16x2(pv[c0] * (__uint_as_float(dv[2 * c]) - dd[c0]),
-                                        pv[c0 + 1] * (__uint_as_float(dv[2 * c + 1]) - dd[c0 + 1]));
+          const float d0 = __shfl_sync(0xffffffffu, my_d.x, c0 >> 1);
+          const float d1 = __shfl_sync(0xffffffffu, my_d.y, c0 >> 1);
+          pk[16 * q2 + c] = pack_bf16x2(pv[c0] * (__uint_as_float(dv[2 * c]) - d0),
+                                        pv[c0 + 1] * (__uint_as_float(dv[2 * c + 1]) - d1));
         }
       }
       tmem_st_x32(tB, pk);
