@@ -37,10 +37,12 @@ METRIC = "attention fwd TFLOP/s (bf16, d=128, 1 B200) and % of dense-BF16 tensor
 METRIC_E4M3 = "attention fwd TFLOP/s (e4m3 inputs, d=128, 1 B200) and % of dense-FP8 tensor peak"
 
 
-def metric_for(w: ai.Workload) -> str:
-    return METRIC_E4M3 if w.e4m3 else METRIC
 FLUSH_BYTES = 256 << 20
 MUFU_EX2_PER_CLK_PER_SM = 16  # 4 SFU lanes per SM sub-partition, 4 sub-partitions
+
+
+def metric_for(w: ai.Workload) -> str:
+    return METRIC_E4M3 if w.e4m3 else METRIC
 
 
 def visible_pairs(L: int, causal: bool, window=None) -> float:
@@ -70,15 +72,24 @@ def workload_exps(w: ai.Workload) -> float:
     return workload_flops(w) / (4.0 * w.d)
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source with comments and blank lines removed (string literals in these
+    files hold PTX, which has no comment markers)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash() -> str:
-    """sha256 of the forward kernel's sources (the ncu traffic figure applies only
-    to the kernel these hash to)."""
+    """sha256 of the forward kernel's sources without comments (the ncu traffic
+    figure applies only to the kernel these hash to)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_103_b200", "csrc")
     for name in ("attn_fwd_sm100.cu", "attn_fwd_sm100.h", "sm100_ptx.cuh", "exp2_poly.h"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 

@@ -23,8 +23,10 @@
 //   P~  = 2^(scale*S*log2e - m_ref)    MUFU ex2, or for POLY of every 8 column pairs
 //       the FMA-pipe polynomial ("FlashAttention V4 deep-dive", section 3.2);
 //       l += sum P~ (fp32, before rounding)
-//   P~ -> bf16, written back over S_s in TMEM
-//   O_s += P~ V_j                      tcgen05.mma, A = P~ from TMEM, B = V from smem
+//   P~ -> bf16 (E4M3 on the 8-bit path), written back over S_s in TMEM in two
+//       halves of 64 keys, each released to the MMA warp as soon as it is stored
+//   O_s += P~ V_j                      tcgen05.mma, A = P~ from TMEM, B = V from smem,
+//                                      issued per half of P~
 // after the last key tile: O = O_s / l -> bf16 -> global; LSE = ln2*(m_ref + log2 l).
 // The mask hook (MaskFn below) decides which key tiles an item visits and which
 // keys of a tile are hidden: causal items skip key tiles above the diagonal

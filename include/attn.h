@@ -16,7 +16,8 @@
  *  - Every tensor pointer is a DEVICE pointer owned by the caller; the library
  *    never frees or retains it.  Calls are asynchronous on `stream`; argument
  *    errors are returned before anything is launched.
- *  - Q, K, V, O are bf16, contiguous, head dimension innermost:
+ *  - Q, K, V, O are bf16 (attn_fwd_e4m3: Q, K, V are E4M3), contiguous, head
+ *    dimension innermost:
  *      dense:  [B, N, H, d]   (row stride H*d elements)
  *      varlen: [T, H, d]      packed, T = cu_seqlens[B]
  *    Their base addresses must be 16-byte aligned.
