@@ -41,6 +41,9 @@ BWD_DENSE = [
     (2, 300, 3, 128, True),
     (1, 513, 2, 64, True),
     (1, 1, 1, 128, False),
+    (1, 1100, 2, 128, True),     # nine tiles: the pipelined order wraps the ring several times
+    (1, 1100, 2, 128, False),
+    (1, 700, 2, 64, False),
 ]
 
 
@@ -105,3 +108,34 @@ def test_bwd_full_workload_sampled():
         rq, rk, rv = oracle.bwd_sampled(q.reshape(shp), k.reshape(shp), v.reshape(shp),
                                         do.reshape(shp), cu, True, 1 / math.sqrt(w.d), b, h, rows, rows)
         _check([dq[b, rows, h], dk[b, rows, h], dv[b, rows, h]], [rq, rk, rv], f"full b{b} h{h}")
+
+
+def test_bwd_peaked_rows():
+    """Q x 4: sharply peaked probability rows (P close to one-hot)."""
+    ea = _ea()
+    B, N, H, d = 1, 640, 2, 128
+    q, k, v, do = ai.make_custom(B, N, H, d, seed=12, n=4)
+    q = (q.float() * 4).to(torch.bfloat16)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = ea.fwd(qd, kd, vd, causal=True)
+    dq, dk, dv = ea.bwd(qd, kd, vd, o, lse, dod, causal=True)
+    ea.get_device_status()
+    shp = (B * N, H, d)
+    refs = oracle.bwd(q.reshape(shp), k.reshape(shp), v.reshape(shp), do.reshape(shp),
+                      oracle.dense_cu(B, N), True, 1 / math.sqrt(d))
+    _check([g.cpu().reshape(shp) for g in (dq, dk, dv)], refs, "q x4")
+
+
+def test_bwd_parity_varlen_d64():
+    ea = _ea()
+    lengths = [130, 7, 600, 256]
+    H, d = 2, 64
+    q, k, v, do = ai.make_custom(0, 0, H, d, seed=13, lengths=lengths, n=4)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    cu_d = torch.from_numpy(cu).to(DEV)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = ea.fwd(qd, kd, vd, causal=True, cu_seqlens=cu_d, max_seqlen=max(lengths))
+    grads = ea.bwd(qd, kd, vd, o, lse, dod, causal=True, cu_seqlens=cu_d, max_seqlen=max(lengths))
+    ea.get_device_status()
+    refs = oracle.bwd(q, k, v, do, cu, True, 1 / math.sqrt(d))
+    _check([g.cpu() for g in grads], refs, "varlen d64")
