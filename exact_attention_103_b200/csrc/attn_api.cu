@@ -108,6 +108,9 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 constexpr float kDefaultTau = 8.0f;
+// E4M3 path: a lower threshold leaves room to scale P~ up by 2^floor(8 - tau), so
+// small probabilities stay normal E4M3 numbers instead of flushing to subnormals.
+constexpr float kDefaultTauE4m3 = 2.0f;
 constexpr int kMaxVarlenB = 1024;
 constexpr int kMaxVarlenN = 131072;
 
@@ -140,7 +143,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   if (items_bound > INT32_MAX / 2 || dense_tokens * H > INT64_MAX / 256 || dense_tokens > INT32_MAX)
     return fail(ATTN_ERR_UNSUPPORTED, "problem too large for 32-bit tile indexing");
   if (varlen && !aligned(cu_seqlens, 4)) return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens misaligned");
-  float tau = kDefaultTau;
+  float tau = f8 ? kDefaultTauE4m3 : kDefaultTau;
   uint64_t timeout = kDefaultTimeoutNs;
   unsigned long long* stats = nullptr;
   int test_fault = 0, poly = 0, has_window = 0, wl = -1, wr = -1;
@@ -220,6 +223,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
   a.p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634 *
                                       (f8 ? static_cast<double>(f8->q) * f8->k : 1.0));
   a.p.o_scale = f8 ? f8->v : 1.f;
+  a.p.p_shift = f8 ? std::floor(8.f - tau) : 0.f;
   a.p.tau = tau;
   a.p.err = dev->err;
   a.p.stats = stats;

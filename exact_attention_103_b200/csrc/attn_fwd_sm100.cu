@@ -478,7 +478,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // FMA-pipe polynomial for the exponential, partial row sums, packing.  In
         // kPSplit parts: each is stored and released to the MMA warp (the PV K steps
         // over its keys) while the next is computed.
-        const float nm = (MASK == kMaskWindow && m_ref == -INFINITY) ? 0.f : -m_ref;
+        float nm = (MASK == kMaskWindow && m_ref == -INFINITY) ? 0.f : -m_ref;
+        if constexpr (F8) nm += p.p_shift;  // P~ * 2^p_shift <= 256 stays in E4M3's range
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int half = 0; half < kPSplit; ++half) {
@@ -574,7 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (store) {
-        const float lse = (m_ref + __log2f(l)) * kLn2;
+        float lse2 = m_ref + __log2f(l);
+        if constexpr (F8) lse2 -= p.p_shift;
+        const float lse = lse2 * kLn2;
         int64_t li;
         if (p.cu_seqlens == nullptr)
           li = (static_cast<int64_t>(b) * p.H + h) * p.N + q_row;

@@ -31,6 +31,8 @@ struct FwdParams {
   int test_fault;        // 1: withhold the first Q copy (failure-path tests only)
   int wl, wr;            // kMaskWindow bounds, both >= 0 (an open side holds a large value)
   float o_scale;         // E4M3 path: V's per-tensor scale, applied with 1/l
+  float p_shift;         // E4M3 path: P~ carries a factor 2^p_shift (an integer) so
+                         // it spans E4M3's normal range; l carries it too
 };
 
 struct FwdLaunch {

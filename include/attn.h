@@ -139,11 +139,14 @@ ATTN_API attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, 
  * are q * q_scale, k * k_scale, v * v_scale (per-tensor scales, finite and > 0).
  * O is bf16 and LSE fp32 exactly as in attn_fwd (LSE of the scaled scores of the
  * real inputs).  S = Q K^T and O += P~ V run on tcgen05.mma kind::f8f6f4; P~
- * (<= 2^tau) is rounded to E4M3 (nearest even, saturating) for the PV product,
- * while the row sum l adds the unrounded fp32 P~.  d must be 128
+ * (<= 2^tau) is computed with an extra factor 2^floor(8 - tau), so that it fills
+ * E4M3's range (at most 256 of the 448 maximum) and small probabilities stay
+ * normal numbers, and is rounded to E4M3 (nearest even, saturating) for the PV
+ * product, while the row sum l adds the unrounded fp32 values (the factor cancels
+ * in O = sum P~ v / l and is taken out of LSE).  d must be 128
  * (ATTN_ERR_UNSUPPORTED otherwise); opts as for attn_fwd_ex, except that
- * exp_poly_per8 must be 0 and rescale_threshold at most 8, so that P~ <= 256 stays
- * inside the E4M3 range.  Errors as for attn_fwd_ex.
+ * exp_poly_per8 must be 0, rescale_threshold is at most 8, and its default on
+ * this path is 2.  Errors as for attn_fwd_ex.
  */
 ATTN_API attn_status_t attn_fwd_e4m3(const void* q, const void* k, const void* v, void* o,
                                      float* lse, int B, int H, int N, int d, int causal,

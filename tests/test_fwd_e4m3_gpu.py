@@ -85,6 +85,23 @@ def test_e4m3_parity_dense(B, N, H, causal, window):
     compare_lse(lse.cpu(), oracle.lse_to_dense(l_ref, B, N))
 
 
+def test_e4m3_peaked_rows():
+    """Q x 4: sharply peaked rows, where most P~ are far below the row maximum."""
+    ea = _ea()
+    B, N, H, d = 1, 768, 2, 128
+    q, k, v = ai.make_custom(B, N, H, d, seed=17)
+    q = (q.float() * 4).to(torch.bfloat16)
+    (q8, k8, v8), sc = _quant((q, k, v))
+    scale = 1.0 / math.sqrt(d)
+    for causal in (False, True):
+        o, lse = ea.fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), causal=causal, scale=scale,
+                        e4m3_scales=sc)
+        ea.get_device_status()
+        o_ref, l_ref, a_ref = _oracle(q8, k8, v8, sc, oracle.dense_cu(B, N), causal, scale)
+        compare_o_e4m3(o.cpu().reshape(-1, H, d), o_ref, a_ref, f"e4m3 q x4 causal={causal}")
+        compare_lse(lse.cpu(), oracle.lse_to_dense(l_ref, B, N))
+
+
 def test_e4m3_parity_varlen():
     ea = _ea()
     lengths = [5, 0, 300, 129, 700]
