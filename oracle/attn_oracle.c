@@ -9,7 +9,7 @@
  *   "FlashAttention 1-4 详解", section 原算法 (standard attention):
  *       Attention(Q,K,V) = softmax(Q K^T / sqrt(d_k)) V
  *   with the scale passed in by the caller (the pages use 1/sqrt(d)), a causal
- *   option ("lower triangle": key j visible to query i iff j <= i, section
+ *   option (the lower-triangle mask: key j visible to query i iff j <= i, section
  *   其他优化 / FlashAttention 2 的工程优化, causal mask), and packed variable-length
  *   batches (sequence b owns tokens [cu[b], cu[b+1]); indices are local to it).
  *
