@@ -110,7 +110,7 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 constexpr float kDefaultTau = 8.0f;
 // E4M3 path: a lower threshold leaves room to scale P~ up by 2^floor(8 - tau), so
 // small probabilities stay normal E4M3 numbers instead of flushing to subnormals.
-constexpr float kDefaultTauE4m3 = 2.0f;
+constexpr float kDefaultTauE4m3 = 4.0f;
 constexpr int kMaxVarlenB = 1024;
 constexpr int kMaxVarlenN = 131072;
 
