@@ -68,6 +68,9 @@ def _load():
         lib.oracle_online_fwd.restype = ctypes.c_int64
         lib.oracle_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, ci, i64p, ci, ci, ci, cd, ci]
         lib.oracle_bwd.restype = ci
+        lib.oracle_bwd_masked.argtypes = [dp, dp, dp, dp, dp, dp, dp, ci, i64p, ci, ci, ci, ci, ci,
+                                          cd, ci]
+        lib.oracle_bwd_masked.restype = ci
         lib.oracle_bwd_sampled.argtypes = [dp, dp, dp, dp, ci, i64p, ci, ci, ci, cd, ci, ci,
                                            ip, ci, ip, ci, dp, dp, dp, ci]
         lib.oracle_bwd_sampled.restype = ci
@@ -175,15 +178,17 @@ def online_fwd(q, k, v, cu, causal: bool, scale: float, Br: int, Bc: int, tau: f
     return o, lse, int(n)
 
 
-def bwd(q, k, v, dout, cu, causal: bool, scale: float, nthreads: int = 0):
-    """Textbook backward: returns (dq, dk, dv), each [T,H,d] fp64."""
+def bwd(q, k, v, dout, cu, causal: bool, scale: float, nthreads: int = 0, window=None):
+    """Textbook backward: returns (dq, dk, dv), each [T,H,d] fp64 (``window`` as
+    for ``fwd``)."""
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     T, H, d = q.shape
     cu = _cu(cu, T)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
-    rc = _load().oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                            cu.size - 1, _ptr(cu, ctypes.c_int64), H, d, int(causal),
-                            float(scale), int(nthreads))
+    wl, wr = _window(window)
+    rc = _load().oracle_bwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), cu.size - 1, _ptr(cu, ctypes.c_int64), H, d,
+                                   int(causal), wl, wr, float(scale), int(nthreads))
     if rc < 0:
         raise ValueError("oracle_bwd rejected its arguments")
     return dq, dk, dv

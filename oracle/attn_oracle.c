@@ -25,7 +25,8 @@
  *   oracle_online_fwd  the tiled online-softmax algorithm in the pages' steps
  *                      (FlashAttention 1 recurrences, FlashAttention 2 deferred
  *                      normalisation, FlashAttention 4 conditional rescale)
- *   oracle_bwd         the textbook backward pass (recomputes P)
+ *   oracle_bwd         the textbook backward pass (recomputes P); *_masked adds
+ *                      the sliding window
  *   oracle_bwd_sampled the same gradients for selected query rows (dQ) and key
  *                      rows (dK, dV) of one (sequence, head), for full-size checks
  *
@@ -318,9 +319,9 @@ int64_t oracle_online_fwd(const double* q, const double* k, const double* v, dou
  *   dK_j  = scale sum_i dS_ij q_i
  * O is recomputed here from the definition (not taken from the caller).  One
  * thread owns a whole (sequence, head), so the accumulations do not race. */
-int oracle_bwd(const double* q, const double* k, const double* v, const double* dout,
-               double* dq, double* dk, double* dv, int nseq, const int64_t* cu, int H, int d,
-               int causal, double scale, int nthreads) {
+int oracle_bwd_masked(const double* q, const double* k, const double* v, const double* dout,
+                      double* dq, double* dk, double* dv, int nseq, const int64_t* cu, int H,
+                      int d, int causal, int wl, int wr, double scale, int nthreads) {
   if (nseq < 0 || H <= 0 || d <= 0 || !cu) return -1;
   const int used = set_threads(nthreads);
   const int64_t T = cu[nseq];
@@ -343,10 +344,11 @@ int oracle_bwd(const double* q, const double* k, const double* v, const double* 
         const int64_t ti = base + i;
         const double* q_row = q + (ti * H + h) * (int64_t)d;
         const double* do_row = dout + (ti * H + h) * (int64_t)d;
-        const int nvis = visible_keys(i, L, causal);
-        /* P row by the definition. */
+        int lo, hi;
+        visible_range(i, L, causal, wl, wr, &lo, &hi);
+        /* P row by the definition (entries [lo, hi) of prow). */
         double mx = -INFINITY;
-        for (int j = 0; j < nvis; ++j) {
+        for (int j = lo; j < hi; ++j) {
           const double* k_row = k + ((base + j) * H + h) * (int64_t)d;
           double acc = 0.0;
           for (int c = 0; c < d; ++c) acc += q_row[c] * k_row[c];
@@ -354,18 +356,18 @@ int oracle_bwd(const double* q, const double* k, const double* v, const double* 
           if (prow[j] > mx) mx = prow[j];
         }
         double l = 0.0;
-        for (int j = 0; j < nvis; ++j) { prow[j] = exp(prow[j] - mx); l += prow[j]; }
-        for (int j = 0; j < nvis; ++j) prow[j] /= l;
+        for (int j = lo; j < hi; ++j) { prow[j] = exp(prow[j] - mx); l += prow[j]; }
+        for (int j = lo; j < hi; ++j) prow[j] /= l;
         /* O row and D_i. */
         for (int c = 0; c < d; ++c) orow[c] = 0.0;
-        for (int j = 0; j < nvis; ++j) {
+        for (int j = lo; j < hi; ++j) {
           const double* v_row = v + ((base + j) * H + h) * (int64_t)d;
           for (int c = 0; c < d; ++c) orow[c] += prow[j] * v_row[c];
         }
         double Di = 0.0;
         for (int c = 0; c < d; ++c) Di += do_row[c] * orow[c];
         double* dq_row = dq + (ti * H + h) * (int64_t)d;
-        for (int j = 0; j < nvis; ++j) {
+        for (int j = lo; j < hi; ++j) {
           const int64_t tj = base + j;
           const double* k_row = k + (tj * H + h) * (int64_t)d;
           const double* v_row = v + (tj * H + h) * (int64_t)d;
@@ -386,6 +388,13 @@ int oracle_bwd(const double* q, const double* k, const double* v, const double* 
     free(orow);
   }
   return used;
+}
+
+int oracle_bwd(const double* q, const double* k, const double* v, const double* dout,
+               double* dq, double* dk, double* dv, int nseq, const int64_t* cu, int H, int d,
+               int causal, double scale, int nthreads) {
+  return oracle_bwd_masked(q, k, v, dout, dq, dk, dv, nseq, cu, H, d, causal, -1, -1, scale,
+                           nthreads);
 }
 
 /* The textbook backward of oracle_bwd, for one (sequence b, head h), evaluated only

@@ -409,3 +409,47 @@ def test_window_rows_equal_full_and_wide_window_is_unmasked():
     o_w, _, _ = oracle.fwd(qp, kp, vp, cu, True, 0.25, window=(1000, 1000))
     o_c, _, _ = oracle.fwd(qp, kp, vp, cu, True, 0.25)
     np.testing.assert_array_equal(o_w, o_c)
+
+
+# ------------------------------------------------- windowed backward
+@pytest.mark.parametrize("wl,wr,causal", [(3, 0, True), (5, 2, False), (0, 0, False), (-1, 3, False)])
+def test_bwd_window_matches_torch_autograd_fp64(wl, wr, causal):
+    """Library special case: PyTorch fp64 autograd through SDPA with the visibility
+    matrix as a boolean mask."""
+    B, N, H, d = 2, 21, 2, 8
+    q, k, v, do = make_custom(B, N, H, d, seed=31, n=4)
+    mask = _window_bool_mask(N, wl, wr, causal)
+    qt, kt, vt = (x.double().permute(0, 2, 1, 3).requires_grad_(True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.4)
+    (o * do.double().permute(0, 2, 1, 3)).sum().backward()
+    refs = [t.grad.permute(0, 2, 1, 3).numpy().reshape(B * N, H, d) for t in (qt, kt, vt)]
+    got = oracle.bwd(_packed(q), _packed(k), _packed(v), _packed(do), oracle.dense_cu(B, N),
+                     causal, 0.4, window=(wl, wr))
+    for g, r in zip(got, refs):
+        np.testing.assert_allclose(g, r, rtol=0, atol=1e-11)
+
+
+def test_bwd_window_central_finite_differences():
+    """d/dx of L = sum(dO * O) by central differences for a few entries of q, k, v,
+    with a causal one-key-back window on a packed pair of sequences."""
+    lengths = [7, 5]
+    H, d = 1, 4
+    q, k, v, do = (_packed(t) for t in make_custom(0, 0, H, d, seed=32, lengths=lengths, n=4))
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    win = (1, 0)
+    dq, dk, dv = oracle.bwd(q, k, v, do, cu, True, 0.7, window=win)
+
+    def loss(q_, k_, v_):
+        o, _, _ = oracle.fwd(q_, k_, v_, cu, True, 0.7, window=win)
+        return float((o * do).sum())
+
+    eps = 1e-6
+    for arr, grad in ((q, dq), (k, dk), (v, dv)):
+        for idx in [(0, 0, 0), (3, 0, 2), (6, 0, 1), (7, 0, 3), (11, 0, 0)]:
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += eps
+            minus[idx] -= eps
+            args_p = [plus if a is arr else a for a in (q, k, v)]
+            args_m = [minus if a is arr else a for a in (q, k, v)]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - grad[idx]) < 1e-6, (idx, fd, grad[idx])
