@@ -26,13 +26,20 @@ ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_WORKSPACE = 3, 4, 5
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_ex", "attn_bwd", "attn_bwd_workspace_size",
                     "attn_get_device_status", "attn_status_string", "attn_last_error",
                     "attn_selftest_umma", "attn_fwd_noalloc", "attn_fwd_e4m3",
-                    "attn_selftest_umma_e4m3")
+                    "attn_selftest_umma_e4m3", "attn_bwd_ex")
 
 
 class AttnError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{status_string(status) if _lib else status}: {message}")
         self.status = status
+
+
+class BwdOpts(ctypes.Structure):
+    _fields_ = [("has_window", ctypes.c_int),
+                ("window_left", ctypes.c_int),
+                ("window_right", ctypes.c_int),
+                ("timeout_ns", ctypes.c_uint64)]
 
 
 class FwdOpts(ctypes.Structure):
@@ -68,6 +75,9 @@ def load_library(path: str = LIB_PATH):
     lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, ci,
                              vp, cs, vp]
     lib.attn_bwd.restype = ci
+    lib.attn_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, ci,
+                                vp, cs, ctypes.POINTER(BwdOpts), vp]
+    lib.attn_bwd_ex.restype = ci
     lib.attn_bwd_workspace_size.argtypes = [ci, ci, ci, ci, ci, ci]
     lib.attn_bwd_workspace_size.restype = cs
     lib.attn_get_device_status.argtypes = [vp]
@@ -343,12 +353,13 @@ def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Te
 def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
         dout: torch.Tensor, causal: bool = False, scale: Optional[float] = None,
         cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: Optional[int] = None,
-        deterministic: bool = False, stream: Optional[torch.cuda.Stream] = None):
+        deterministic: bool = False, stream: Optional[torch.cuda.Stream] = None,
+        window: Optional[Tuple[int, int]] = None):
     """Exact attention backward on the GPU: returns (dq, dk, dv), bf16, layout of q.
 
-    ``o`` and ``lse`` are the forward's outputs.  The workspace (the per-row
-    <dO, O>) is allocated with torch.  Results are bitwise reproducible whether or
-    not ``deterministic`` is set."""
+    ``o`` and ``lse`` are the forward's outputs (``window`` as given to ``fwd``).
+    The workspace (the per-row <dO, O>) is allocated with torch.  Results are
+    bitwise reproducible whether or not ``deterministic`` is set."""
     lib = load_library()
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
         _need(t, n)
@@ -366,10 +377,13 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse:
     ws_bytes = lib.attn_bwd_workspace_size(B, H, N, d, total, int(bool(deterministic)))
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
     with torch.cuda.device(q.device):
-        st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                          dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
-                          int(bool(causal)), float(scale), cu_ptr, int(bool(deterministic)),
-                          ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+        opts = BwdOpts(0 if window is None else 1, -1 if window is None else int(window[0]),
+                       -1 if window is None else int(window[1]), 0)
+        st = lib.attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                             dv.data_ptr(), B, H, N, d, int(bool(causal)), float(scale), cu_ptr,
+                             int(bool(deterministic)), ws.data_ptr(), ws.numel(),
+                             ctypes.byref(opts), _stream_ptr(stream))
     _check(st)
     return dq, dk, dv
 

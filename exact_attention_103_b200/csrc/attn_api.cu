@@ -114,6 +114,24 @@ constexpr float kDefaultTauE4m3 = 4.0f;
 constexpr int kMaxVarlenB = 1024;
 constexpr int kMaxVarlenN = 131072;
 
+// The mask of a call: a window bound of N - 1 or more hides nothing on that side,
+// so a window collapses to the causal or the unmasked kernel where it can; open
+// sides hold N.  Causal forces the right bound to 0.
+attn_status_t select_mask(int N, int causal, int has_window, int wl, int wr, attn::MaskKind* mask,
+                          int* win_l, int* win_r) {
+  *mask = causal ? attn::kMaskCausal : attn::kMaskNone;
+  *win_l = *win_r = 0;
+  if (!has_window) return ATTN_OK;
+  if (N >= (1 << 30)) return fail(ATTN_ERR_UNSUPPORTED, "sliding window needs N < 2^30");
+  *win_l = (wl < 0 || wl > N) ? N : wl;
+  *win_r = causal ? 0 : ((wr < 0 || wr > N) ? N : wr);
+  const bool left_open = *win_l >= N - 1, right_open = *win_r >= N - 1;
+  if (left_open && right_open) *mask = attn::kMaskNone;
+  else if (left_open && *win_r == 0) *mask = attn::kMaskCausal;
+  else *mask = attn::kMaskWindow;
+  return ATTN_OK;
+}
+
 // Per-tensor scales of the E4M3 entry point (real value = stored value * scale).
 struct E4m3Scales {
   float q, k, v;
@@ -168,23 +186,14 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
       wr = opts->window_right;
     }
   }
-  // The mask: a window bound of N - 1 or more hides nothing on that side, so the
-  // window collapses to the causal or the unmasked kernel where it can.
-  attn::MaskKind mask = causal ? attn::kMaskCausal : attn::kMaskNone;
-  int win_l = 0, win_r = 0;
-  if (has_window) {
-    if (N >= (1 << 30)) return fail(ATTN_ERR_UNSUPPORTED, "sliding window needs N < 2^30");
-    win_l = (wl < 0 || wl > N) ? N : wl;
-    win_r = causal ? 0 : ((wr < 0 || wr > N) ? N : wr);
-    const bool left_open = win_l >= N - 1, right_open = win_r >= N - 1;
-    if (left_open && right_open) mask = attn::kMaskNone;
-    else if (left_open && win_r == 0) mask = attn::kMaskCausal;
-    else mask = attn::kMaskWindow;
-    if (mask == attn::kMaskWindow) stats = nullptr;  // counters are not kept under a window
-  }
+  attn::MaskKind mask;
+  int win_l, win_r;
+  attn_status_t st = select_mask(N, causal, has_window, wl, wr, &mask, &win_l, &win_r);
+  if (st != ATTN_OK) return st;
+  if (mask == attn::kMaskWindow) stats = nullptr;  // counters are not kept under a window
 
   DeviceState* dev = nullptr;
-  attn_status_t st = device_state(&dev);
+  st = device_state(&dev);
   if (st != ATTN_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
@@ -299,11 +308,14 @@ attn_status_t attn_fwd_e4m3(const void* q, const void* k, const void* v, void* o
   return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, hint, opts, stream, &f8);
 }
 
-attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+}  // extern "C"
+
+namespace {
+attn_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o,
                        const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
                        int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
                        int deterministic, void* workspace, size_t workspace_bytes,
-                       attn_stream_t stream) {
+                       const attn_bwd_opts_t* opts, attn_stream_t stream) {
   (void)deterministic;  // every call is deterministic: no atomic accumulation
   if (B < 0 || H <= 0 || N < 0) return fail(ATTN_ERR_INVALID_ARG, "B=%d H=%d N=%d", B, H, N);
   if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
@@ -322,8 +334,13 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   const int64_t dense_tokens = static_cast<int64_t>(B) * N;
   if (grid > INT32_MAX / 2 || dense_tokens > INT32_MAX)
     return fail(ATTN_ERR_UNSUPPORTED, "problem too large for 32-bit tile indexing");
+  attn::MaskKind mask;
+  int win_l, win_r;
+  attn_status_t st = select_mask(N, causal, opts ? opts->has_window : 0, opts ? opts->window_left : -1,
+                                 opts ? opts->window_right : -1, &mask, &win_l, &win_r);
+  if (st != ATTN_OK) return st;
   DeviceState* dev = nullptr;
-  attn_status_t st = device_state(&dev);
+  st = device_state(&dev);
   if (st != ATTN_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   int64_t total = dense_tokens;
@@ -359,11 +376,34 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   a.p.scale = scale;
   a.p.scale_log2 = scale * 1.4426950408889634f;
   a.p.err = dev->err;
-  a.p.timeout_ns = kDefaultTimeoutNs;
+  a.p.timeout_ns = (opts && opts->timeout_ns) ? opts->timeout_ns : kDefaultTimeoutNs;
+  a.p.wl = win_l;
+  a.p.wr = win_r;
   a.grid = static_cast<int>(grid);
-  const cudaError_t e = attn::launch_bwd(a, o, dout, d, causal ? 1 : 0, cs);
+  const cudaError_t e = attn::launch_bwd(a, o, dout, d, static_cast<int>(mask), cs);
   if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
   return ATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                       int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
+                       int deterministic, void* workspace, size_t workspace_bytes,
+                       attn_stream_t stream) {
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, causal, scale, cu_seqlens,
+                  deterministic, workspace, workspace_bytes, nullptr, stream);
+}
+
+attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                          int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
+                          int deterministic, void* workspace, size_t workspace_bytes,
+                          const attn_bwd_opts_t* opts, attn_stream_t stream) {
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, causal, scale, cu_seqlens,
+                  deterministic, workspace, workspace_bytes, opts, stream);
 }
 
 size_t attn_bwd_workspace_size(int B, int H, int N, int d, int total_tokens, int deterministic) {

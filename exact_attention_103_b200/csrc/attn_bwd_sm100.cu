@@ -206,13 +206,15 @@ __global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
 // Per query tile i:  S^T = K_j Q_i^T (TMEM A), dP^T = V_j dO_i^T (TMEM B);
 //   P^T = exp2(scale*log2e*S^T - LSE2_i) (causal: zero where query < key) -> A;
 //   dV += P^T dO_i;  dS^T = P^T o (dP^T - D_i) -> B;  dK += dS^T Q_i.
-template <int D, bool CAUSAL>
+// MASK: 0 none, 1 causal, 2 sliding window (see BwdParams::wl, wr).
+template <int D, int MASK>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p) {
   using Lay = BwdLayout<D>;
   BwdItem it;
+  constexpr bool CAUSAL = MASK == 1;
   if (!decode_block(p, true, CAUSAL, it)) return;  // uniform for the CTA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -229,8 +231,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int j = it.tile;
   const int ntiles = ceil_div(it.L, kTile);
-  const int i_first = CAUSAL ? j : 0;
-  const int nq = ntiles - i_first;
+  // Query tiles that see some key of this tile: causal from the diagonal on; a
+  // window from key - wr to key + wl.
+  int i_first = CAUSAL ? j : 0, i_end = ntiles;
+  if (MASK == 2) {
+    i_first = max(j * kTile - p.wr, 0) / kTile;
+    i_end = min(ntiles, (j * kTile + kTile - 1 + p.wl) / kTile + 1);
+  }
+  const int nq = i_end - i_first;
   float* vec = reinterpret_cast<float*>(smem + Lay::VEC_OFF);
 
   if (warp < 8) {
@@ -258,14 +266,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_x64(tA, sv);
       // P^T for this thread's 64 query columns (causal diagonal tile: a query
       // sees the key only if query >= key; rows past the sequence have LSE2 = +inf).
-      const int lim = (CAUSAL && i == j) ? r - 64 * hf : -1;  // columns < lim are masked
+      // Window: query q = qb + c sees this key iff key - wr <= q <= key + wl.
+      int lim = (CAUSAL && i == j) ? r - 64 * hf : -1;  // columns < lim are masked
+      int lim_hi = 64;                                   // columns > lim_hi are masked
+      if (MASK == 2) {
+        const int qb = i * kTile + 64 * hf;
+        lim = key - p.wr - qb;
+        lim_hi = key + p.wl - qb;
+      }
       float pv[64];
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         const float lc = __shfl_sync(0xffffffffu, (c & 1) ? my_l.y : my_l.x, c >> 1);
         const float e = fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lc));
-        pv[c] = (c < lim) ? 0.f : e;
+        pv[c] = (c < lim || (MASK == 2 && c > lim_hi)) ? 0.f : e;
       }
 #pragma unroll
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
@@ -471,13 +486,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Per key tile j:  S = Q_i K_j^T (TMEM A), dP = dO_i V_j^T (TMEM B);
 //   P = exp2(scale*log2e*S - LSE2_row) (causal: zero where key > query);
 //   dS = P o (dP - D_row) -> B;  dQ += dS K_j.  dQ is scaled at the end.
-template <int D, bool CAUSAL>
+template <int D, int MASK>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p) {
   using Lay = BwdLayout<D>;
   BwdItem it;
+  constexpr bool CAUSAL = MASK == 1;
   if (!decode_block(p, false, CAUSAL, it)) return;  // uniform for the CTA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -494,7 +510,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int i = it.tile;
   const int ntiles = ceil_div(it.L, kTile);
-  const int nk = CAUSAL ? (i + 1 < ntiles ? i + 1 : ntiles) : ntiles;
+  // Key tiles [j_first, j_first + nk) holding a key some row of this tile sees.
+  int j_first = 0, j_end = CAUSAL ? (i + 1 < ntiles ? i + 1 : ntiles) : ntiles;
+  if (MASK == 2) {
+    j_first = max(i * kTile - p.wl, 0) / kTile;
+    j_end = min(ntiles, ceil_div(i * kTile + kTile + p.wr, kTile));
+  }
+  const int nk = j_end - j_first;
 
   if (warp < 8) {
     const int hf = warp >> 2, wq = warp & 3;
@@ -521,15 +543,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t sv[64];
       tmem_ld_x64(sb2 ? tA1 : tA0, sv);
-      // keys visible to this row: key < L and (causal) key <= q_row
-      const int kb = j * kTile + 64 * hf;
-      int lim = it.L - kb;
+      // keys visible to this row: key < L, (causal) key <= q_row, (window)
+      // q_row - wl <= key <= q_row + wr
+      const int kb = (j_first + j) * kTile + 64 * hf;
+      int lim = it.L - kb, lim_lo = 0;
       if (CAUSAL && q_row - kb + 1 < lim) lim = q_row - kb + 1;
+      if (MASK == 2) {
+        lim = min(lim, q_row + p.wr + 1 - kb);
+        lim_lo = q_row - p.wl - kb;
+      }
       float pv[64];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         const float e = fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lse2));
-        pv[c] = (c < lim) ? e : 0.f;
+        pv[c] = (c < lim && (MASK != 2 || c >= lim_lo)) ? e : 0.f;
       }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DP), dp_phase, wc, timeout_code(kSiteS)));
       if (!ok) break;
@@ -584,9 +611,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           tma_load_3d(base + c * Lay::CHUNK, &tm_k, bar(Lay::B_FULL + st), c * 64, it.h,
-                      it.seq_start + j * kTile, pol_ring);
+                      it.seq_start + (j_first + j) * kTile, pol_ring);
           tma_load_3d(base + Lay::TILE + c * Lay::CHUNK, &tm_v, bar(Lay::B_FULL + st), c * 64, it.h,
-                      it.seq_start + j * kTile, pol_ring);
+                      it.seq_start + (j_first + j) * kTile, pol_ring);
         }
       }
       __syncwarp();
@@ -691,11 +718,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 9) tmem_dealloc(tmem, 512);
 }
 
-template <int D, bool CAUSAL>
+template <int D, int MASK>
 cudaError_t launch_main(const BwdLaunch& a, cudaStream_t st) {
   const int smem = 1024 + BwdLayout<D>::SMEM;
-  auto k1 = bwd_dkdv_kernel<D, CAUSAL>;
-  auto k2 = bwd_dq_kernel<D, CAUSAL>;
+  auto k1 = bwd_dkdv_kernel<D, MASK>;
+  auto k2 = bwd_dq_kernel<D, MASK>;
   cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -708,7 +735,7 @@ cudaError_t launch_main(const BwdLaunch& a, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_bwd(const BwdLaunch& a, const void* o, const void* dout, int D, int causal,
+cudaError_t launch_bwd(const BwdLaunch& a, const void* o, const void* dout, int D, int mask,
                        cudaStream_t st) {
   const int64_t units = static_cast<int64_t>(a.p.total) * a.p.H;
   int blocks = static_cast<int>((units + 7) / 8);
@@ -718,8 +745,12 @@ cudaError_t launch_bwd(const BwdLaunch& a, const void* o, const void* dout, int 
                                           static_cast<const __nv_bfloat16*>(dout), a.p, D);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (D == 128) return causal ? launch_main<128, true>(a, st) : launch_main<128, false>(a, st);
-  return causal ? launch_main<64, true>(a, st) : launch_main<64, false>(a, st);
+  if (D == 128) {
+    if (mask == 2) return launch_main<128, 2>(a, st);
+    return mask == 1 ? launch_main<128, 1>(a, st) : launch_main<128, 0>(a, st);
+  }
+  if (mask == 2) return launch_main<64, 2>(a, st);
+  return mask == 1 ? launch_main<64, 1>(a, st) : launch_main<64, 0>(a, st);
 }
 
 }  // namespace attn

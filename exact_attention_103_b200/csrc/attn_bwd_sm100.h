@@ -22,6 +22,8 @@ struct BwdParams {
   float scale_log2;        // scale * log2(e)
   int* err;                // device error word
   uint64_t timeout_ns;
+  int wl, wr;              // sliding window (mask kind 2): key j visible to query i iff
+                           // i - wl <= j <= i + wr; both >= 0, an open side holds N
 };
 
 struct BwdLaunch {
@@ -30,7 +32,8 @@ struct BwdLaunch {
   int grid;  // B * ntiles * H CTAs for each main kernel
 };
 
-cudaError_t launch_bwd(const BwdLaunch& a, const void* o, const void* dout, int D, int causal,
+// mask: 0 none, 1 causal, 2 sliding window (the forward's MaskKind values).
+cudaError_t launch_bwd(const BwdLaunch& a, const void* o, const void* dout, int D, int mask,
                        cudaStream_t st);
 
 }  // namespace attn

@@ -169,6 +169,28 @@ ATTN_API attn_status_t attn_bwd(const void* q, const void* k, const void* v, con
                        const int32_t* cu_seqlens, int deterministic, void* workspace,
                        size_t workspace_bytes, attn_stream_t stream);
 
+/* Options for attn_bwd_ex.  Zero-initialise, then set fields.
+ *  has_window, window_left, window_right: the sliding-window mask of the forward
+ *      call whose gradients are wanted, with the meaning they have in
+ *      attn_fwd_opts_t (the mask hook; the causal flag still applies on top).
+ *  timeout_ns: limit of every internal wait; 0 selects the default (2 s). */
+typedef struct {
+  int has_window;
+  int window_left;
+  int window_right;
+  uint64_t timeout_ns;
+} attn_bwd_opts_t;
+
+/* attn_bwd with options (opts may be NULL = attn_bwd).  Under a window both
+ * kernels visit only the tiles the window reaches and mask its edges; the
+ * gradients are those of the windowed forward. */
+ATTN_API attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                                   const float* lse, const void* dout, void* dq, void* dk,
+                                   void* dv, int B, int H, int N, int d, int causal, float scale,
+                                   const int32_t* cu_seqlens, int deterministic, void* workspace,
+                                   size_t workspace_bytes, const attn_bwd_opts_t* opts,
+                                   attn_stream_t stream);
+
 /* Workspace bytes attn_bwd needs (total_tokens = B*N dense, cu_seqlens[B] varlen). */
 ATTN_API size_t attn_bwd_workspace_size(int B, int H, int N, int d, int total_tokens, int deterministic);
 

@@ -129,3 +129,10 @@ def test_e4m3_argument_checks(lib):
     assert call(opts=ea.FwdOpts(-1.0, None, 0, 0, 0, 0, 0, 0, 2)) == ea.ATTN_ERR_UNSUPPORTED
     assert call(opts=ea.FwdOpts(9.0, None, 0, 0, 0, 0, 0, 0, 0)) == ea.ATTN_ERR_INVALID_ARG
     assert call(B=0) == ea.ATTN_OK
+
+
+def test_backward_window_limit(lib):
+    opts = ea.BwdOpts(1, 64, 0, 0)
+    st = lib.attn_bwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1 << 30, 64,
+                         1, 0.1, None, 0, None, 0, ctypes.byref(opts), None)
+    assert st == ea.ATTN_ERR_UNSUPPORTED

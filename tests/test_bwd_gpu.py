@@ -139,3 +139,43 @@ def test_bwd_parity_varlen_d64():
     ea.get_device_status()
     refs = oracle.bwd(q, k, v, do, cu, True, 1 / math.sqrt(d))
     _check([g.cpu() for g in grads], refs, "varlen d64")
+
+
+@pytest.mark.parametrize("B,N,H,d,causal,window", [
+    (1, 700, 2, 128, True, (64, 0)),
+    (1, 640, 2, 128, False, (100, 30)),
+    (2, 300, 2, 64, False, (0, 0)),
+    (1, 900, 2, 128, False, (-1, 130)),
+    (1, 1100, 1, 128, True, (300, 0)),
+])
+def test_bwd_parity_window(B, N, H, d, causal, window):
+    """The backward of the sliding-window forward (the mask hook) against the
+    oracle's windowed textbook backward."""
+    ea = _ea()
+    q, k, v, do = ai.make_custom(B, N, H, d, seed=200 + N, n=4)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = ea.fwd(qd, kd, vd, causal=causal, window=window)
+    dq, dk, dv = ea.bwd(qd, kd, vd, o, lse, dod, causal=causal, window=window)
+    ea.get_device_status()
+    shp = (B * N, H, d)
+    refs = oracle.bwd(q.reshape(shp), k.reshape(shp), v.reshape(shp), do.reshape(shp),
+                      oracle.dense_cu(B, N), causal, 1 / math.sqrt(d), window=window)
+    _check([g.cpu().reshape(shp) for g in (dq, dk, dv)], refs, f"window {window} causal={causal}")
+
+
+def test_bwd_parity_window_varlen():
+    ea = _ea()
+    lengths = [200, 1, 128, 333, 700]
+    H, d = 2, 128
+    window = (90, 0)
+    q, k, v, do = ai.make_custom(0, 0, H, d, seed=201, lengths=lengths, n=4)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    cu_d = torch.from_numpy(cu).to(DEV)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = ea.fwd(qd, kd, vd, causal=True, cu_seqlens=cu_d, max_seqlen=max(lengths),
+                    window=window)
+    grads = ea.bwd(qd, kd, vd, o, lse, dod, causal=True, cu_seqlens=cu_d, max_seqlen=max(lengths),
+                   window=window)
+    ea.get_device_status()
+    refs = oracle.bwd(q, k, v, do, cu, True, 1 / math.sqrt(d), window=window)
+    _check([g.cpu() for g in grads], refs, "varlen window")
