@@ -16,7 +16,12 @@
 // Both main kernels: warps 0-7 elementwise work (warp w owns TMEM lanes
 // 32(w%4)..+31, one row per thread, and columns 64*(w/4)..+63 of each 128-column
 // tile), warp 8 TMA producer, warp 9 TMEM owner and MMA issuer (whole warp, one
-// elected lane issues).  Every wait is bounded as in the forward kernel.
+// elected lane issues).  The MMA warps issue their products in a software-
+// pipelined order so the next tile's exponentials overlap the current tile's
+// products (dK/dV: dV(n), S^T(n+1), dK(n), dP^T(n+1); dQ: dQ(j), dP(j+1), S(j+2)
+// with S double-buffered).  MASK selects the visibility rule of the forward's mask
+// hook: none, causal, or the sliding window (only the tiles the window reaches are
+// visited).  Every wait is bounded as in the forward kernel.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
