@@ -177,7 +177,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, flo
     poly = opts->exp_poly_per8;
     if (poly != 0 && poly != 2 && poly != 8)
       return fail(ATTN_ERR_INVALID_ARG, "exp_poly_per8 must be 0, 2 or 8");
-    if (f8 && poly != 0) return fail(ATTN_ERR_UNSUPPORTED, "E4M3 path: exp_poly_per8 must be 0");
+    if (f8 && poly != 0 && poly != 2)
+      return fail(ATTN_ERR_UNSUPPORTED, "E4M3 path: exp_poly_per8 must be 0 or 2");
     if (f8 && !(tau <= 8.f))
       return fail(ATTN_ERR_INVALID_ARG, "E4M3 path: rescale_threshold must be <= 8 (P~ <= 256 < 448)");
     if (opts->has_window) {

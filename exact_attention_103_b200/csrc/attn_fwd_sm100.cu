@@ -809,7 +809,12 @@ static cudaError_t launch_m(const FwdLaunch& a, MaskKind mask, int poly, cudaStr
 }
 
 cudaError_t launch_fwd(const FwdLaunch& a, int D, MaskKind mask, int poly, int fp8, cudaStream_t st) {
-  if (fp8) {  // E4M3: d = 128, all-MUFU exponentials
+  if (fp8) {  // E4M3: d = 128; exponentials all on MUFU or 2 of every 8 pairs on the FMA pipe
+    if (poly == 2) {
+      if (mask == kMaskCausal) return launch_t<128, kMaskCausal, 2, true>(a, st);
+      if (mask == kMaskWindow) return launch_t<128, kMaskWindow, 2, true>(a, st);
+      return launch_t<128, kMaskNone, 2, true>(a, st);
+    }
     if (mask == kMaskCausal) return launch_t<128, kMaskCausal, 0, true>(a, st);
     if (mask == kMaskWindow) return launch_t<128, kMaskWindow, 0, true>(a, st);
     return launch_t<128, kMaskNone, 0, true>(a, st);

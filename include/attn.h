@@ -145,8 +145,8 @@ ATTN_API attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, 
  * product, while the row sum l adds the unrounded fp32 values (the factor cancels
  * in O = sum P~ v / l and is taken out of LSE).  d must be 128
  * (ATTN_ERR_UNSUPPORTED otherwise); opts as for attn_fwd_ex, except that
- * exp_poly_per8 must be 0, rescale_threshold is at most 8, and its default on
- * this path is 4.  Errors as for attn_fwd_ex.
+ * exp_poly_per8 must be 0 or 2, rescale_threshold is at most 8, and its default
+ * on this path is 4.  Errors as for attn_fwd_ex.
  */
 ATTN_API attn_status_t attn_fwd_e4m3(const void* q, const void* k, const void* v, void* o,
                                      float* lse, int B, int H, int N, int d, int causal,

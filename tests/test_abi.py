@@ -126,7 +126,7 @@ def test_e4m3_argument_checks(lib):
     assert call(d=64) == ea.ATTN_ERR_UNSUPPORTED
     assert call(qs=0.0) == ea.ATTN_ERR_INVALID_ARG
     assert call(qs=float("nan")) == ea.ATTN_ERR_INVALID_ARG
-    assert call(opts=ea.FwdOpts(-1.0, None, 0, 0, 0, 0, 0, 0, 2)) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(opts=ea.FwdOpts(-1.0, None, 0, 0, 0, 0, 0, 0, 8)) == ea.ATTN_ERR_UNSUPPORTED
     assert call(opts=ea.FwdOpts(9.0, None, 0, 0, 0, 0, 0, 0, 0)) == ea.ATTN_ERR_INVALID_ARG
     assert call(B=0) == ea.ATTN_OK
 

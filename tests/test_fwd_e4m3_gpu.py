@@ -162,3 +162,18 @@ def test_e4m3_full_workload_sampled(name):
     a_ref, _ = oracle.fwd_rows(q, k, v.abs(), cu, w.causal, scale, rows, heads)
     compare_o_e4m3(o[rows, heads], o_ref, a_ref, name)
     compare_lse(lse[heads, rows], l_ref, name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_e4m3_poly_split(causal):
+    """2 of every 8 exponential pairs on the FMA-pipe polynomial, on the 8-bit path."""
+    ea = _ea()
+    B, N, H, d = 2, 600, 2, 128
+    (q8, k8, v8), sc = _quant(ai.make_custom(B, N, H, d, seed=19))
+    scale = 1.0 / math.sqrt(d)
+    o, lse = ea.fwd(q8.to(DEV), k8.to(DEV), v8.to(DEV), causal=causal, scale=scale,
+                    e4m3_scales=sc, exp_poly_per8=2)
+    ea.get_device_status()
+    o_ref, l_ref, a_ref = _oracle(q8, k8, v8, sc, oracle.dense_cu(B, N), causal, scale)
+    compare_o_e4m3(o.cpu().reshape(-1, H, d), o_ref, a_ref, f"e4m3 poly 2/8 causal={causal}")
+    compare_lse(lse.cpu(), oracle.lse_to_dense(l_ref, B, N))
