@@ -81,15 +81,25 @@ def _code_only(text: str) -> str:
     return "\n".join(ln for ln in lines if ln)
 
 
+def _device_part(text: str) -> str:
+    """The kernel file up to its host-side launch functions (which only pick the
+    template instantiation to launch)."""
+    cut = text.find("\nint fwd_smem_bytes(")
+    return text if cut < 0 else text[:cut]
+
+
 def kernel_source_hash() -> str:
-    """sha256 of the forward kernel's sources without comments (the ncu traffic
-    figure applies only to the kernel these hash to)."""
+    """sha256 of the forward kernel's device sources without comments (the ncu
+    traffic figure applies only to the kernel these hash to)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_103_b200", "csrc")
     for name in ("attn_fwd_sm100.cu", "attn_fwd_sm100.h", "sm100_ptx.cuh", "exp2_poly.h"):
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
-            h.update(_code_only(f.read()).encode())
+            text = f.read()
+        if name.endswith(".cu"):
+            text = _device_part(text)
+        h.update(_code_only(text).encode())
     return h.hexdigest()
 
 
