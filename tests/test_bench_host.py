@@ -49,3 +49,10 @@ def test_e4m3_inputs_are_exact_and_in_range():
     xr = x.float() / sc
     big = xr.abs() >= 2.0 ** -6
     assert torch.all((x8.float() - xr).abs()[big] <= xr.abs()[big] * 2.0 ** -4 + 1e-12)
+
+
+def test_source_hash_ignores_comments_and_launch_code():
+    src = "a = 1; // note\n/* block\n comment */\nint f();\n\nint fwd_smem_bytes(int D) { return 0; }\n"
+    assert bench._code_only(src) == "a = 1;\nint f();\nint fwd_smem_bytes(int D) { return 0; }"
+    assert bench._device_part(src) == "a = 1; // note\n/* block\n comment */\nint f();\n"
+    assert bench._code_only("x;  // a\n\n  y; /* b */\n") == "x;\n  y;"
