@@ -136,3 +136,18 @@ def test_backward_window_limit(lib):
     st = lib.attn_bwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1 << 30, 64,
                          1, 0.1, None, 0, None, 0, ctypes.byref(opts), None)
     assert st == ea.ATTN_ERR_UNSUPPORTED
+
+
+def test_missing_library_fails_loudly():
+    """No fallback: without the built library the binding raises (run in a fresh
+    interpreter so the already-loaded library is not reused)."""
+    import subprocess
+    import sys
+    code = ("import exact_attention_103_b200 as ea\n"
+            "try:\n"
+            "    ea.load_library('/nonexistent/libattn.so')\n"
+            "except RuntimeError as e:\n"
+            "    print('raised', 'not found' in str(e))\n")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT,
+                       timeout=300)
+    assert r.stdout.strip() == "raised True", r.stdout + r.stderr
