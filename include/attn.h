@@ -158,10 +158,14 @@ ATTN_API attn_status_t attn_fwd_e4m3(const void* q, const void* k, const void* v
  * Backward pass (dQ, dK, dV) from Q, K, V, O, LSE and dO, recomputing P from LSE
  * ("FlashAttention 1-4 详解", 总结 table: 反向传播重计算; "FlashAttention V4
  * deep-dive", section 3.3).  Same layouts as the forward; dq/dk/dv are bf16.
- * `deterministic` != 0 makes the result bitwise reproducible run to run.
- * `workspace` is a caller-owned DEVICE buffer of at least
- * attn_bwd_workspace_size(...) bytes, 256-byte aligned (may be NULL when that
- * size is 0).  Not yet provided by this build: returns ATTN_ERR_UNSUPPORTED.
+ * Three launches on `stream`: D_i = <dO_i, O_i> into the workspace, a kernel per
+ * 128-key tile accumulating dK and dV, and a kernel per 128-query tile
+ * accumulating dQ.  No result is accumulated with atomics, so every call is
+ * bitwise reproducible run to run; `deterministic` is accepted for interface
+ * compatibility and changes nothing.  `workspace` is a caller-owned DEVICE buffer
+ * of at least attn_bwd_workspace_size(...) bytes, 256-byte aligned (may be NULL
+ * when that size is 0); too small or misaligned: ATTN_ERR_WORKSPACE.  Same limits
+ * as the forward (d in {64, 128}); varlen reads cu_seqlens[B] back to the host.
  */
 ATTN_API attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
                        const float* lse, const void* dout, void* dq, void* dk, void* dv,
