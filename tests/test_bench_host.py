@@ -56,3 +56,25 @@ def test_source_hash_ignores_comments_and_launch_code():
     assert bench._code_only(src) == "a = 1;\nint f();\nint fwd_smem_bytes(int D) { return 0; }"
     assert bench._device_part(src) == "a = 1; // note\n/* block\n comment */\nint f();\n"
     assert bench._code_only("x;  // a\n\n  y; /* b */\n") == "x;\n  y;"
+
+
+def test_reference_arm_prints_one_contract_line():
+    """bench.py --impl reference times the oracle on the host and prints the
+    contract's JSON line (here on the tiny workload, so it runs in seconds)."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2",
+                        "--warmup", "3", "--workload", "B1-H1-N256-d64"],
+                       capture_output=True, text=True, cwd=root, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3
+    assert d["unit"] == "TFLOP/s" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"] == "B1-H1-N256-d64"
