@@ -81,8 +81,6 @@ attn_status_t device_state(DeviceState** out) {
   return ATTN_OK;
 }
 
-// 3-D bf16 view {d, H, total} of a token-major [total, H, d] tensor; box
-// {64, 1, 128} (one 128-byte swizzle chunk by 128 rows), 128-byte swizzle.
 // A 3-D view {d, H, total} of a token-major [total, H, d] tensor of esz-byte
 // elements (2: bf16, 1: E4M3 moved as bytes); box = one 128-byte-wide chunk of
 // 128 rows, 128-byte swizzle.
