@@ -1,0 +1,102 @@
+"""The pins are strong enough to catch plausible mistakes: each case plants one
+mistake in a private copy of the oracle's C source (never in the oracle itself),
+builds it, and checks that a pin from test_oracle_pins.py's families fails on it
+while the real oracle passes the same check."""
+import importlib.util
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attn_inputs import make_custom
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "attn_oracle.c")
+
+
+def _mutant(tmp_path, old, new):
+    text = open(SRC).read()
+    assert text.count(old) == 1, old
+    src = tmp_path / "attn_oracle_mutant.c"
+    src.write_text(text.replace(old, new))
+    spec = importlib.util.spec_from_file_location(f"oracle_mutant_{abs(hash(new))}",
+                                                  os.path.join(ROOT, "oracle", "__init__.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod._SRC = str(src)
+    mod._LIB_PATH = str(tmp_path / "liboracle_mutant.so")
+    mod._lib = None
+    return mod
+
+
+def _packed(t):
+    a = t.double().numpy()
+    return a.reshape(-1, a.shape[-2], a.shape[-1])
+
+
+def _sdpa_check(mod, causal):
+    B, N, H, d = 2, 17, 3, 16
+    q, k, v = make_custom(B, N, H, d, seed=11 + N)
+    o, _, _ = mod.fwd(_packed(q), _packed(k), _packed(v), mod.dense_cu(B, N), causal, 1 / math.sqrt(d))
+    qt, kt, vt = (x.double().permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=causal)
+    return np.allclose(o.reshape(B, N, H, d), ref.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-12)
+
+
+def _lse_check(mod):
+    B, N, H, d = 2, 23, 2, 16
+    q, k, v = make_custom(B, N, H, d, seed=12)
+    _, lse, _ = mod.fwd(_packed(q), _packed(k), _packed(v), mod.dense_cu(B, N), False, 0.3)
+    s = torch.einsum("bihc,bjhc->bhij", q.double(), k.double()) * 0.3
+    return np.allclose(mod.lse_to_dense(lse, B, N), torch.logsumexp(s, -1).numpy(), rtol=0, atol=1e-12)
+
+
+def _overflow_check(mod):
+    q, k, v = make_custom(1, 16, 1, 8, seed=8)
+    o, lse, _ = mod.fwd(_packed(q) * 200.0, _packed(k), _packed(v), [0, 16], False, 1.0)
+    return bool(np.all(np.isfinite(o)) and np.all(np.isfinite(lse)))
+
+
+def _window_check(mod):
+    L = 23
+    _, k, v = make_custom(1, L, 1, 4, seed=23)
+    vp = _packed(v)
+    o, _, _ = mod.fwd(np.zeros((L, 1, 4)), _packed(k), vp, [0, L], False, 1.0, window=(2, 3))
+    return all(np.allclose(o[i, 0], vp[max(0, i - 2):min(L, i + 4), 0].mean(axis=0), atol=1e-12)
+               for i in range(L))
+
+
+def _bwd_check(mod):
+    B, N, H, d = 2, 19, 2, 8
+    q, k, v, do = make_custom(B, N, H, d, seed=17, n=4)
+    got = mod.bwd(_packed(q), _packed(k), _packed(v), _packed(do), mod.dense_cu(B, N), True, 0.35)
+    qt, kt, vt = (x.double().permute(0, 2, 1, 3).requires_grad_(True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True, scale=0.35)
+    (o * do.double().permute(0, 2, 1, 3)).sum().backward()
+    refs = [t.grad.permute(0, 2, 1, 3).numpy().reshape(B * N, H, d) for t in (qt, kt, vt)]
+    return all(np.allclose(g, r, rtol=0, atol=1e-10) for g, r in zip(got, refs))
+
+
+MUTATIONS = [
+    ("dropped scale", "    srow[j - lo] = scale * acc;", "    srow[j - lo] = acc;",
+     lambda m: _sdpa_check(m, False)),
+    ("causal off by one", "  if (causal && i + 1 < b) b = i + 1;", "  if (causal && i < b) b = i > 0 ? i : 1;",
+     lambda m: _sdpa_check(m, True)),
+    ("no max subtraction", "srow[j] = exp(srow[j] - m); l += srow[j];", "srow[j] = exp(srow[j]); l += srow[j];",
+     _overflow_check),
+    ("LSE without the max", "  *lse_out = m + log(l);", "  *lse_out = log(l);", _lse_check),
+    ("window edge off by one", "  if (wl >= 0 && i - wl > a) a = i - wl;",
+     "  if (wl >= 0 && i - wl + 1 > a) a = i - wl + 1;", _window_check),
+    ("backward sign", "const double ds = prow[j] * (dp - Di);", "const double ds = prow[j] * (Di - dp);",
+     _bwd_check),
+]
+
+
+@pytest.mark.parametrize("name,old,new,check", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pin_catches_planted_mistake(tmp_path, name, old, new, check):
+    assert check(oracle), f"the real oracle fails the {name} check"
+    with np.errstate(all="ignore"):
+        assert not check(_mutant(tmp_path, old, new)), f"{name} went unnoticed"
