@@ -80,6 +80,16 @@ def _bwd_check(mod):
     return all(np.allclose(g, r, rtol=0, atol=1e-10) for g, r in zip(got, refs))
 
 
+def _online_check(mod):
+    lengths = [131, 45]
+    q, k, v = make_custom(0, 0, 2, 16, seed=9, lengths=lengths)
+    q = (q.float() * 4).to(torch.bfloat16)
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    o2, l2, _ = mod.fwd(_packed(q), _packed(k), _packed(v), cu, False, 0.25)
+    o1, l1, _ = mod.online_fwd(_packed(q), _packed(k), _packed(v), cu, False, 0.25, 16, 16, 0.0)
+    return np.allclose(o1, o2, rtol=0, atol=1e-12) and np.allclose(l1, l2, rtol=0, atol=1e-12)
+
+
 MUTATIONS = [
     ("dropped scale", "    srow[j - lo] = scale * acc;", "    srow[j - lo] = acc;",
      lambda m: _sdpa_check(m, False)),
@@ -92,6 +102,8 @@ MUTATIONS = [
      "  if (wl >= 0 && i - wl + 1 > a) a = i - wl + 1;", _window_check),
     ("backward sign", "const double ds = prow[j] * (dp - Di);", "const double ds = prow[j] * (Di - dp);",
      _bwd_check),
+    ("rescale factor inverted", "const double alpha = exp(m[r] - rowmax);",
+     "const double alpha = exp(rowmax - m[r]);", _online_check),
 ]
 
 
