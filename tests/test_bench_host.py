@@ -78,3 +78,21 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"] == "B1-H1-N256-d64"
+
+
+def test_input_recipe_varlen_lengths():
+    """The packed workload's lengths come from randint(512, 16385, 16) with seed 1."""
+    assert ai.varlen_lengths() == [2910, 7918, 11825, 6298, 15585, 5661, 2365, 9874, 11314, 11831,
+                                   4855, 1877, 14574, 2629, 15279, 1046]
+    assert ai.VARLEN.total_tokens == 125841 and ai.VARLEN.N == 15585
+
+
+def test_input_recipe_is_seeded_bf16():
+    import torch
+    a = ai.make_qkv(ai.TINY)
+    b = ai.make_qkv(ai.TINY)
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    assert all(x.dtype == torch.bfloat16 and tuple(x.shape) == (1, 256, 1, 64) for x in a)
+    q4 = ai.make_qkv(ai.DENSE_X4)[0]
+    q1 = ai.make_qkv(ai.DENSE)[0]
+    assert torch.equal(q4.float(), q1.float() * 4)  # exact: a power-of-two multiple
