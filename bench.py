@@ -104,22 +104,19 @@ def kernel_source_hash() -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary of this workload, or
-    None when there is none or it was taken on a different kernel source."""
-    path = os.path.join(ROOT, "profiles", f"fwd_kernel_{workload}.md")
+    """DRAM bytes per launch from the committed machine-readable ncu record of this
+    workload (``profiles/fwd_kernel_<workload>.json``), or None when there is none
+    or it was taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", f"fwd_kernel_{workload}.json")
     if not os.path.exists(path):
         return None
-    fields = {}
     with open(path) as f:
-        for line in f:
-            if line.startswith("- ") and ": " in line:
-                k, v = line[2:].strip().split(": ", 1)
-                fields[k.strip("`")] = v.strip().strip("`")
-    if fields.get("kernel_source_sha256") != kernel_source_hash():
+        rec = json.load(f)
+    if rec.get("kernel_source_sha256") != kernel_source_hash():
         return None
     try:
-        return float(fields["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
+        return float(rec["dram_bytes_per_launch"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 
@@ -244,7 +241,8 @@ def e4m3_scales(w: ai.Workload):
 def cpu_oracle_sample(w: ai.Workload, q, k, v, budget_s: float):
     """Times the fp64 oracle on whole (sequence, head) units of the workload until
     about budget_s of CPU time is spent; returns (TFLOP/s, threads, description).
-    E4M3 inputs are dequantised (x8 * scale) first, outside the timing."""
+    E4M3 inputs are dequantised (x8 * scale) first, outside the timing.  Returns
+    (TFLOP/s, threads, description, seconds spent)."""
     import numpy as np
     import oracle
     lengths = w.seq_lengths()
@@ -275,7 +273,7 @@ def cpu_oracle_sample(w: ai.Workload, q, k, v, budget_s: float):
         del sl
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     desc = f"{units} of {len(lengths) * w.H} (sequence, head) units, {done_flops / 1e9:.1f} GFLOP"
-    return done_flops / spent / 1e12, threads, desc
+    return done_flops / spent / 1e12, threads, desc, spent
 
 
 def bench_config(w: ai.Workload, world: int) -> dict:
@@ -285,29 +283,36 @@ def bench_config(w: ai.Workload, world: int) -> dict:
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle on the host cores.  Each step is a bounded
+    sample of the workload (whole (sequence, head) units until about --ref-seconds
+    of CPU time); value = the sample's FLOPs over its time, ms_per_step = the
+    sample's time (what was actually run), and the time the whole workload would
+    take at that rate is reported separately."""
     if rank != 0:
         return
     w = ai.ALL[args.workload]
     q, k, v, _ = make_inputs(w, "cpu")
     flops = workload_flops(w)
-    # warm-up: build / load the oracle
     import oracle
     oracle.build()
-    vals = []
-    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals, step_ms = [], []
+    per_step = args.ref_seconds
+    desc, threads = "", 0
     for i in range(args.warmup + args.steps):
-        tf, threads, desc = cpu_oracle_sample(w, q, k, v, per_step)
+        tf, threads, desc, spent = cpu_oracle_sample(w, q, k, v, per_step)
         if i >= args.warmup:
             vals.append(tf)
+            step_ms.append(spent * 1e3)
     value = statistics.median(vals)
-    ms = flops / (value * 1e12) * 1e3
     line = {"metric": metric_for(w), "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(step_ms),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": bench_config(w, world),
+            "step": f"a bounded sample of the workload: {desc}",
+            "workload_ms_at_this_rate": flops / (value * 1e12) * 1e3,
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                             "sample": desc + " per step; ms_per_step extrapolated to the workload"},
+                             "sample": desc + " per step"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -359,6 +364,20 @@ def run_ours(args, rank, world, local):
     total_ms = max_over_ranks(sum(times), world)
     ms_per_step = total_ms / args.steps
     value = whole_job_tflops(flops, args.steps, world, total_ms)
+
+    # One untimed launch with the kernel's counters on: how often the conditional
+    # rescale fired (the counters are not kept under a sliding window).
+    rescale = None
+    if w.window is None:
+        counters = torch.zeros(2, dtype=torch.int64, device=dev)
+        ea.fwd(q, k, v, causal=w.causal, scale=scale, cu_seqlens=cu, max_seqlen=max_len,
+               out=out, lse=lse, exp_poly_per8=args.exp_poly_per8, e4m3_scales=f8,
+               stats=counters)
+        ea.get_device_status()
+        rescaled, row_tiles = (int(x) for x in counters.cpu())
+        rescale = {"rows_rescaled": rescaled, "row_tiles_after_first": row_tiles,
+                   "skip_rate": (1.0 - rescaled / row_tiles) if row_tiles else None,
+                   "tau_log2": 4.0 if w.e4m3 else 8.0}
     achieved = flops / (statistics.mean(times) / 1e3) / 1e12  # per launch, this rank
     # An E4M3 contraction's peak: the measured bf16 burst peak x the nominal 2x
     # ratio of dense FP8 to BF16 tensor throughput.
@@ -372,6 +391,45 @@ def run_ours(args, rank, world, local):
     mufu_share = 1.0 - args.exp_poly_per8 / 8.0
     mufu_achieved = mufu_share * workload_exps(w) / (statistics.mean(times) / 1e3)
 
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(args, ea, w, q_h, k_h, v_h, cu_h, out, lse, scale, max_len, f8, dev,
+                          world, flops)
+    barrier(world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, threads, desc, _ = cpu_oracle_sample(w, q_h, k_h, v_h, args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {"metric": metric_for(w), "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "e4m3" if w.e4m3 else "bf16", "data": "synthetic",
+                "config": bench_config(w, world),
+                "options": {"exp_poly_per8": args.exp_poly_per8},
+                "rescale": rescale,
+                "pct_of_peak": 100.0 * achieved / peak,
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                             "unit": "TFLOP/s", "frac": achieved / peak,
+                             "peak_source": peak_source,
+                             "traffic": profiled_traffic(w.name),
+                             "traffic_unit": "bytes per launch (ncu dram read+write)"},
+                "mufu": {"achieved_ex2_per_s": mufu_achieved, "peak_ex2_per_s": mufu_peak,
+                         "frac": mufu_achieved / mufu_peak,
+                         "mufu_share_of_exps": mufu_share,
+                         "note": "ex2 executed on MUFU (the rest on the FMA-pipe polynomial); "
+                                 "peak = SMs x 16 ex2/clk at the median sampled SM clock"},
+                "e2e": e2e,
+                "gpu_launches": args.steps,
+                "clocks": clk,
+                "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+
+
+def measure_e2e(args, ea, w, q_h, k_h, v_h, cu_h, out, lse, scale, max_len, f8, dev, world,
+                flops):
     # End to end through the public API from pinned host buffers: every call copies
     # its Q/K/V (and cu_seqlens) to the device, runs the forward and copies O and
     # LSE back; HostPipeline overlaps neighbouring calls' copies with compute.
@@ -399,37 +457,9 @@ def run_ours(args, rank, world, local):
     d2h = o_h.numel() * 2 + l_h.numel() * 4
     barrier(world)
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, threads, desc = cpu_oracle_sample(w, q_h, k_h, v_h, args.cpu_seconds)
-        cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
-
-    if rank == 0:
-        line = {"metric": metric_for(w), "value": value, "unit": "TFLOP/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "e4m3" if w.e4m3 else "bf16", "data": "synthetic",
-                "config": dict(bench_config(w, world), exp_poly_per8=args.exp_poly_per8),
-                "pct_of_peak": 100.0 * achieved / peak,
-                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
-                             "unit": "TFLOP/s", "frac": achieved / peak,
-                             "peak_source": peak_source,
-                             "traffic": profiled_traffic(w.name),
-                             "traffic_unit": "bytes per launch (ncu dram read+write)"},
-                "mufu": {"achieved_ex2_per_s": mufu_achieved, "peak_ex2_per_s": mufu_peak,
-                         "frac": mufu_achieved / mufu_peak,
-                         "mufu_share_of_exps": mufu_share,
-                         "note": "ex2 executed on MUFU (the rest on the FMA-pipe polynomial); "
-                                 "peak = SMs x 16 ex2/clk at the median sampled SM clock"},
-                "e2e": {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                        "ms_per_step": e2e_ms,
-                        "api": "HostPipeline (2 device buffer sets, copy-in / compute / "
-                               "copy-out streams)"},
-                "gpu_launches": args.steps,
-                "clocks": clk,
-                "cpu_baseline": cpu}
-        print(json.dumps(line), flush=True)
+    return {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+            "api": "HostPipeline (2 device buffer sets, copy-in / compute / copy-out streams)"}
 
 
 def run_bwd(args, rank, world, local):
@@ -486,10 +516,15 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=ai.DENSE.name, choices=sorted(ai.ALL) + [ai.BWD_NAME])
+    ap.add_argument("--workload", default=ai.VARLEN.name, choices=sorted(ai.ALL) + [ai.BWD_NAME])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU time of the cpu_baseline sample (our arm, rank 0, N=1)")
+    ap.add_argument("--ref-seconds", type=float, default=2.0,
+                    help="CPU time of each reference-arm step (a bounded sample)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg (profiling runs only)")
     ap.add_argument("--exp-poly-per8", type=int, default=0, choices=[0, 2, 8],
                     help="exponential pairs of every 8 computed by the FMA-pipe polynomial")
     args = ap.parse_args()

@@ -39,7 +39,8 @@ class BwdOpts(ctypes.Structure):
     _fields_ = [("has_window", ctypes.c_int),
                 ("window_left", ctypes.c_int),
                 ("window_right", ctypes.c_int),
-                ("timeout_ns", ctypes.c_uint64)]
+                ("timeout_ns", ctypes.c_uint64),
+                ("total_tokens", ctypes.c_int64)]
 
 
 class FwdOpts(ctypes.Structure):
@@ -325,11 +326,14 @@ class HostPipeline:
 def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                 lse: torch.Tensor, causal: bool = False, scale: Optional[float] = None,
                 cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: Optional[int] = None,
-                check: bool = True, stream: Optional[torch.cuda.Stream] = None) -> None:
+                total_tokens: Optional[int] = None, check: bool = True,
+                stream: Optional[torch.cuda.Stream] = None) -> None:
     """The allocation-free forward ``attn_fwd_noalloc``: the caller supplies ``out``
     and ``lse`` (layouts as for ``fwd``); the library allocates no device memory.
-    With ``check`` the call synchronises the stream and raises on a kernel-recorded
-    error."""
+    Varlen: ``total_tokens`` must equal ``cu_seqlens[B]`` (default: ``q.shape[0]``;
+    pass it for a packed buffer longer than the batch).  With ``check`` the call
+    synchronises the stream and raises on a kernel-recorded error; without it that
+    status is not reported anywhere."""
     lib = load_library()
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
         _need(t, n)
@@ -342,7 +346,8 @@ def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Te
     else:
         _need(cu_seqlens, "cu_seqlens", torch.int32)
         B, H, N = cu_seqlens.numel() - 1, q.shape[1], int(max_seqlen)
-        total, cu_ptr = q.shape[0], cu_seqlens.data_ptr()
+        total = q.shape[0] if total_tokens is None else int(total_tokens)
+        cu_ptr = cu_seqlens.data_ptr()
     with torch.cuda.device(q.device):
         st = lib.attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                   lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
@@ -378,7 +383,8 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse:
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
     with torch.cuda.device(q.device):
         opts = BwdOpts(0 if window is None else 1, -1 if window is None else int(window[0]),
-                       -1 if window is None else int(window[1]), 0)
+                       -1 if window is None else int(window[1]), 0,
+                       0 if cu_seqlens is None else int(total))
         st = lib.attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                              lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
                              dv.data_ptr(), B, H, N, d, int(bool(causal)), float(scale), cu_ptr,

@@ -12,6 +12,7 @@
 #include "../../include/attn.h"
 #include "attn_fwd_sm100.h"
 #include "attn_bwd_sm100.h"
+#include "attn_internal.h"
 
 namespace {
 
@@ -130,128 +131,10 @@ attn_status_t select_mask(int N, int causal, int has_window, int wl, int wr, att
   return ATTN_OK;
 }
 
-// Per-tensor scales of the E4M3 entry point (real value = stored value * scale).
-struct E4m3Scales {
-  float q, k, v;
-};
-
-attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                       int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
-                       int64_t total_hint, const attn_fwd_opts_t* opts, attn_stream_t stream,
-                       const E4m3Scales* f8 = nullptr) {
-  if (B < 0 || H <= 0 || N < 0) return fail(ATTN_ERR_INVALID_ARG, "B=%d H=%d N=%d", B, H, N);
-  if (f8 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "E4M3 path: head dim %d (supported: 128)", d);
-  if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
-  if (!(std::isfinite(scale) && scale > 0.f)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite and > 0");
-  if (f8 && !(std::isfinite(f8->q) && f8->q > 0.f && std::isfinite(f8->k) && f8->k > 0.f &&
-              std::isfinite(f8->v) && f8->v > 0.f))
-    return fail(ATTN_ERR_INVALID_ARG, "E4M3 scales must be finite and > 0");
-  if (B == 0 || N == 0) return ATTN_OK;
-  if (!q || !k || !v || !o || !lse) return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
-    return fail(ATTN_ERR_INVALID_ARG, "q/k/v/o must be 16-byte aligned and lse 4-byte aligned");
-  const bool varlen = cu_seqlens != nullptr;
-  if (varlen && (B > kMaxVarlenB || N > kMaxVarlenN))
-    return fail(ATTN_ERR_UNSUPPORTED, "varlen supports B <= %d and N <= %d", kMaxVarlenB, kMaxVarlenN);
-  const int64_t T256 = (static_cast<int64_t>(N) + 255) / 256;
-  const int64_t items_bound = static_cast<int64_t>(B) * T256 * H;
-  const int64_t dense_tokens = static_cast<int64_t>(B) * N;
-  if (items_bound > INT32_MAX / 2 || dense_tokens * H > INT64_MAX / 256 || dense_tokens > INT32_MAX)
-    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for 32-bit tile indexing");
-  if (varlen && !aligned(cu_seqlens, 4)) return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens misaligned");
-  float tau = f8 ? kDefaultTauE4m3 : kDefaultTau;
-  uint64_t timeout = kDefaultTimeoutNs;
-  unsigned long long* stats = nullptr;
-  int test_fault = 0, poly = 0, has_window = 0, wl = -1, wr = -1;
-  if (opts) {
-    if (opts->test_fault != 0 && opts->test_fault != 1)
-      return fail(ATTN_ERR_INVALID_ARG, "test_fault must be 0 or 1");
-    test_fault = opts->test_fault;
-    if (opts->rescale_threshold >= 0.f) tau = opts->rescale_threshold;
-    if (!(tau <= 64.f)) return fail(ATTN_ERR_INVALID_ARG, "rescale_threshold must be <= 64");
-    if (opts->timeout_ns) timeout = opts->timeout_ns;
-    stats = opts->stats;
-    if (stats && !aligned(stats, 8)) return fail(ATTN_ERR_INVALID_ARG, "stats misaligned");
-    poly = opts->exp_poly_per8;
-    if (poly != 0 && poly != 2 && poly != 8)
-      return fail(ATTN_ERR_INVALID_ARG, "exp_poly_per8 must be 0, 2 or 8");
-    if (f8 && poly != 0 && poly != 2)
-      return fail(ATTN_ERR_UNSUPPORTED, "E4M3 path: exp_poly_per8 must be 0 or 2");
-    if (f8 && !(tau <= 8.f))
-      return fail(ATTN_ERR_INVALID_ARG, "E4M3 path: rescale_threshold must be <= 8 (P~ <= 256 < 448)");
-    if (opts->has_window) {
-      has_window = 1;
-      wl = opts->window_left;
-      wr = opts->window_right;
-    }
-  }
-  attn::MaskKind mask;
-  int win_l, win_r;
-  attn_status_t st = select_mask(N, causal, has_window, wl, wr, &mask, &win_l, &win_r);
-  if (st != ATTN_OK) return st;
-  if (mask == attn::kMaskWindow) stats = nullptr;  // counters are not kept under a window
-
-  DeviceState* dev = nullptr;
-  st = device_state(&dev);
-  if (st != ATTN_OK) return st;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-
-  int64_t total = dense_tokens;
-  if (varlen) {
-    if (total_hint >= 0) {
-      total = total_hint;
-    } else {
-      // The TMA views need the packed token count; read cu_seqlens[B] (4 bytes).
-      int32_t t = 0;
-      cudaError_t e = cudaMemcpyAsync(&t, cu_seqlens + B, sizeof(int32_t), cudaMemcpyDeviceToHost, cs);
-      if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
-      if (e != cudaSuccess) return cuda_fail(e, "reading cu_seqlens[B]");
-      total = t;
-    }
-    if (total < 0 || total > dense_tokens)
-      return fail(ATTN_ERR_INVALID_ARG, "packed token count %lld outside [0, B*N]", (long long)total);
-    if (total == 0) return ATTN_OK;
-  }
-
-  attn::FwdLaunch a;
-  std::memset(&a, 0, sizeof(a));
-  const int esz = f8 ? 1 : 2;
-  if (!make_map_esz(&a.tm_q, q, total, H, d, esz) || !make_map_esz(&a.tm_k, k, total, H, d, esz) ||
-      !make_map_esz(&a.tm_v, v, total, H, d, esz))
-    return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled rejected the Q/K/V views");
-  a.p.o = static_cast<__nv_bfloat16*>(o);
-  a.p.lse = lse;
-  a.p.cu_seqlens = cu_seqlens;
-  a.p.B = B;
-  a.p.H = H;
-  a.p.N = N;
-  a.p.T = static_cast<int>(T256);
-  a.p.total = static_cast<int>(total);
-  // The E4M3 scales of Q and K fold into the score scale; V's into 1/l.
-  a.p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634 *
-                                      (f8 ? static_cast<double>(f8->q) * f8->k : 1.0));
-  a.p.o_scale = f8 ? f8->v : 1.f;
-  a.p.p_shift = f8 ? std::floor(8.f - tau) : 0.f;
-  a.p.tau = tau;
-  a.p.err = dev->err;
-  a.p.stats = stats;
-  a.p.timeout_ns = timeout;
-  a.p.test_fault = test_fault;
-  a.p.wl = win_l;
-  a.p.wr = win_r;
-  // Dense unmasked launches may split their last wave into half items (see the
-  // kernel), so up to twice as many CTAs can be useful there.
-  const int64_t useful = (!varlen && mask == attn::kMaskNone) ? 2 * items_bound : items_bound;
-  a.grid = static_cast<int>(useful < dev->sms ? useful : dev->sms);
-  a.smem = attn::fwd_smem_bytes(d, B, static_cast<int>(T256), varlen ? 1 : 0, f8 ? 1 : 0);
-  const cudaError_t e = attn::launch_fwd(a, d, mask, poly, f8 ? 1 : 0, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
-  return ATTN_OK;
-}
-
 }  // namespace
 
 namespace attn_internal {
+
 // Device preparation and the TMA view builder, for the diagnostic entry point.
 attn_status_t prepare_selftest(int** err, bool (**mk)(CUtensorMap*, const void*, int64_t, int, int)) {
   DeviceState* dev = nullptr;
@@ -261,8 +144,7 @@ attn_status_t prepare_selftest(int** err, bool (**mk)(CUtensorMap*, const void*,
   *mk = make_map;
   return ATTN_OK;
 }
-// Pieces shared with the allocation-free entry point (attn_noalloc.cu).  None of
-// them allocates device memory.
+
 attn_status_t load_tensor_map_encoder() {
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_encode) return ATTN_OK;
@@ -274,28 +156,173 @@ attn_status_t load_tensor_map_encoder() {
   g_encode = reinterpret_cast<EncodeTiledFn>(fn);
   return ATTN_OK;
 }
-bool make_tensor_map(CUtensorMap* m, const void* ptr, int64_t total, int H, int d) {
-  return make_map(m, ptr, total, H, d);
-}
+
+attn_status_t report(attn_status_t s, const char* message) { return fail(s, "%s", message); }
+
 bool make_tensor_map_e4m3(CUtensorMap* m, const void* ptr, int64_t total, int H, int d) {
   return make_map_esz(m, ptr, total, H, d, 1);
 }
-attn_status_t report(attn_status_t s, const char* message) { return fail(s, "%s", message); }
+
+attn_status_t plan_fwd(const FwdCall& c, FwdPlan* pl) {
+  const int B = c.B, H = c.H, N = c.N, d = c.d;
+  const attn_internal::E4m3Scales* f8 = c.f8;
+  std::memset(pl, 0, sizeof(*pl));
+  if (B < 0 || H <= 0 || N < 0) return fail(ATTN_ERR_INVALID_ARG, "B=%d H=%d N=%d", B, H, N);
+  if (f8 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "E4M3 path: head dim %d (supported: 128)", d);
+  if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (!(std::isfinite(c.scale) && c.scale > 0.f))
+    return fail(ATTN_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (f8 && !(std::isfinite(f8->q) && f8->q > 0.f && std::isfinite(f8->k) && f8->k > 0.f &&
+              std::isfinite(f8->v) && f8->v > 0.f))
+    return fail(ATTN_ERR_INVALID_ARG, "E4M3 scales must be finite and > 0");
+  if (B == 0 || N == 0) {
+    pl->noop = true;
+    return ATTN_OK;
+  }
+  if (!c.q || !c.k || !c.v || !c.o || !c.lse) return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned(c.q, 16) || !aligned(c.k, 16) || !aligned(c.v, 16) || !aligned(c.o, 16) ||
+      !aligned(c.lse, 4))
+    return fail(ATTN_ERR_INVALID_ARG, "q/k/v/o must be 16-byte aligned and lse 4-byte aligned");
+  const bool varlen = c.cu_seqlens != nullptr;
+  if (varlen && (B > kMaxVarlenB || N > kMaxVarlenN))
+    return fail(ATTN_ERR_UNSUPPORTED, "varlen supports B <= %d and N <= %d", kMaxVarlenB, kMaxVarlenN);
+  pl->T256 = (static_cast<int64_t>(N) + 255) / 256;
+  pl->items_bound = static_cast<int64_t>(B) * pl->T256 * H;
+  pl->dense_tokens = static_cast<int64_t>(B) * N;
+  if (pl->items_bound > INT32_MAX / 2 || pl->dense_tokens * H > INT64_MAX / 256 ||
+      pl->dense_tokens > INT32_MAX)
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large for 32-bit tile indexing");
+  if (varlen && !aligned(c.cu_seqlens, 4)) return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens misaligned");
+  pl->tau = f8 ? kDefaultTauE4m3 : kDefaultTau;
+  pl->timeout = kDefaultTimeoutNs;
+  int has_window = 0, wl = -1, wr = -1;
+  if (const attn_fwd_opts_t* opts = c.opts) {
+    if (opts->test_fault != 0 && opts->test_fault != 1)
+      return fail(ATTN_ERR_INVALID_ARG, "test_fault must be 0 or 1");
+    pl->test_fault = opts->test_fault;
+    if (opts->rescale_threshold >= 0.f) pl->tau = opts->rescale_threshold;
+    if (!(pl->tau <= 64.f)) return fail(ATTN_ERR_INVALID_ARG, "rescale_threshold must be <= 64");
+    if (opts->timeout_ns) pl->timeout = opts->timeout_ns;
+    pl->stats = opts->stats;
+    if (pl->stats && !aligned(pl->stats, 8)) return fail(ATTN_ERR_INVALID_ARG, "stats misaligned");
+    pl->poly = opts->exp_poly_per8;
+    if (pl->poly != 0 && pl->poly != 2 && pl->poly != 8)
+      return fail(ATTN_ERR_INVALID_ARG, "exp_poly_per8 must be 0, 2 or 8");
+    if (f8 && pl->poly != 0 && pl->poly != 2)
+      return fail(ATTN_ERR_UNSUPPORTED, "E4M3 path: exp_poly_per8 must be 0 or 2");
+    if (f8 && !(pl->tau <= 8.f))
+      return fail(ATTN_ERR_INVALID_ARG, "E4M3 path: rescale_threshold must be <= 8 (P~ <= 256 < 448)");
+    if (opts->has_window) {
+      has_window = 1;
+      wl = opts->window_left;
+      wr = opts->window_right;
+    }
+  }
+  const attn_status_t st = select_mask(N, c.causal, has_window, wl, wr, &pl->mask, &pl->win_l, &pl->win_r);
+  if (st != ATTN_OK) return st;
+  if (pl->mask == attn::kMaskWindow) pl->stats = nullptr;  // counters are not kept under a window
+  return ATTN_OK;
+}
+
+attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total, int sms, int* err,
+                              attn::FwdLaunch* a) {
+  const attn_status_t st = load_tensor_map_encoder();
+  if (st != ATTN_OK) return st;
+  std::memset(a, 0, sizeof(*a));
+  const attn_internal::E4m3Scales* f8 = c.f8;
+  const int esz = f8 ? 1 : 2;
+  if (!make_map_esz(&a->tm_q, c.q, total, c.H, c.d, esz) || !make_map_esz(&a->tm_k, c.k, total, c.H, c.d, esz) ||
+      !make_map_esz(&a->tm_v, c.v, total, c.H, c.d, esz))
+    return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled rejected the Q/K/V views");
+  const bool varlen = c.cu_seqlens != nullptr;
+  a->p.o = static_cast<__nv_bfloat16*>(c.o);
+  a->p.lse = c.lse;
+  a->p.cu_seqlens = c.cu_seqlens;
+  a->p.B = c.B;
+  a->p.H = c.H;
+  a->p.N = c.N;
+  a->p.T = static_cast<int>(pl.T256);
+  a->p.total = static_cast<int>(total);
+  // The E4M3 scales of Q and K fold into the score scale; V's into 1/l.  One
+  // rounding to fp32, from a double product.
+  a->p.scale_log2 = static_cast<float>(static_cast<double>(c.scale) * 1.4426950408889634 *
+                                       (f8 ? static_cast<double>(f8->q) * f8->k : 1.0));
+  a->p.o_scale = f8 ? f8->v : 1.f;
+  a->p.p_shift = f8 ? std::floor(8.f - pl.tau) : 0.f;
+  a->p.tau = pl.tau;
+  a->p.err = err;
+  a->p.stats = pl.stats;
+  a->p.timeout_ns = pl.timeout;
+  a->p.test_fault = pl.test_fault;
+  a->p.wl = pl.win_l;
+  a->p.wr = pl.win_r;
+  // Dense unmasked launches may split their last wave into half items (see the
+  // kernel), so up to twice as many CTAs can be useful there.
+  const int64_t useful = (!varlen && pl.mask == attn::kMaskNone) ? 2 * pl.items_bound : pl.items_bound;
+  a->grid = static_cast<int>(useful < sms ? useful : sms);
+  a->smem = attn::fwd_smem_bytes(c.d, c.B, static_cast<int>(pl.T256), varlen ? 1 : 0, f8 ? 1 : 0);
+  return ATTN_OK;
+}
+
+attn_status_t launch_planned_fwd(const FwdCall& c, const FwdPlan& pl, const attn::FwdLaunch& a,
+                                 attn_stream_t stream) {
+  const cudaError_t e = attn::launch_fwd(a, c.d, pl.mask, pl.poly, c.f8 ? 1 : 0,
+                                         reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "forward kernel launch");
+  return ATTN_OK;
+}
+
 }  // namespace attn_internal
+
+namespace {
+
+attn_status_t fwd_impl(const attn_internal::FwdCall& c, int64_t total_hint, attn_stream_t stream) {
+  attn_internal::FwdPlan pl;
+  attn_status_t st = attn_internal::plan_fwd(c, &pl);
+  if (st != ATTN_OK || pl.noop) return st;
+  DeviceState* dev = nullptr;
+  st = device_state(&dev);
+  if (st != ATTN_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  int64_t total = pl.dense_tokens;
+  if (c.cu_seqlens) {
+    if (total_hint >= 0) {
+      total = total_hint;
+    } else {
+      // The TMA views need the packed token count; read cu_seqlens[B] (4 bytes).
+      int32_t t = 0;
+      cudaError_t e = cudaMemcpyAsync(&t, c.cu_seqlens + c.B, sizeof(int32_t), cudaMemcpyDeviceToHost, cs);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+      if (e != cudaSuccess) return cuda_fail(e, "reading cu_seqlens[B]");
+      total = t;
+    }
+    if (total < 0 || total > pl.dense_tokens)
+      return fail(ATTN_ERR_INVALID_ARG, "packed token count %lld outside [0, B*N]", (long long)total);
+    if (total == 0) return ATTN_OK;
+  }
+  attn::FwdLaunch a;
+  st = attn_internal::fill_fwd_launch(c, pl, total, dev->sms, dev->err, &a);
+  if (st != ATTN_OK) return st;
+  return attn_internal::launch_planned_fwd(c, pl, a, stream);
+}
+
+}  // namespace
 
 extern "C" {
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                        int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
                        attn_stream_t stream) {
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, -1, nullptr, stream);
+  const attn_internal::FwdCall c{q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, nullptr, nullptr};
+  return fwd_impl(c, -1, stream);
 }
 
 attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                           int H, int N, int d, int causal, float scale, const int32_t* cu_seqlens,
                           const attn_fwd_opts_t* opts, attn_stream_t stream) {
   const int64_t hint = (opts && opts->total_tokens > 0) ? opts->total_tokens : -1;
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, hint, opts, stream);
+  const attn_internal::FwdCall c{q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, opts, nullptr};
+  return fwd_impl(c, hint, stream);
 }
 
 attn_status_t attn_fwd_e4m3(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -303,8 +330,9 @@ attn_status_t attn_fwd_e4m3(const void* q, const void* k, const void* v, void* o
                             float k_scale, float v_scale, const int32_t* cu_seqlens,
                             const attn_fwd_opts_t* opts, attn_stream_t stream) {
   const int64_t hint = (opts && opts->total_tokens > 0) ? opts->total_tokens : -1;
-  const E4m3Scales f8{q_scale, k_scale, v_scale};
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, hint, opts, stream, &f8);
+  const attn_internal::E4m3Scales f8{q_scale, k_scale, v_scale};
+  const attn_internal::FwdCall c{q, k, v, o, lse, B, H, N, d, causal, scale, cu_seqlens, opts, &f8};
+  return fwd_impl(c, hint, stream);
 }
 
 }  // extern "C"
@@ -344,11 +372,15 @@ attn_status_t bwd_impl(const void* q, const void* k, const void* v, const void* 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   int64_t total = dense_tokens;
   if (varlen) {
-    int32_t t = 0;
-    cudaError_t e = cudaMemcpyAsync(&t, cu_seqlens + B, sizeof(int32_t), cudaMemcpyDeviceToHost, cs);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
-    if (e != cudaSuccess) return cuda_fail(e, "reading cu_seqlens[B]");
-    total = t;
+    if (opts && opts->total_tokens > 0) {
+      total = opts->total_tokens;  // checked against cu_seqlens[B] on the device
+    } else {
+      int32_t t = 0;
+      cudaError_t e = cudaMemcpyAsync(&t, cu_seqlens + B, sizeof(int32_t), cudaMemcpyDeviceToHost, cs);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+      if (e != cudaSuccess) return cuda_fail(e, "reading cu_seqlens[B]");
+      total = t;
+    }
     if (total < 0 || total > dense_tokens)
       return fail(ATTN_ERR_INVALID_ARG, "packed token count %lld outside [0, B*N]", (long long)total);
     if (total == 0) return ATTN_OK;

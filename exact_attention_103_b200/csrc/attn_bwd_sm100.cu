@@ -38,7 +38,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 __host__ __device__ constexpr int timeout_code(int site) { return 4 | (site << 8); }
 enum BwdSite { kSiteKv = 32, kSiteStageFull, kSiteStageEmpty, kSiteS, kSiteP, kSiteDs, kSiteAcc,
-               kSiteDrain };
+               kSiteDrain, kSiteBadLen };
 
 template <int D>
 struct BwdLayout {
@@ -85,6 +85,11 @@ __device__ __forceinline__ uint32_t packed_col(int kk) { return (kk < 4) ? kk * 
 struct BwdItem {
   int b, h, tile, seq_start, L;
 };
+// False when the CTA has no work.  Varlen: a sequence whose bounds fall outside
+// [0, total) or whose length exceeds ntiles * 128 is not processed (its CTAs write
+// nothing) and ATTN_ERR_INVALID_ARG is recorded in the device error word, as is
+// cu[0] != 0 or cu[B] != total; so a malformed cu_seqlens never makes a store
+// leave the packed tensors.
 __device__ __forceinline__ bool decode_block(const BwdParams& p, bool key_tiles, bool causal,
                                              BwdItem& it) {
   const int nbh = p.B * p.H;
@@ -97,8 +102,16 @@ __device__ __forceinline__ bool decode_block(const BwdParams& p, bool key_tiles,
     it.seq_start = it.b * p.N;
     it.L = p.N;
   } else {
-    it.seq_start = __ldg(p.cu_seqlens + it.b);
-    it.L = __ldg(p.cu_seqlens + it.b + 1) - it.seq_start;
+    const int c0 = __ldg(p.cu_seqlens + it.b), c1 = __ldg(p.cu_seqlens + it.b + 1);
+    const bool bad = c0 < 0 || c1 < c0 || c1 > p.total ||
+                     static_cast<int64_t>(c1 - c0) > static_cast<int64_t>(p.ntiles) * kTile;
+    const bool bad_ends = idx == 0 && (__ldg(p.cu_seqlens) != 0 || __ldg(p.cu_seqlens + p.B) != p.total);
+    if (bad || bad_ends) {
+      if (threadIdx.x == 0 && p.err) atomicCAS(p.err, 0, 1 | (kSiteBadLen << 8));
+      if (bad) return false;
+    }
+    it.seq_start = c0;
+    it.L = c1 - c0;
   }
   return it.tile * kTile < it.L;
 }

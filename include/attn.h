@@ -165,7 +165,8 @@ ATTN_API attn_status_t attn_fwd_e4m3(const void* q, const void* k, const void* v
  * compatibility and changes nothing.  `workspace` is a caller-owned DEVICE buffer
  * of at least attn_bwd_workspace_size(...) bytes, 256-byte aligned (may be NULL
  * when that size is 0); too small or misaligned: ATTN_ERR_WORKSPACE.  Same limits
- * as the forward (d in {64, 128}); varlen reads cu_seqlens[B] back to the host.
+ * as the forward (d in {64, 128}); varlen reads cu_seqlens[B] back to the host
+ * (attn_bwd_ex with opts->total_tokens avoids that).
  */
 ATTN_API attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
                        const float* lse, const void* dout, void* dq, void* dk, void* dv,
@@ -177,12 +178,20 @@ ATTN_API attn_status_t attn_bwd(const void* q, const void* k, const void* v, con
  *  has_window, window_left, window_right: the sliding-window mask of the forward
  *      call whose gradients are wanted, with the meaning they have in
  *      attn_fwd_opts_t (the mask hook; the causal flag still applies on top).
- *  timeout_ns: limit of every internal wait; 0 selects the default (2 s). */
+ *  timeout_ns: limit of every internal wait; 0 selects the default (2 s).
+ *  total_tokens: varlen only; if > 0 it must equal cu_seqlens[B] and the call does
+ *      not synchronise `stream`; when 0, cu_seqlens[B] is read back to the host
+ *      (a 4-byte copy and a stream synchronisation).  Either way the kernels check
+ *      cu_seqlens on the device: cu[0] != 0, cu[B] != the token count, a negative
+ *      length or one above N make them record ATTN_ERR_INVALID_ARG in the device
+ *      error word, and the sequences concerned are not processed (their gradients
+ *      are left unwritten). */
 typedef struct {
   int has_window;
   int window_left;
   int window_right;
   uint64_t timeout_ns;
+  int64_t total_tokens;
 } attn_bwd_opts_t;
 
 /* attn_bwd with options (opts may be NULL = attn_bwd).  Under a window both
@@ -206,13 +215,19 @@ ATTN_API size_t attn_bwd_workspace_size(int B, int H, int N, int d, int total_to
  * this is an interface of this library.)  The ordinary entry points allocate a
  * 4-byte device status word on a device's first call; here that scratch lives in
  * a static device array of 256 bytes inside the library, which every GPU that
- * loads the library holds until the process exits.  Same operation, layouts and
- * limits as attn_fwd, default rescale threshold.
- *  - total_tokens: varlen only, must equal cu_seqlens[B] (no device read-back);
- *    ignored for dense batches.
- *  - check: 0 = return after launching; != 0 = synchronise `stream` and return the
- *    status the kernel recorded (ATTN_ERR_TIMEOUT, or ATTN_ERR_INVALID_ARG for bad
- *    cu_seqlens).
+ * loads the library holds until the process exits.  Same operation, layouts,
+ * argument checks and limits as attn_fwd, default rescale threshold; the same
+ * kernel runs with the same parameters, so O and LSE are bitwise equal to
+ * attn_fwd's.
+ *  - total_tokens: varlen only, must equal cu_seqlens[B] (there is no device
+ *    read-back; the kernel checks it); 0 is an empty packed batch (nothing is
+ *    launched, ATTN_OK); ignored for dense batches.
+ *  - check: != 0 = synchronise `stream` and return the status the kernel recorded
+ *    (ATTN_ERR_TIMEOUT, or ATTN_ERR_INVALID_ARG for bad cu_seqlens).  0 = return
+ *    after launching; the kernel's status then stays in the static array, where
+ *    attn_get_device_status does NOT see it (that reads the ordinary entry points'
+ *    word), until the next call of this entry point clears it: a caller that needs
+ *    the status must pass check != 0.
  *  - The first call on a device does its set-up there (looks up the array's
  *    device address); make that first call before any stream capture.
  *  - Every call shares the array: each call clears the status word on `stream`

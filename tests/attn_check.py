@@ -1,10 +1,18 @@
 """Comparison helpers for GPU-vs-oracle parity tests (no attention arithmetic here).
 
-Tolerances (forward): max-abs error of O <= 1e-2 plus half a bf16 ulp of the exact
-value (the output is bf16, so rounding the exact result alone can cost half an
-ulp: 1.6e-2 where |O| >= 4), relative L2 error of O <= 5e-3, LSE abs error <= 1e-3.
+Tolerances (forward), the stated bar: max-abs error of O <= 1e-2, relative L2
+error of O <= 5e-3, LSE abs error <= 1e-3.  One reading: O is bf16, so rounding
+the exact result alone can cost half a bf16 ulp, 1.6e-2 where |O| >= 4; on inputs
+whose outputs reach that size (Q scaled by 4) the raw 1e-2 bar is not attainable
+by any bf16 output, and those comparisons use the gate
+|O - O_ref| <= 1e-2 + half a bf16 ulp of O_ref instead (``raw_bar=False``); every
+other comparison asserts the raw bar.  Every comparison can append its figures to
+the JSON-lines file named by the environment variable ATTN_PARITY_LOG.
 """
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 import torch
@@ -12,6 +20,15 @@ import torch
 O_MAX_ABS = 1e-2
 O_REL_L2 = 5e-3
 LSE_ABS = 1e-3
+
+
+def log_parity(label: str, **figures) -> None:
+    """Appends {"label": ..., figures...} to $ATTN_PARITY_LOG (when set)."""
+    path = os.environ.get("ATTN_PARITY_LOG")
+    if not path:
+        return
+    with open(path, "a") as f:
+        f.write(json.dumps(dict(label=label, **figures)) + "\n")
 
 
 def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
@@ -27,28 +44,38 @@ def to_np(t) -> np.ndarray:
     return np.asarray(t, dtype=np.float64)
 
 
-def compare_o(o_gpu, o_ref, label: str = ""):
-    """Asserts the forward-output bar; returns (raw max-abs, rel-L2)."""
+def compare_o(o_gpu, o_ref, label: str = "", raw_bar: bool = True):
+    """Asserts the forward-output bar; returns (raw max-abs, rel-L2).
+
+    raw_bar: assert max-abs <= 1e-2 itself (else the half-ulp gate of the module
+    docstring, for inputs whose outputs reach |O| >= 2)."""
     o, r = to_np(o_gpu), to_np(o_ref)
     assert o.shape == r.shape, (o.shape, r.shape)
     assert np.all(np.isfinite(o)), f"{label}: non-finite output"
     err = np.abs(o - r)
-    bound = O_MAX_ABS + bf16_half_ulp(r)
-    worst = np.argmax(err - bound)
-    assert np.all(err <= bound), (
+    bound = O_MAX_ABS if raw_bar else O_MAX_ABS + bf16_half_ulp(r)
+    excess = err - bound
+    worst = int(np.argmax(excess))
+    bnd = bound if np.isscalar(bound) else bound.flat[worst]
+    assert np.all(excess <= 0), (
         f"{label}: |O-O_ref| = {err.flat[worst]:.3e} at {np.unravel_index(worst, err.shape)} "
-        f"exceeds {bound.flat[worst]:.3e} (ref {r.flat[worst]:.4f}, got {o.flat[worst]:.4f})")
+        f"exceeds {bnd:.3e} (ref {r.flat[worst]:.4f}, got {o.flat[worst]:.4f})")
     rel = float(np.linalg.norm(o - r) / max(np.linalg.norm(r), 1e-30))
     assert rel <= O_REL_L2, f"{label}: rel-L2 {rel:.3e} > {O_REL_L2}"
-    return float(err.max()), rel
+    max_abs = float(err.max()) if err.size else 0.0
+    log_parity(label, o_max_abs=max_abs, o_rel_l2=rel, raw_bar=raw_bar, elements=int(err.size))
+    return max_abs, rel
 
 
 def compare_lse(lse_gpu, lse_ref, label: str = ""):
     l, r = to_np(lse_gpu), to_np(lse_ref)
     assert l.shape == r.shape, (l.shape, r.shape)
+    assert np.all(np.isfinite(l)), f"{label}: non-finite LSE"
     err = np.abs(l - r)
     assert np.all(err <= LSE_ABS), f"{label}: LSE error {err.max():.3e} > {LSE_ABS}"
-    return float(err.max())
+    max_abs = float(err.max()) if err.size else 0.0
+    log_parity(label, lse_max_abs=max_abs, elements=int(err.size))
+    return max_abs
 
 
 # E4M3 forward (attn_fwd_e4m3), against the exact attention of the dequantised

@@ -66,9 +66,12 @@ def test_reference_arm_prints_one_contract_line():
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    import time
+    t0 = time.time()
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2",
-                        "--warmup", "3", "--workload", "B1-H1-N256-d64"],
+                        "--warmup", "3", "--workload", "B1-H1-N256-d64", "--ref-seconds", "0.5"],
                        capture_output=True, text=True, cwd=root, timeout=600)
+    wall = time.time() - t0
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
@@ -78,6 +81,20 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"] == "B1-H1-N256-d64"
+    # the steps it reports are the steps it ran: they fit in the process's wall time
+    assert d["steps"] * d["ms_per_step"] / 1e3 <= wall
+    assert d["config"] == bench.bench_config(ai.TINY, 1)  # the same config as our arm's
+
+
+def test_default_workload_is_the_largest_single_gpu_forward():
+    """With no flags the bench measures the packed causal workload (the largest
+    forward configuration, N up to 16384)."""
+    import argparse
+    import inspect
+    src = inspect.getsource(bench.main)
+    assert "default=ai.VARLEN.name" in src
+    assert bench.workload_flops(ai.VARLEN) == max(bench.workload_flops(w) for w in ai.ALL.values()
+                                                  if not w.e4m3)
 
 
 def test_input_recipe_varlen_lengths():

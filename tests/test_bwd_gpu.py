@@ -11,7 +11,7 @@ import torch
 
 import attn_inputs as ai
 import oracle
-from attn_check import to_np
+from attn_check import log_parity, to_np
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -31,6 +31,7 @@ def _check(grads, refs, label):
         assert np.all(np.isfinite(a)), f"{label} {name}: non-finite"
         err = float(np.linalg.norm(a - b))
         bound = REL_L2 * float(np.linalg.norm(b)) + 1e-5 * math.sqrt(b.size)
+        log_parity(f"{label} {name}", rel_l2=err / max(float(np.linalg.norm(b)), 1e-30))
         assert err <= bound, f"{label} {name}: |g-r| {err:.3e} > {bound:.3e} (|r| {np.linalg.norm(b):.3e})"
 
 
@@ -89,25 +90,31 @@ def test_bwd_bitwise_repeatable():
         assert torch.equal(x, y) and torch.equal(x, z)
 
 
-def test_bwd_full_workload_sampled():
-    """The causal B2-H16-N8192-d128 backward, checked at sampled query rows (dQ)
-    and key rows (dK, dV) of two heads against the per-position oracle."""
+def test_bwd_full_workload():
+    """The causal B2-H16-N8192-d128 backward at full size, as the benchmark runs it:
+    run once normally and twice in deterministic mode, all three bitwise equal; dQ,
+    dK and dV of four whole heads (both sequences, every row) against the oracle's
+    textbook backward; every gradient finite."""
     ea = _ea()
     w = ai.BWD_CAUSAL
     q, k, v, do = ai.make_qkv(w, with_dout=True)
     qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
     o, lse = ea.fwd(qd, kd, vd, causal=True)
-    dq, dk, dv = (g.cpu() for g in ea.bwd(qd, kd, vd, o, lse, dod, causal=True))
+    normal = ea.bwd(qd, kd, vd, o, lse, dod, causal=True, deterministic=False)
+    det1 = ea.bwd(qd, kd, vd, o, lse, dod, causal=True, deterministic=True)
+    det2 = ea.bwd(qd, kd, vd, o, lse, dod, causal=True, deterministic=True)
     ea.get_device_status()
-    shp = (w.B * w.N, w.H, w.d)
+    for name, a, b, c in zip(("dq", "dk", "dv"), normal, det1, det2):
+        assert torch.equal(b, c), f"{name}: deterministic runs differ"
+        assert torch.equal(a, b), f"{name}: normal and deterministic runs differ"
+        assert torch.isfinite(a.float()).all(), f"{name}: non-finite"
+    dq, dk, dv = (g.cpu() for g in normal)
     cu = oracle.dense_cu(w.B, w.N)
-    rng = np.random.default_rng(5)
-    rows = sorted({0, 1, 127, 128, 255, 4095, 4096, w.N - 2, w.N - 1} |
-                  set(rng.integers(0, w.N, 23).tolist()))
-    for b, h in ((0, 3), (1, 14)):
-        rq, rk, rv = oracle.bwd_sampled(q.reshape(shp), k.reshape(shp), v.reshape(shp),
-                                        do.reshape(shp), cu, True, 1 / math.sqrt(w.d), b, h, rows, rows)
-        _check([dq[b, rows, h], dk[b, rows, h], dv[b, rows, h]], [rq, rk, rv], f"full b{b} h{h}")
+    for h in (0, 5, 10, 15):
+        one = [t[:, :, h:h + 1].reshape(w.B * w.N, 1, w.d) for t in (q, k, v, do)]
+        refs = oracle.bwd(*one, cu, True, 1 / math.sqrt(w.d))
+        got = [g[:, :, h:h + 1].reshape(w.B * w.N, 1, w.d) for g in (dq, dk, dv)]
+        _check(got, refs, f"full-size head {h}")
 
 
 def test_bwd_peaked_rows():
@@ -179,3 +186,29 @@ def test_bwd_parity_window_varlen():
     ea.get_device_status()
     refs = oracle.bwd(q, k, v, do, cu, True, 1 / math.sqrt(d), window=window)
     _check([g.cpu() for g in grads], refs, "varlen window")
+
+
+def test_bwd_varlen_checks_cu_seqlens_on_device():
+    """The backward takes the packed token count from the caller (no read-back of
+    cu_seqlens[B]) and checks cu_seqlens on the device: a last entry that is not
+    the token count records ATTN_ERR_INVALID_ARG; a sequence that runs past the
+    packed tensors is not processed (its gradients stay unwritten) and records the
+    same; the next correct call succeeds."""
+    ea = _ea()
+    lengths = [100, 100]
+    H, d = 1, 64
+    q, k, v, do = ai.make_custom(0, 0, H, d, seed=25, lengths=lengths, n=4)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    good = torch.tensor([0, 100, 200], dtype=torch.int32, device=DEV)
+    o, lse = ea.fwd(qd, kd, vd, cu_seqlens=good, max_seqlen=100)
+    ea.get_device_status()
+    for bad in ([0, 100, 150], [0, 100, 260]):
+        ea.bwd(qd, kd, vd, o, lse, dod, cu_seqlens=torch.tensor(bad, dtype=torch.int32, device=DEV),
+               max_seqlen=100)
+        with pytest.raises(ea.AttnError) as e:
+            ea.get_device_status()
+        assert e.value.status == ea.ATTN_ERR_INVALID_ARG, bad
+    grads = ea.bwd(qd, kd, vd, o, lse, dod, cu_seqlens=good, max_seqlen=100)
+    ea.get_device_status()
+    refs = oracle.bwd(q, k, v, do, np.array([0, 100, 200]), False, 1 / math.sqrt(d))
+    _check([g.cpu() for g in grads], refs, "varlen after rejected calls")
