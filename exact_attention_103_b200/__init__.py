@@ -26,7 +26,7 @@ ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_WORKSPACE = 3, 4, 5
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_ex", "attn_bwd", "attn_bwd_workspace_size",
                     "attn_get_device_status", "attn_status_string", "attn_last_error",
                     "attn_selftest_umma", "attn_fwd_noalloc", "attn_fwd_e4m3",
-                    "attn_selftest_umma_e4m3", "attn_bwd_ex")
+                    "attn_selftest_umma_e4m3", "attn_bwd_ex", "attn_selftest_exp2")
 
 
 class AttnError(RuntimeError):
@@ -94,6 +94,8 @@ def load_library(path: str = LIB_PATH):
     lib.attn_fwd_e4m3.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, cf, cf, cf, vp,
                                   ctypes.POINTER(FwdOpts), vp]
     lib.attn_fwd_e4m3.restype = ci
+    lib.attn_selftest_exp2.argtypes = [vp, vp, vp, vp, ci, vp]
+    lib.attn_selftest_exp2.restype = ci
     lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp,
                                      ctypes.c_int64, ci, vp]
     lib.attn_fwd_noalloc.restype = ci
@@ -412,6 +414,16 @@ def selftest_umma_e4m3(a: torch.Tensor, b: torch.Tensor, v: torch.Tensor):
                                                   s_out.data_ptr(), o_out.data_ptr(),
                                                   _stream_ptr(None)))
     return s_out, o_out
+
+
+def selftest_exp2(x: torch.Tensor):
+    """The forward kernel's FMA-pipe exponential on a CUDA fp32 tensor x: returns
+    (packed form, scalar form, exp2f), each like x."""
+    _need(x, "x", torch.float32)
+    outs = [torch.empty_like(x) for _ in range(3)]
+    _check(load_library().attn_selftest_exp2(x.data_ptr(), outs[0].data_ptr(), outs[1].data_ptr(),
+                                             outs[2].data_ptr(), x.numel(), _stream_ptr(None)))
+    return tuple(outs)
 
 
 def selftest_umma(a: torch.Tensor, b: torch.Tensor, v: torch.Tensor):

@@ -18,7 +18,7 @@ OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libattn.so")
 SOURCES = ["attn_api.cu", "attn_fwd_sm100.cu", "attn_bwd_sm100.cu", "selftest_sm100.cu",
            "attn_noalloc.cu"]
-HEADERS = ["attn_fwd_sm100.h", "attn_bwd_sm100.h", "attn_internal.h", "sm100_ptx.cuh", "exp2_poly.h"]
+HEADERS = ["attn_fwd_sm100.h", "attn_bwd_sm100.h", "attn_internal.h", "sm100_ptx.cuh", "softmax_math.cuh", "exp2_poly.h"]
 PUBLIC_HEADERS = [os.path.join(ROOT, "include", h) for h in ("attn.h", "attn_selftest.h")]
 NVCC = os.environ.get("NVCC", "nvcc")
 # Extra nvcc flags (e.g. -DATTN_P_SPLIT=4 to change how P~ is handed to the PV product).

@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/attn.h"
@@ -38,10 +39,18 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 
 constexpr int kMaxDevices = 64;
 
+// Claim counters of the forward kernel's dynamic scheduler: a launch takes the
+// next of these slots in turn (two words each, zero between launches: the
+// launch's last CTA returns them to zero), so up to kWorkSlots forward launches
+// may be in flight on one device at once.
+constexpr int kWorkSlots = 64;
+
 struct DeviceState {
   bool ready = false;
   int sms = 0;
-  int* err = nullptr;  // device error word
+  int* err = nullptr;        // device error word
+  unsigned* work = nullptr;  // kWorkSlots claim-counter slots (same allocation)
+  std::atomic<unsigned> next_slot{0};
 };
 
 std::mutex g_mu;
@@ -71,10 +80,15 @@ attn_status_t device_state(DeviceState** out) {
         return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
       g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     }
-    e = cudaMalloc(&st.err, sizeof(int));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(error word)");
-    e = cudaMemset(st.err, 0, sizeof(int));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(error word)");
+    // One allocation: the error word, then (256 bytes in) the claim counters.
+    const size_t bytes = 256 + kWorkSlots * 2 * sizeof(unsigned);
+    void* mem = nullptr;
+    e = cudaMalloc(&mem, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(error word and claim counters)");
+    e = cudaMemset(mem, 0, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(error word and claim counters)");
+    st.err = static_cast<int*>(mem);
+    st.work = reinterpret_cast<unsigned*>(static_cast<char*>(mem) + 256);
     st.sms = prop.multiProcessorCount;
     st.ready = true;
   }
@@ -206,8 +220,8 @@ attn_status_t plan_fwd(const FwdCall& c, FwdPlan* pl) {
     pl->stats = opts->stats;
     if (pl->stats && !aligned(pl->stats, 8)) return fail(ATTN_ERR_INVALID_ARG, "stats misaligned");
     pl->poly = opts->exp_poly_per8;
-    if (pl->poly != 0 && pl->poly != 2 && pl->poly != 8)
-      return fail(ATTN_ERR_INVALID_ARG, "exp_poly_per8 must be 0, 2 or 8");
+    if (pl->poly != 0 && pl->poly != 2 && pl->poly != 3 && pl->poly != 4 && pl->poly != 8)
+      return fail(ATTN_ERR_INVALID_ARG, "exp_poly_per8 must be 0, 2, 3, 4 or 8");
     if (f8 && pl->poly != 0 && pl->poly != 2)
       return fail(ATTN_ERR_UNSUPPORTED, "E4M3 path: exp_poly_per8 must be 0 or 2");
     if (f8 && !(pl->tau <= 8.f))
@@ -225,7 +239,7 @@ attn_status_t plan_fwd(const FwdCall& c, FwdPlan* pl) {
 }
 
 attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total, int sms, int* err,
-                              attn::FwdLaunch* a) {
+                              unsigned* work, attn::FwdLaunch* a) {
   const attn_status_t st = load_tensor_map_encoder();
   if (st != ATTN_OK) return st;
   std::memset(a, 0, sizeof(*a));
@@ -251,6 +265,7 @@ attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total
   a->p.p_shift = f8 ? std::floor(8.f - pl.tau) : 0.f;
   a->p.tau = pl.tau;
   a->p.err = err;
+  a->p.work = work;
   a->p.stats = pl.stats;
   a->p.timeout_ns = pl.timeout;
   a->p.test_fault = pl.test_fault;
@@ -301,7 +316,8 @@ attn_status_t fwd_impl(const attn_internal::FwdCall& c, int64_t total_hint, attn
     if (total == 0) return ATTN_OK;
   }
   attn::FwdLaunch a;
-  st = attn_internal::fill_fwd_launch(c, pl, total, dev->sms, dev->err, &a);
+  unsigned* work = dev->work + 2 * (dev->next_slot.fetch_add(1u) % kWorkSlots);
+  st = attn_internal::fill_fwd_launch(c, pl, total, dev->sms, dev->err, work, &a);
   if (st != ATTN_OK) return st;
   return attn_internal::launch_planned_fwd(c, pl, a, stream);
 }

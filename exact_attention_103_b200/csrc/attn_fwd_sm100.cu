@@ -35,10 +35,14 @@
 // edges; packed variable-length batches mask keys past the sequence end.
 //
 // Scheduling ("FlashAttention V4 deep-dive", section 3.4 dynamic tile scheduling;
-// FlashAttention-4 summary (reportify.cn) item [14], the new tile scheduler):
-// items are ordered longest-first (causal: by tile-pair index t, descending) and
-// dealt to CTAs in a snake order (wave k goes left-to-right when k is even,
-// right-to-left when odd), which balances causal and varlen work without atomics.
+// FlashAttention-4 summary (reportify.cn) item [14], the new tile scheduler): a
+// dynamic scheduler.  Items form one list; each CTA's producer warp claims the
+// next list position from a device counter when it is ready for a new item and
+// hands it to the CTA's other roles through a two-entry shared-memory queue, so
+// CTAs that finish early take more work.  The list keeps the items of one
+// (sequence, head) together (its K/V tiles stay in L2 while the CTAs that claimed
+// its items stream them), longest sequences first, and puts its last groups in
+// longest-item-first order so the final claims are the short items.
 //
 // TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D, 256+2D).
 // Every wait is bounded (see sm100_ptx.cuh); on expiry the CTA stops, drains
@@ -47,8 +51,8 @@
 #include <cuda_runtime.h>
 
 #include "attn_fwd_sm100.h"
-#include "exp2_poly.h"
 #include "sm100_ptx.cuh"
+#include "softmax_math.cuh"
 
 namespace attn {
 
@@ -67,29 +71,12 @@ constexpr float kLn2 = 0.693147180559945309f;
 constexpr int kPSplit = ATTN_P_SPLIT;
 static_assert(kPSplit == 1 || kPSplit == 2 || kPSplit == 4, "P~ split");
 
-// 2^y without MUFU: j = round(y) by the 1.5*2^23 trick, f = y - j in [-1/2, 1/2],
-// p(f) ~ 2^f (minimax, exp2_poly.h), then 2^j is added to the exponent field as an
-// integer.  y is clamped below at -125 so the result stays a normal float (the
-// exact value there is < 2^-125, far below a bf16 P~).  Valid for y <= 64 (the
-// conditional-rescale threshold keeps y <= tau <= 64).  Scalar FMA-pipe
-// instructions only: one max, three adds, three FMAs and an integer shift-add.
-__device__ __forceinline__ float exp2_poly(float y) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  y = fmaxf(y, -125.f);
-  const float t = y + kMagic;            // rounds y to an integer in t's low bits
-  const float f = y - (t - kMagic);
-  float p = fmaf(f, ATTN_EXP2_C3, ATTN_EXP2_C2);
-  p = fmaf(p, f, ATTN_EXP2_C1);
-  p = fmaf(p, f, ATTN_EXP2_C0);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
 // Error codes recorded in the device error word: 4 (= ATTN_ERR_TIMEOUT) in the
 // low byte, the waiting site above it.
 __host__ __device__ constexpr int timeout_code(int site) { return 4 | (site << 8); }
 enum WaitSite {
   kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteOFull,
-  kSiteDrain, kSiteBadLen
+  kSiteDrain, kSiteBadLen, kSiteItemFull, kSiteItemEmpty
 };
 
 template <int D, bool F8>
@@ -106,8 +93,8 @@ struct Layout {
   // barrier indices
   // B_PFULL + kPSplit*s + h: part h of P~ of sub-tile s is in TMEM
   static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4,
-                       B_OFULL = 4 + 2 * kPSplit, B_DRAIN = B_OFULL + 2, B_KVFULL = B_DRAIN + 1,
-                       B_KVEMPTY = B_KVFULL + NSTAGE;
+                       B_OFULL = 4 + 2 * kPSplit, B_DRAIN = B_OFULL + 2, B_ITEMF = B_DRAIN + 1,
+                       B_ITEME = B_ITEMF + 2, B_KVFULL = B_ITEME + 2, B_KVEMPTY = B_KVFULL + NSTAGE;
   static constexpr int NBARS = B_KVEMPTY + NSTAGE;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int TABLE_OFF = MISC_OFF + 64;
@@ -121,21 +108,45 @@ struct Item {
   bool two;
 };
 
-// Work-item decoding shared by every role (all roles walk the same list).
-struct Sched {
-  const int* cu;  // device cu_seqlens or null (dense)
-  int B, H, N, T;
-  const int* order;  // varlen: sequences sorted by tile-pair count, descending
-  const int* start;  // varlen: first pair index of bucket t (buckets by t descending)
-  int pairs;         // 256-row items before any split
-  int split;         // dense non-causal: the last `split` pairs become 2*split half items
-  int count;         // number of items
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-  __device__ __forceinline__ int item(int k) const {
-    const int G = gridDim.x, c = blockIdx.x;
-    const int idx = k * G + ((k & 1) ? (G - 1 - c) : c);
-    return idx < count ? idx : -1;
+// The work list, decoded identically by every role.  Groups are (sequence, head)
+// pairs, sequences in list order (dense: b = 0..B-1; varlen: by tile-pair count,
+// descending, stable), heads inside; group g has T_g items (256-row tile pairs).
+//   bulk: groups [0, gtail), each group's items consecutive, t = T_g - 1 down to 0;
+//   tail: groups [gtail, groups), t-major: for t from the largest T_g down to 0,
+//         every tail group with T_g > t (the tail groups are sorted by T_g, so they
+//         are a prefix of the tail).
+// The tail holds the last groups covering at least two items per CTA, so the
+// claims that end the launch are the shortest items.  Dense non-causal launches
+// whose last wave would leave CTAs idle split their last `split` items into two
+// 128-row half items each.
+struct Sched {
+  const int* cu;      // device cu_seqlens or null (dense)
+  int B, H, T;        // T: tile pairs of the longest sequence
+  int N;
+  const int* order;   // varlen: sorted position -> sequence
+  const int* gstart;  // varlen: first item of sorted sequence i (items of earlier sequences)
+  const int* tstart;  // varlen tail: first tail item of level t (levels t' > t first)
+  int pairs;          // 256-row items before any split
+  int split;          // dense non-causal: the last `split` items become 2*split half items
+  int count;          // number of list positions
+  int nbulk;          // items in the bulk
+  int gtail;          // first tail group
+
+  __device__ __forceinline__ int seq_T(int i, int& b, int& start, int& L) const {
+    if (cu == nullptr) {
+      b = i;
+      start = i * N;
+      L = N;
+      return T;
+    }
+    b = order[i];
+    start = __ldg(cu + b);
+    L = __ldg(cu + b + 1) - start;
+    return ceil_div(L, 2 * kBM);
   }
+
   // SPLIT: the launch may hold half items (dense non-causal only).
   template <bool SPLIT>
   __device__ __forceinline__ Item decode(int idx) const {
@@ -146,33 +157,50 @@ struct Sched {
       idx = pairs - split + (u >> 1);
       sub = u & 1;
     }
-    const int pr = idx / H;
-    it.h = idx - pr * H;
-    int t;
-    if (cu == nullptr) {
-      const int tt = pr / B;
-      t = T - 1 - tt;
-      it.b = pr - tt * B;
-      it.seq_start = it.b * N;
-      it.L = N;
-    } else {
-      int lo = 0, hi = T - 1;  // smallest t with start[t] <= pr
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (start[mid] <= pr) hi = mid; else lo = mid + 1;
+    int g, t;  // group and tile pair
+    if (idx < nbulk) {
+      if (cu == nullptr) {
+        g = idx / T;
+        t = T - 1 - (idx - g * T);
+      } else {
+        int lo = 0, hi = B - 1;  // last sorted sequence with gstart <= idx
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (gstart[mid] <= idx) lo = mid; else hi = mid - 1;
+        }
+        int b, st, L;
+        const int Ti = seq_T(lo, b, st, L);
+        const int r = idx - gstart[lo];
+        const int hh = r / Ti;
+        g = lo * H + hh;
+        t = Ti - 1 - (r - hh * Ti);
       }
-      t = lo;
-      it.b = order[pr - start[lo]];
-      it.seq_start = __ldg(cu + it.b);
-      it.L = __ldg(cu + it.b + 1) - it.seq_start;
+    } else {
+      const int u = idx - nbulk;
+      if (cu == nullptr) {
+        const int k = B * H - gtail;  // tail groups, all with T items
+        const int lev = u / k;
+        t = T - 1 - lev;
+        g = gtail + (u - lev * k);
+      } else {
+        int lo = 0, hi = T - 1;  // smallest t with tstart[t] <= u
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (tstart[mid] <= u) hi = mid; else lo = mid + 1;
+        }
+        t = lo;
+        g = gtail + (u - tstart[lo]);
+      }
     }
+    const int i = g / H;
+    it.h = g - i * H;
+    seq_T(i, it.b, it.seq_start, it.L);
     it.row_base = t * 2 * kBM + ((SPLIT && sub > 0) ? kBM : 0);
     it.two = !SPLIT || sub < 0;
     return it;
   }
 };
 
-__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // The mask hook, one compile-time functor per MaskKind.  For the 128 query rows
 // [row0, row0 + 128) of a sequence of length L:
@@ -248,14 +276,22 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   return v;
 }
 
-// Builds the varlen tables (one warp).  tab layout: order[B] | off[T+1] | cnt[T] | start[T].
-// Returns the number of (sequence, tile-pair) pairs, or -1 if cu[0] != 0,
-// cu[B] != total, or some length is negative or exceeds T*256.
-__device__ int build_varlen_tables(const int* cu, int B, int T, int total, int* tab, int lane) {
+// Varlen table layout in shared memory (ints):
+//   order[B] | gstart[B+1] | off[T+1] | cnt[T+1] | tstart[T]
+__host__ __device__ constexpr int varlen_table_ints(int B, int T) { return 2 * B + 3 * T + 3; }
+
+// Builds the varlen list tables (one warp): sequences sorted by tile-pair count
+// (descending, stable counting sort), the items before each sorted sequence, and
+// the tail of the list (the last groups holding at least `tail_items` items, see
+// Sched).  Writes gtail and nbulk; returns the number of items, or -1 if cu[0] !=
+// 0, cu[B] != total, or some length is negative or exceeds T*256.
+__device__ int build_varlen_tables(const int* cu, int B, int H, int T, int total, int tail_items,
+                                   int* tab, int lane, int* gtail_out, int* nbulk_out) {
   int* order = tab;
-  int* off = tab + B;
+  int* gstart = order + B;
+  int* off = gstart + B + 1;
   int* cnt = off + T + 1;
-  int* start = cnt + T;
+  int* tstart = cnt + T + 1;
   for (int i = lane; i <= T; i += 32) off[i] = 0;
   __syncwarp();
   int bad = (lane == 0 && (__ldg(cu) != 0 || __ldg(cu + B) != total)) ? 1 : 0;
@@ -279,7 +315,7 @@ __device__ int build_varlen_tables(const int* cu, int B, int T, int total, int* 
     carry += __shfl_sync(0xffffffffu, incl, 31);
     __syncwarp();
   }
-  for (int t = lane; t < T; t += 32) cnt[t] = off[t];
+  for (int t = lane; t <= T; t += 32) cnt[t] = off[t];
   __syncwarp();
   // Stable placement of sequences by tile-pair count, descending.
   const uint32_t lt_mask = (1u << lane) - 1u;
@@ -294,17 +330,55 @@ __device__ int build_varlen_tables(const int* cu, int B, int T, int total, int* 
     if (b < B && lane == __ffs(same) - 1) off[key] += __popc(same);
     __syncwarp();
   }
-  // start[t] = sum_{t' > t} cnt[t']: exclusive suffix scan over t = T-1 down.
+  // gstart[i] = H * sum_{i' < i} nt(order[i']): exclusive prefix scan.
+  carry = 0;
+  for (int base = 0; base < B; base += 32) {
+    const int i = base + lane;
+    int v = 0;
+    if (i < B) {
+      const int b = order[i];
+      v = H * ceil_div(__ldg(cu + b + 1) - __ldg(cu + b), 2 * kBM);
+    }
+    const int incl = warp_incl_scan(v, lane);
+    if (i < B) gstart[i] = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  const int items = carry;
+  if (lane == 0) gstart[B] = items;
+  __syncwarp();
+  // The tail: the last groups (sorted sequence i0 from head h0 on, then every later
+  // sequence) that hold at least tail_items items; everything when there are fewer.
+  int i0 = 0, h0 = 0;
+  if (items > tail_items) {
+    int lo = 0, hi = B - 1;  // last sorted sequence with gstart <= items - tail_items
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (gstart[mid] <= items - tail_items) lo = mid; else hi = mid - 1;
+    }
+    i0 = lo;
+    const int Ti = (gstart[i0 + 1] - gstart[i0]) / H;  // >= 1: empty sequences sort last
+    const int rest = items - gstart[i0 + 1];
+    h0 = H - ceil_div(tail_items - rest, Ti);
+    if (h0 < 0) h0 = 0;
+  }
+  const int Ti0 = (gstart[i0 + 1] - gstart[i0]) / H;
+  // n(t) = tail groups with more than t tile pairs; tstart[t] = sum_{t' > t} n(t').
   carry = 0;
   for (int base = 0; base < T; base += 32) {
     const int t = T - 1 - (base + lane);
-    const int v = t >= 0 ? cnt[t] : 0;
+    int v = 0;
+    if (t >= 0) {
+      const int later = cnt[t] - (i0 + 1);  // sorted sequences after i0 with nt > t
+      v = H * (later > 0 ? later : 0) + (Ti0 > t ? H - h0 : 0);
+    }
     const int incl = warp_incl_scan(v, lane);
-    if (t >= 0) start[t] = carry + incl - v;
+    if (t >= 0) tstart[t] = carry + incl - v;
     carry += __shfl_sync(0xffffffffu, incl, 31);
   }
   __syncwarp();
-  return carry;  // total pairs
+  *gtail_out = i0 * H + h0;
+  *nbulk_out = gstart[i0] + h0 * Ti0;
+  return items;
 }
 
 // Bounded wait that ignores the abort flag (used to drain before exit).
@@ -336,10 +410,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
-  // misc[0] TMEM base, misc[1] abort flag, misc[2] number of 256-row items
+  // misc[0] TMEM base, misc[1] abort flag, misc[2] items in the list, misc[3] first
+  // tail group, misc[4] bulk items, misc[8 + e] list position in queue entry e
+  volatile int* queue = reinterpret_cast<volatile int*>(misc + 8);
   int* tab = reinterpret_cast<int*>(smem + Lay::TABLE_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tail_items = 2 * static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Lay::B_QFULL), 1);
@@ -348,6 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(Lay::B_SFULL + s), 1);
       for (int h = 0; h < kPSplit; ++h) mbar_init(bar(Lay::B_PFULL + kPSplit * s + h), 4);
       mbar_init(bar(Lay::B_OFULL + s), 1);
+      mbar_init(bar(Lay::B_ITEMF + s), 1);  // the producer publishes a claimed position
+      mbar_init(bar(Lay::B_ITEME + s), 9);  // the MMA warp and the 8 softmax warps read it
     }
     mbar_init(bar(Lay::B_DRAIN), 1);
     for (int i = 0; i < NS; ++i) {
@@ -362,19 +441,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (warp == 8) {
-    int count;
+    int count, gtail, nbulk;
     if (p.cu_seqlens == nullptr) {
-      count = p.B * p.T * p.H;
+      const int groups = p.B * p.H;
+      int k = ceil_div(tail_items, p.T);
+      if (k > groups) k = groups;
+      count = groups * p.T;
+      gtail = groups - k;
+      nbulk = gtail * p.T;
     } else {
-      const int pairs = build_varlen_tables(p.cu_seqlens, p.B, p.T, p.total, tab, lane);
-      if (pairs < 0) {
-        count = 0;
+      count = build_varlen_tables(p.cu_seqlens, p.B, p.H, p.T, p.total, tail_items, tab, lane, &gtail,
+                                  &nbulk);
+      if (count < 0) {
+        count = gtail = nbulk = 0;
         if (lane == 0 && p.err) atomicCAS(p.err, 0, 1 | (kSiteBadLen << 8));
-      } else {
-        count = pairs * p.H;
       }
     }
-    if (lane == 0) misc[2] = static_cast<uint32_t>(count);
+    if (lane == 0) {
+      misc[2] = static_cast<uint32_t>(count);
+      misc[3] = static_cast<uint32_t>(gtail);
+      misc[4] = static_cast<uint32_t>(nbulk);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -385,12 +472,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   sch.cu = p.cu_seqlens;
   sch.B = p.B; sch.H = p.H; sch.N = p.N; sch.T = p.T;
   sch.order = tab;
-  sch.start = tab + p.B + 2 * p.T + 1;
+  sch.gstart = tab + p.B;
+  sch.tstart = tab + 2 * p.B + 2 * p.T + 3;
   sch.pairs = static_cast<int>(misc[2]);
+  sch.gtail = static_cast<int>(misc[3]);
+  sch.nbulk = static_cast<int>(misc[4]);
   // Dense non-causal items all cost the same: when the last wave would leave
-  // CTAs idle, its pairs are split into 128-row half items so it spreads over
+  // CTAs idle, its items are split into 128-row half items so it spreads over
   // more SMs (a half item runs without a ping-pong partner, but the wave is
-  // shorter).  Causal and varlen items are already longest-first.
+  // shorter).  Causal and varlen lists end with their shortest items.
   sch.split = 0;
   if (SPLIT && p.cu_seqlens == nullptr) {
     const int rem = sch.pairs % static_cast<int>(gridDim.x);
@@ -404,6 +494,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   MaskFn<MASK> mk;
   mk.wl = p.wl;
   mk.wr = p.wr;
+  // Consumer roles (the MMA warp, the softmax warps): the k-th list position this
+  // CTA claimed, from the queue (one arrival per warp frees the entry); -1 ends
+  // the list, and so does an expired wait.
+  auto take_item = [&](int k) -> int {
+    const int e = k & 1;
+    if (!__all_sync(0xffffffffu, mbar_wait(bar(Lay::B_ITEMF + e), (k >> 1) & 1, wc,
+                                           timeout_code(kSiteItemFull))))
+      return -1;
+    const int idx = queue[e];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(Lay::B_ITEME + e));
+    return idx;
+  };
 
   if (warp < 8) {
     // ------------------------------------------------------------ softmax
@@ -418,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_phase = 0, o_phase = 0;
     unsigned long long n_rescale = 0, n_rowtiles = 0;
     for (int k = 0;; ++k) {
-      const int idx = sch.item(k);
+      const int idx = take_item(k);
       if (idx < 0) break;
       const Item it = sch.template decode<SPLIT>(idx);
       const int b = it.b, h = it.h, seq_start = it.seq_start, L = it.L;
@@ -435,28 +538,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         s_phase ^= 1u;
         tc_fence_after();
-        uint32_t sv[128];
-        tmem_ld_x128(t_s, sv);
+        // The score row in two halves: the second half's load is in flight while
+        // the first half's maximum is taken.
+        uint32_t sa[64], sz[64];
+        tmem_ld_x64(t_s, sa);
+        tmem_ld_x64_async(t_s + 64, sz);
         const int kb = j * kBN;
-        if (mk.partial(kb, row0, L)) {
-          int c_lo, c_hi;  // keys [kb + c_lo, kb + c_hi) are visible to this row
+        const bool part = mk.partial(kb, row0, L);
+        int c_lo = 0, c_hi = kBN;  // keys [kb + c_lo, kb + c_hi) are visible to this row
+        if (part) {
           mk.cols(q_row, kb, L, c_lo, c_hi);
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c < c_lo || c >= c_hi) sv[c] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < 64; ++c)
+            if (c < c_lo || c >= c_hi) sa[c] = __float_as_uint(-INFINITY);
         }
         // Row maximum: four independent 3-input max chains, then a small tree.
         float m4[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          m4[i] = fmax3(__uint_as_float(sv[i]), __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 8]));
+          m4[i] = fmax3(__uint_as_float(sa[i]), __uint_as_float(sa[i + 4]), __uint_as_float(sa[i + 8]));
 #pragma unroll
-        for (int c = 12; c < 124; c += 8)
+        for (int c = 12; c < 60; c += 8)
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            m4[i] = fmax3(m4[i], __uint_as_float(sv[c + i]), __uint_as_float(sv[c + 4 + i]));
+            m4[i] = fmax3(m4[i], __uint_as_float(sa[c + i]), __uint_as_float(sa[c + 4 + i]));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], __uint_as_float(sv[124 + i]));
+        for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], __uint_as_float(sa[60 + i]));
+        tmem_wait_ld_x64(sz);
+        if (part) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c + 64 < c_lo || c + 64 >= c_hi) sz[c] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int c = 0; c < 64; c += 8)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            m4[i] = fmax3(m4[i], __uint_as_float(sz[c + i]), __uint_as_float(sz[c + 4 + i]));
         const float m_tile = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sl;
         bool need = false;
         float alpha = 1.f;
@@ -474,8 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++n_rescale;
           }
         }
-        // P~ = 2^(s*scale*log2e - m_ref): one FMA for the argument, MUFU ex2 or the
-        // FMA-pipe polynomial for the exponential, partial row sums, packing.  In
+        // P~ = 2^(s*scale*log2e - m_ref): one packed FMA per column pair for the
+        // arguments, MUFU ex2 or (for POLY of every 8 pairs) the packed FMA-pipe
+        // polynomial for the exponentials, packed partial row sums, packing.  In
         // kPSplit parts: each is stored and released to the MMA warp (the PV K steps
         // over its keys) while the next is computed.
         float nm = (MASK == kMaskWindow && m_ref == -INFINITY) ? 0.f : -m_ref;
@@ -488,17 +607,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int cc = 0; cc < PAIRS; ++cc) {
             const int c = PAIRS * half + cc;  // column pair (keys 2c, 2c+1)
-            float a = fmaf(__uint_as_float(sv[2 * c]), sl, nm);
-            float e = fmaf(__uint_as_float(sv[2 * c + 1]), sl, nm);
+            const uint32_t x0 = c < 32 ? sa[2 * c] : sz[2 * c - 64];
+            const uint32_t x1 = c < 32 ? sa[2 * c + 1] : sz[2 * c - 63];
+            float a, e;
+            ffma2_bc(a, e, __uint_as_float(x0), __uint_as_float(x1), sl, nm);
             if ((c & 7) >= 8 - POLY) {
-              a = exp2_poly(a);
-              e = exp2_poly(e);
+              exp2_poly_x2(a, e);
             } else {
               a = fast_exp2(a);
               e = fast_exp2(e);
             }
-            ls[2 * (c & 1)] += a;
-            ls[2 * (c & 1) + 1] += e;
+            if (c & 1) fadd2_acc(ls[2], ls[3], a, e);
+            else fadd2_acc(ls[0], ls[1], a, e);
             if constexpr (F8) {
               const uint32_t h = pack_e4m3x2(a, e);  // bytes 2(c&1), +1 of word c/2
               if (cc & 1) pk[cc >> 1] |= h << 16; else pk[cc >> 1] = h;
@@ -605,7 +725,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     int n_items = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int idx = sch.item(k);
+      // Claim the next list position once its queue entry is free, and publish it.
+      const int e = k & 1;
+      if (k >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_ITEME + e), ((k >> 1) - 1) & 1, wc,
+                                               timeout_code(kSiteItemEmpty)));
+        if (!ok) break;
+      }
+      int idx = -1;
+      if (lane == 0) {
+        const unsigned c = atomicAdd(p.work, 1u);
+        if (c < static_cast<unsigned>(sch.count)) idx = static_cast<int>(c);
+        queue[e] = idx;
+        mbar_arrive(bar(Lay::B_ITEMF + e));
+      }
+      idx = __shfl_sync(0xffffffffu, idx, 0);
       if (idx < 0) break;
       const Item it = sch.template decode<SPLIT>(idx);
       const int h = it.h, seq_start = it.seq_start;
@@ -672,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t n_ld = 0, q_phase = 0, p_phase0 = 0, p_phase1 = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int idx = sch.item(k);
+      const int idx = take_item(k);
       if (idx < 0) break;
       const Item it = sch.template decode<SPLIT>(idx);
       int jlo, nkv, lo0, hi0, lo1, hi1;
@@ -755,7 +889,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (elect_one()) {
           if (jj < nkv) tc_commit(bar(Lay::B_KVEMPTY + slotK));
           if (jj > 0) tc_commit(bar(Lay::B_KVEMPTY + slotV));
-          if (jj == nkv - 1) tc_commit(bar(Lay::B_QEMPTY));
+          // The query tiles are free after the item's last S product (an item
+          // without key tiles -- an empty half item -- frees them at once).
+          if (jj == (nkv > 0 ? nkv - 1 : 0)) tc_commit(bar(Lay::B_QEMPTY));
         }
         __syncwarp();
       }
@@ -772,6 +908,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 9) tmem_dealloc(tmem, 512);
+  // The last CTA to finish returns the claim counter to zero for the next launch
+  // that uses it: every CTA's producer has made its last claim before its CTA
+  // counts itself finished here.
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.work + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.work, 0u);
+      atomicExch(p.work + 1, 0u);
+    }
+  }
 }
 
 template <int D, bool F8>
@@ -782,7 +928,7 @@ constexpr int smem_bytes_fixed() { return 1024 + Layout<D, F8>::TABLE_OFF; }
 int fwd_smem_bytes(int D, int B, int T, int varlen, int fp8) {
   const int fixed = fp8 ? smem_bytes_fixed<128, true>()
                         : (D == 128 ? smem_bytes_fixed<128, false>() : smem_bytes_fixed<64, false>());
-  return fixed + (varlen ? (B + 3 * T + 1) * 4 : 0);
+  return fixed + (varlen ? varlen_table_ints(B, T) * 4 : 0);
 }
 
 template <int D, int MASK, int POLY, bool F8 = false>
@@ -797,6 +943,8 @@ static cudaError_t launch_t(const FwdLaunch& a, cudaStream_t st) {
 template <int D, int MASK>
 static cudaError_t launch_p(const FwdLaunch& a, int poly, cudaStream_t st) {
   if (poly == 2) return launch_t<D, MASK, 2>(a, st);
+  if (poly == 3) return launch_t<D, MASK, 3>(a, st);
+  if (poly == 4) return launch_t<D, MASK, 4>(a, st);
   if (poly == 8) return launch_t<D, MASK, 8>(a, st);
   return launch_t<D, MASK, 0>(a, st);
 }

@@ -26,6 +26,8 @@ struct FwdParams {
   float scale_log2;      // scale * log2(e)
   float tau;             // conditional-rescale threshold, log2 units
   int* err;              // device error word
+  unsigned* work;        // [0] list positions claimed, [1] CTAs finished; zero at launch,
+                         // returned to zero by the launch's last CTA
   unsigned long long* stats;  // optional [rescaled rows, row-tiles]
   uint64_t timeout_ns;   // limit of every internal wait
   int test_fault;        // 1: withhold the first Q copy (failure-path tests only)

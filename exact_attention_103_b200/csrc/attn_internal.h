@@ -41,10 +41,10 @@ struct FwdPlan {
 // Checks every argument of a forward call on the host; touches no device state.
 attn_status_t plan_fwd(const FwdCall& c, FwdPlan* pl);
 // Builds the launch of a planned forward call over `total` packed tokens (dense:
-// B*N) on a device with `sms` SMs, the kernel recording errors in `err` (a device
-// address).
+// B*N) on a device with `sms` SMs, the kernel recording errors in `err` and
+// claiming work items through the two zeroed words at `work` (device addresses).
 attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total, int sms, int* err,
-                              attn::FwdLaunch* a);
+                              unsigned* work, attn::FwdLaunch* a);
 attn_status_t launch_planned_fwd(const FwdCall& c, const FwdPlan& pl, const attn::FwdLaunch& a,
                                  attn_stream_t stream);
 // Looks up the driver's tensor-map encoder once per process.

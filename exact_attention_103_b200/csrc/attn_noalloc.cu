@@ -22,11 +22,12 @@
 
 namespace {
 
-// Scratch of the allocation-free forward: the kernel's status word lives at word 0.
-// Every GPU that loads the library holds these bytes until the process exits.
+// Scratch of the allocation-free forward: the kernel's status word at word 0 and
+// its scheduler's two claim counters at words 2 and 3.  Every GPU that loads the
+// library holds these bytes until the process exits.
 constexpr size_t kScratchBytes = 256;
 static __device__ __align__(256) int g_noalloc_scratch[kScratchBytes / sizeof(int)];
-constexpr size_t kFwdScratchNeeded = sizeof(int);  // the status word
+constexpr size_t kFwdScratchNeeded = 4 * sizeof(int);  // status word, pad, claim counters
 
 constexpr int kMaxDevices = 64;
 struct NoAllocDevice {
@@ -94,11 +95,13 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
   st = setup_device(&dev);
   if (st != ATTN_OK) return st;
   attn::FwdLaunch a;
-  st = attn_internal::fill_fwd_launch(c, pl, total, dev->sms, dev->scratch, &a);
+  st = attn_internal::fill_fwd_launch(c, pl, total, dev->sms, dev->scratch,
+                                      reinterpret_cast<unsigned*>(dev->scratch + 2), &a);
   if (st != ATTN_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
-  // The status word must start at zero; it keeps the previous call's value otherwise.
+  // The status word and the claim counters must start at zero; the array keeps the
+  // previous call's values otherwise.
   cudaError_t e = cudaMemsetAsync(dev->scratch, 0, kFwdScratchNeeded, cs);
   if (e != cudaSuccess) return report(ATTN_ERR_CUDA, "attn_fwd_noalloc: clearing the status word failed");
   st = attn_internal::launch_planned_fwd(c, pl, a, stream);

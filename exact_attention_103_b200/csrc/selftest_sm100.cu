@@ -6,9 +6,30 @@
 
 #include "../../include/attn_selftest.h"
 #include "sm100_ptx.cuh"
+#include "softmax_math.cuh"
 
 namespace attn {
 namespace {
+
+// The forward kernel's FMA-pipe exponential over an input array: y_poly from the
+// packed two-lane form (the one the kernel runs), y_scalar from the scalar form,
+// y_ref from CUDA's exp2f.
+__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* y_poly, float* y_scalar,
+                                     float* y_ref, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  float a = x[i], e = (i + 1 < n) ? x[i + 1] : 0.f;
+  float pa = a, pe = e;
+  exp2_poly_x2(pa, pe);
+  y_poly[i] = pa;
+  y_scalar[i] = exp2_poly(a);
+  y_ref[i] = exp2f(a);
+  if (i + 1 < n) {
+    y_poly[i + 1] = pe;
+    y_scalar[i + 1] = exp2_poly(e);
+    y_ref[i + 1] = exp2f(e);
+  }
+}
 
 // F8: E4M3 inputs (kind::f8f6f4, K = 32 per instruction) and P = e4m3(S).
 template <int D, bool F8>
@@ -171,4 +192,16 @@ extern "C" attn_status_t attn_selftest_umma_e4m3(const void* a, const void* b, c
   if (e == cudaSuccess) attn::selftest_kernel<128, true><<<1, 128, smem, cs>>>(ta, tb, tv, s_out, o_out, err);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+extern "C" attn_status_t attn_selftest_exp2(const float* x, float* y_poly, float* y_scalar,
+                                            float* y_ref, int n, attn_stream_t stream) {
+  if (n < 0) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  if (!x || !y_poly || !y_scalar || !y_ref) return ATTN_ERR_INVALID_ARG;
+  const int threads = 256;
+  const int pairs = (n + 1) / 2;
+  attn::exp2_selftest_kernel<<<(pairs + threads - 1) / threads, threads, 0,
+                               reinterpret_cast<cudaStream_t>(stream)>>>(x, y_poly, y_scalar, y_ref, n);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -67,6 +67,8 @@ SMALL = [
     (1, 1000, 1, 64, False, 1.0),
     (2, 640, 2, 128, False, 4.0),    # Q x4: the running maximum moves often
     (1, 768, 2, 128, True, 4.0),
+    (1, 100, 300, 64, False, 1.0),   # 300 one-sub-tile pairs: the split last wave holds empty
+    (2, 100, 150, 128, False, 1.0),  # halves, and a CTA may claim more work after one
 ]
 
 
@@ -307,7 +309,10 @@ def test_varlen_max_sequences(causal):
                     cu_seqlens=torch.from_numpy(cu).to(DEV), max_seqlen=max(lengths))
     ea.get_device_status()
     o_ref, lse_ref, _ = oracle.fwd(q, k, v, cu, causal, scale)
-    compare_o(o.cpu(), o_ref, f"1024 sequences causal={causal}")
+    # Sequences of 0..9 tokens: every output row averages at most 9 values, so |O|
+    # reaches 2 and beyond, where half a bf16 ulp of the output alone is 7.8e-3;
+    # the half-ulp gate applies (the raw bar is asserted on the benchmark workloads).
+    compare_o(o.cpu(), o_ref, f"1024 sequences causal={causal}", raw_bar=False)
     compare_lse(lse.cpu(), lse_ref)
 
 
