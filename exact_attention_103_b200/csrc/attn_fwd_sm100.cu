@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_o = tmem + lane_bits + (s ? Lay::TM_O1 : Lay::TM_O0);
     const float sl = p.scale_log2;
     uint32_t s_phase = 0, o_phase = 0;
-    unsigned long long n_rescale = 0, n_rowtiles = 0;
+    uint32_t n_rescale = 0, n_rowtiles = 0;  // this thread's row: < 2^32 tiles per launch
     for (int k = 0;; ++k) {
       const int idx = take_item(k);
       if (idx < 0) break;
@@ -680,19 +680,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool store = q_row < L;
       __nv_bfloat16* dst =
           p.o + (static_cast<int64_t>(seq_start + q_row) * p.H + h) * static_cast<int64_t>(D);
+      // The whole O row in one TMEM load (the score registers are free by now).
+      uint32_t ov[D];
+      if constexpr (D == 128) tmem_ld_x128(t_o, ov);
+      else tmem_ld_x64(t_o, ov);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld_x32(t_o + 32 * c, ov);
-        uint32_t w[16];
+      for (int c = 0; c < D / 8; ++c) {
+        uint32_t w[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
-        if (store) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int i = 0; i < 4; ++i) {
+          float x0, x1;
+          fmul2_bc(x0, x1, __uint_as_float(ov[8 * c + 2 * i]), __uint_as_float(ov[8 * c + 2 * i + 1]), inv);
+          w[i] = pack_bf16x2(x0, x1);
         }
+        if (store) reinterpret_cast<uint4*>(dst)[c] = make_uint4(w[0], w[1], w[2], w[3]);
       }
       if (store) {
         float lse2 = m_ref + __log2f(l);
@@ -707,8 +708,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (p.stats) {
-      atomicAdd(p.stats, n_rescale);
-      atomicAdd(p.stats + 1, n_rowtiles);
+      atomicAdd(p.stats, static_cast<unsigned long long>(n_rescale));
+      atomicAdd(p.stats + 1, static_cast<unsigned long long>(n_rowtiles));
     }
   } else if (warp == 8) {
     // ----------------------------------------------------------- producer
