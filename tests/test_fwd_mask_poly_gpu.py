@@ -63,7 +63,7 @@ def test_window_parity_dense(B, N, H, d, causal, window, qm):
         q = (q.float() * qm).to(torch.bfloat16)
     scale = 1.0 / math.sqrt(d)
     o, lse, o_ref, l_ref = _dense(q, k, v, causal, scale, window)
-    compare_o(o, o_ref, f"window {window} B{B} N{N} d{d} causal={causal}", raw_bar=qm == 1.0)
+    compare_o(o, o_ref, f"window {window} B{B} N{N} d{d} causal={causal}")
     compare_lse(lse, l_ref)
 
 
@@ -124,8 +124,7 @@ def test_exp_poly_parity(poly, B, N, H, d, causal, qm, window):
         q = (q.float() * qm).to(torch.bfloat16)
     scale = 1.0 / math.sqrt(d)
     o, lse, o_ref, l_ref = _dense(q, k, v, causal, scale, window, poly)
-    compare_o(o, o_ref, f"poly {poly}/8 B{B} N{N} d{d} causal={causal} window={window}",
-              raw_bar=qm == 1.0)
+    compare_o(o, o_ref, f"poly {poly}/8 B{B} N{N} d{d} causal={causal} window={window}")
     compare_lse(lse, l_ref)
 
 
