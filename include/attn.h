@@ -33,9 +33,12 @@
  *    device error word.
  *  - Supported: d in {64, 128}; scale finite and > 0.  Varlen: B <= 1024 and
  *    N <= 131072.  B == 0 or N == 0 is a no-op.
- *  - The library allocates, lazily and once per device, a small device error word.
+ *  - The library allocates, lazily and once per device, one small device buffer:
+ *    an error word and 64 slots of work counters for the forward kernel's
+ *    scheduler (a forward launch takes the next slot in turn and leaves it at zero
+ *    when it ends, so up to 64 forward launches may run concurrently on a device).
  *    A kernel whose internal waits exceed their time limit stops, records
- *    ATTN_ERR_TIMEOUT there, and leaves its outputs undefined;
+ *    ATTN_ERR_TIMEOUT in the error word, and leaves its outputs undefined;
  *    attn_get_device_status() reports and clears it.
  */
 #ifndef LIBATTN_ATTN_H
@@ -230,10 +233,13 @@ ATTN_API size_t attn_bwd_workspace_size(int B, int H, int N, int d, int total_to
  *    the status must pass check != 0.
  *  - The first call on a device does its set-up there (looks up the array's
  *    device address); make that first call before any stream capture.
- *  - Every call shares the array: each call clears the status word on `stream`
- *    before its launch, and calls whose kernels overlap on the GPU race on it.
- *  - A kernel that needed more scratch than the array holds would be rejected with
- *    ATTN_ERR_WORKSPACE; the forward kernel needs 4 bytes.
+ *  - Every call shares the array: calls whose kernels overlap on the GPU race on
+ *    it (their status words and their work counters mix), so such calls must be
+ *    ordered, e.g. issued on one stream.
+ *  - The forward kernel uses 16 bytes of the array: the status word and the two
+ *    counters through which its CTAs claim work items (each call clears all 16
+ *    bytes on `stream` before its launch).  A kernel that needed more scratch than
+ *    the array holds would be rejected with ATTN_ERR_WORKSPACE.
  */
 ATTN_API attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
                                         float* lse, int B, int H, int N, int d, int causal,
