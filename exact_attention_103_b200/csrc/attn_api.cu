@@ -7,7 +7,6 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
-#include <atomic>
 #include <mutex>
 
 #include "../../include/attn.h"
@@ -39,10 +38,12 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 
 constexpr int kMaxDevices = 64;
 
-// Claim counters of the forward kernel's dynamic scheduler: a launch takes the
-// next of these slots in turn (two words each, zero between launches: the
-// launch's last CTA returns them to zero), so up to kWorkSlots forward launches
-// may be in flight on one device at once.
+// Claim counters of the forward kernel's dynamic scheduler, two words per slot,
+// zero between launches (a launch's last CTA returns its slot to zero).  Two
+// launches that run at the same time must not share a slot; launches on one
+// stream never do, so each stream keeps its own slot: streams get slots in order
+// of first use, and beyond kWorkSlots streams the least recently used slot passes
+// to the new stream.
 constexpr int kWorkSlots = 64;
 
 struct DeviceState {
@@ -50,7 +51,9 @@ struct DeviceState {
   int sms = 0;
   int* err = nullptr;        // device error word
   unsigned* work = nullptr;  // kWorkSlots claim-counter slots (same allocation)
-  std::atomic<unsigned> next_slot{0};
+  cudaStream_t slot_stream[kWorkSlots] = {};
+  uint64_t slot_use[kWorkSlots] = {};  // 0 = free, else the tick of the last use
+  uint64_t tick = 0;
 };
 
 std::mutex g_mu;
@@ -94,6 +97,22 @@ attn_status_t device_state(DeviceState** out) {
   }
   *out = &st;
   return ATTN_OK;
+}
+
+// The claim-counter slot of `stream` on this device (see kWorkSlots).
+unsigned* work_slot(DeviceState* dev, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int pick = 0;
+  for (int i = 0; i < kWorkSlots; ++i) {
+    if (dev->slot_use[i] != 0 && dev->slot_stream[i] == stream) {
+      pick = i;
+      break;
+    }
+    if (dev->slot_use[i] < dev->slot_use[pick]) pick = i;  // a free slot, else the oldest
+  }
+  dev->slot_stream[pick] = stream;
+  dev->slot_use[pick] = ++dev->tick;
+  return dev->work + 2 * pick;
 }
 
 // A 3-D view {d, H, total} of a token-major [total, H, d] tensor of esz-byte
@@ -316,7 +335,7 @@ attn_status_t fwd_impl(const attn_internal::FwdCall& c, int64_t total_hint, attn
     if (total == 0) return ATTN_OK;
   }
   attn::FwdLaunch a;
-  unsigned* work = dev->work + 2 * (dev->next_slot.fetch_add(1u) % kWorkSlots);
+  unsigned* work = work_slot(dev, cs);
   st = attn_internal::fill_fwd_launch(c, pl, total, dev->sms, dev->err, work, &a);
   if (st != ATTN_OK) return st;
   return attn_internal::launch_planned_fwd(c, pl, a, stream);

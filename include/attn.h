@@ -35,8 +35,13 @@
  *    N <= 131072.  B == 0 or N == 0 is a no-op.
  *  - The library allocates, lazily and once per device, one small device buffer:
  *    an error word and 64 slots of work counters for the forward kernel's
- *    scheduler (a forward launch takes the next slot in turn and leaves it at zero
- *    when it ends, so up to 64 forward launches may run concurrently on a device).
+ *    scheduler.  Each stream that runs forward passes keeps its own slot (launches
+ *    on one stream never overlap, and a launch leaves its slot at zero when it
+ *    ends); with more than 64 such streams on a device the least recently used
+ *    slot passes to the new stream, so forward launches on more than 64 streams
+ *    must not all be in flight at once.  A CUDA graph keeps the slot of the stream
+ *    it was captured on: replays of it must not overlap forward launches on that
+ *    stream or each other.
  *    A kernel whose internal waits exceed their time limit stops, records
  *    ATTN_ERR_TIMEOUT in the error word, and leaves its outputs undefined;
  *    attn_get_device_status() reports and clears it.

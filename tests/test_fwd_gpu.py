@@ -366,3 +366,28 @@ def test_host_pipeline_matches_fwd(varlen):
                         max_seqlen=max(lengths) if varlen else None)
         ea.get_device_status()
         assert torch.equal(o.cpu(), o_h) and torch.equal(lse.cpu(), l_h)
+
+
+def test_concurrent_streams_keep_their_own_work_counters():
+    """Forward launches queued on four streams at once (the kernels may overlap on
+    the GPU; each stream's launches use that stream's claim counters) give exactly
+    the results of the same calls made one at a time."""
+    ea = _lib()
+    probs = [ai.make_custom(1, 700 + 130 * i, 3, 128, seed=90 + i) for i in range(4)]
+    dev = [tuple(t.to(DEV) for t in p) for p in probs]
+    serial = []
+    for q, k, v in dev:
+        serial.append(ea.fwd(q, k, v, causal=True))
+    ea.get_device_status()
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    torch.cuda.synchronize()
+    outs = [[] for _ in range(4)]
+    for rep in range(3):
+        for i, (q, k, v) in enumerate(dev):
+            with torch.cuda.stream(streams[i]):
+                outs[i].append(ea.fwd(q, k, v, causal=True))
+    torch.cuda.synchronize()
+    ea.get_device_status()
+    for i in range(4):
+        for o, lse in outs[i]:
+            assert torch.equal(o, serial[i][0]) and torch.equal(lse, serial[i][1])
