@@ -532,7 +532,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end leg (profiling runs only)")
-    ap.add_argument("--exp-poly-per8", type=int, default=0, choices=[0, 2, 3, 4, 8],
+    ap.add_argument("--exp-poly-per8", type=int, default=0, choices=[0, 2, 8],
                     help="exponential pairs of every 8 computed by the FMA-pipe polynomial")
     args = ap.parse_args()
     if args.warmup < 3:

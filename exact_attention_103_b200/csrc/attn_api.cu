@@ -239,8 +239,8 @@ attn_status_t plan_fwd(const FwdCall& c, FwdPlan* pl) {
     pl->stats = opts->stats;
     if (pl->stats && !aligned(pl->stats, 8)) return fail(ATTN_ERR_INVALID_ARG, "stats misaligned");
     pl->poly = opts->exp_poly_per8;
-    if (pl->poly != 0 && pl->poly != 2 && pl->poly != 3 && pl->poly != 4 && pl->poly != 8)
-      return fail(ATTN_ERR_INVALID_ARG, "exp_poly_per8 must be 0, 2, 3, 4 or 8");
+    if (pl->poly != 0 && pl->poly != 2 && pl->poly != 8)
+      return fail(ATTN_ERR_INVALID_ARG, "exp_poly_per8 must be 0, 2 or 8");
     if (f8 && pl->poly != 0 && pl->poly != 2)
       return fail(ATTN_ERR_UNSUPPORTED, "E4M3 path: exp_poly_per8 must be 0 or 2");
     if (f8 && !(pl->tau <= 8.f))

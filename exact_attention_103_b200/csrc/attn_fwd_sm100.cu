@@ -944,8 +944,6 @@ static cudaError_t launch_t(const FwdLaunch& a, cudaStream_t st) {
 template <int D, int MASK>
 static cudaError_t launch_p(const FwdLaunch& a, int poly, cudaStream_t st) {
   if (poly == 2) return launch_t<D, MASK, 2>(a, st);
-  if (poly == 3) return launch_t<D, MASK, 3>(a, st);
-  if (poly == 4) return launch_t<D, MASK, 4>(a, st);
   if (poly == 8) return launch_t<D, MASK, 8>(a, st);
   return launch_t<D, MASK, 0>(a, st);
 }

@@ -116,7 +116,7 @@ ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, voi
  *  exp_poly_per8: how many of every 8 (even, odd) column pairs of a score row are
  *      exponentiated by the FMA-pipe polynomial instead of MUFU ex2
  *      ("FlashAttention V4 deep-dive", section 3.2: software exp on the FMA
- *      units).  0 (the default, all MUFU), 2, 3, 4 or 8; other values are rejected
+ *      units).  0 (the default, all MUFU), 2 or 8; other values are rejected
  *      (ATTN_ERR_INVALID_ARG).  The polynomial has a relative error below 7.5e-5,
  *      under half a bf16 ulp, so the results differ from the MUFU path only by
  *      the rounding of P~. */

@@ -86,7 +86,7 @@ def test_varlen_limits(lib):
 
 def test_bad_options(lib):
     for opts in (ea.FwdOpts(float("inf"), None, 0, 0, 0), ea.FwdOpts(65.0, None, 0, 0, 0),
-                 ea.FwdOpts(-1.0, None, 0, 0, 2), ea.FwdOpts(-1.0, None, 0, 0, 0, 0, 0, 0, 5),
+                 ea.FwdOpts(-1.0, None, 0, 0, 2), ea.FwdOpts(-1.0, None, 0, 0, 0, 0, 0, 0, 3),
                  ea.FwdOpts(-1.0, None, 0, 0, 0, 0, 0, 0, -1)):
         st = lib.attn_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0, 0.1, None,
                              ctypes.byref(opts), None)

@@ -114,7 +114,7 @@ POLY = [
 ]
 
 
-@pytest.mark.parametrize("poly", [2, 3, 4, 8])
+@pytest.mark.parametrize("poly", [2, 8])
 @pytest.mark.parametrize("B,N,H,d,causal,qm,window", POLY)
 def test_exp_poly_parity(poly, B, N, H, d, causal, qm, window):
     """2 of 8 pairs (FA4-style partial offload) and 8 of 8 (every exponential on
