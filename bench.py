@@ -343,7 +343,7 @@ def run_ours(args, rank, world, local):
     def step():
         ea.fwd(q, k, v, causal=w.causal, scale=scale, cu_seqlens=cu, max_seqlen=max_len,
                out=out, lse=lse, window=w.window, exp_poly_per8=args.exp_poly_per8,
-               e4m3_scales=f8)
+               e4m3_scales=f8, cta_pair=args.cta_pair)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -374,7 +374,7 @@ def run_ours(args, rank, world, local):
         counters = torch.zeros(2, dtype=torch.int64, device=dev)
         ea.fwd(q, k, v, causal=w.causal, scale=scale, cu_seqlens=cu, max_seqlen=max_len,
                out=out, lse=lse, exp_poly_per8=args.exp_poly_per8, e4m3_scales=f8,
-               stats=counters)
+               stats=counters, cta_pair=args.cta_pair)
         ea.get_device_status()
         rescaled, row_tiles = (int(x) for x in counters.cpu())
         rescale = {"rows_rescaled": rescaled, "row_tiles_after_first": row_tiles,
@@ -416,7 +416,7 @@ def run_ours(args, rank, world, local):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "e4m3" if w.e4m3 else "bf16", "data": "synthetic",
                 "config": bench_config(w, world),
-                "options": {"exp_poly_per8": args.exp_poly_per8},
+                "options": {"exp_poly_per8": args.exp_poly_per8, "cta_pair": args.cta_pair},
                 "rescale": rescale,
                 "pct_of_peak": 100.0 * achieved / peak,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
@@ -533,6 +533,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end leg (profiling runs only)")
+    ap.add_argument("--cta-pair", action="store_true",
+                    help="clusters of two CTAs sharing each item (tcgen05.mma.cta_group::2)")
     ap.add_argument("--exp-poly-per8", type=int, default=0, choices=[0, 2, 8],
                     help="exponential pairs of every 8 computed by the FMA-pipe polynomial")
     args = ap.parse_args()

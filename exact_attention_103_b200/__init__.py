@@ -52,7 +52,8 @@ class FwdOpts(ctypes.Structure):
                 ("has_window", ctypes.c_int),
                 ("window_left", ctypes.c_int),
                 ("window_right", ctypes.c_int),
-                ("exp_poly_per8", ctypes.c_int)]
+                ("exp_poly_per8", ctypes.c_int),
+                ("cta_pair", ctypes.c_int)]
 
 
 _lib = None
@@ -138,7 +139,8 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         stream: Optional[torch.cuda.Stream] = None,
         test_fault: int = 0, window: Optional[Tuple[int, int]] = None,
         exp_poly_per8: int = 0,
-        e4m3_scales: Optional[Tuple[float, float, float]] = None
+        e4m3_scales: Optional[Tuple[float, float, float]] = None,
+        cta_pair: bool = False
         ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Exact attention forward on the GPU.
 
@@ -151,7 +153,9 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     (0, 2 or 8) moves that many of every 8 exponential pairs to the FMA pipe.
     ``e4m3_scales = (q_scale, k_scale, v_scale)`` selects the 8-bit entry point
     ``attn_fwd_e4m3``: q, k, v are then ``torch.float8_e4m3fn`` holding the real
-    inputs divided by those per-tensor scales; O is still bf16.
+    inputs divided by those per-tensor scales; O is still bf16.  ``cta_pair``
+    runs the forward in clusters of two CTAs sharing each 512-row item
+    (tcgen05.mma.cta_group::2; bf16, d = 128).
     """
     lib = load_library()
     in_dtype = torch.bfloat16 if e4m3_scales is None else torch.float8_e4m3fn
@@ -165,7 +169,8 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     opts = FwdOpts(-1.0 if rescale_threshold is None else float(rescale_threshold),
                    None if stats is None else stats.data_ptr(), int(timeout_ns), 0, int(test_fault),
                    0 if window is None else 1, -1 if window is None else int(window[0]),
-                   -1 if window is None else int(window[1]), int(exp_poly_per8))
+                   -1 if window is None else int(window[1]), int(exp_poly_per8),
+                   int(bool(cta_pair)))
     if stats is not None:
         _need(stats, "stats", torch.int64)
     if cu_seqlens is None:

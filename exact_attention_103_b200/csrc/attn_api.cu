@@ -49,6 +49,7 @@ constexpr int kWorkSlots = 64;
 struct DeviceState {
   bool ready = false;
   int sms = 0;
+  int pair_clusters = -1;  // clusters of the pair kernel that fit at once (-1: not asked yet)
   int* err = nullptr;        // device error word
   unsigned* work = nullptr;  // kWorkSlots claim-counter slots (same allocation)
   cudaStream_t slot_stream[kWorkSlots] = {};
@@ -136,6 +137,18 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t total, int H, int d) {
   return make_map_esz(m, ptr, total, H, d, 2);
 }
 
+// The bf16 view {d, H, total} with 64-row boxes (the K halves of a CTA pair).
+bool make_map_rows64(CUtensorMap* m, const void* ptr, int64_t total, int H, int d) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(total)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
+  const cuuint32_t box[3] = {64, 1, 64};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
@@ -219,8 +232,10 @@ attn_status_t plan_fwd(const FwdCall& c, FwdPlan* pl) {
   const bool varlen = c.cu_seqlens != nullptr;
   if (varlen && (B > kMaxVarlenB || N > kMaxVarlenN))
     return fail(ATTN_ERR_UNSUPPORTED, "varlen supports B <= %d and N <= %d", kMaxVarlenB, kMaxVarlenN);
-  pl->T256 = (static_cast<int64_t>(N) + 255) / 256;
-  pl->items_bound = static_cast<int64_t>(B) * pl->T256 * H;
+  const int pair = (c.opts && c.opts->cta_pair) ? 1 : 0;
+  pl->pair = pair;
+  pl->T = (static_cast<int64_t>(N) + (pair ? 511 : 255)) / (pair ? 512 : 256);
+  pl->items_bound = static_cast<int64_t>(B) * pl->T * H;
   pl->dense_tokens = static_cast<int64_t>(B) * N;
   if (pl->items_bound > INT32_MAX / 2 || pl->dense_tokens * H > INT64_MAX / 256 ||
       pl->dense_tokens > INT32_MAX)
@@ -250,6 +265,8 @@ attn_status_t plan_fwd(const FwdCall& c, FwdPlan* pl) {
       wl = opts->window_left;
       wr = opts->window_right;
     }
+    if (opts->cta_pair && (f8 || d != 128 || pl->poly != 0))
+      return fail(ATTN_ERR_UNSUPPORTED, "cta_pair: bf16 inputs, d = 128 and exp_poly_per8 = 0 only");
   }
   const attn_status_t st = select_mask(N, c.causal, has_window, wl, wr, &pl->mask, &pl->win_l, &pl->win_r);
   if (st != ATTN_OK) return st;
@@ -257,16 +274,18 @@ attn_status_t plan_fwd(const FwdCall& c, FwdPlan* pl) {
   return ATTN_OK;
 }
 
-attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total, int sms, int* err,
-                              unsigned* work, attn::FwdLaunch* a) {
+attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total, int sms, int pair_clusters,
+                              int* err, unsigned* work, attn::FwdLaunch* a) {
   const attn_status_t st = load_tensor_map_encoder();
   if (st != ATTN_OK) return st;
   std::memset(a, 0, sizeof(*a));
   const attn_internal::E4m3Scales* f8 = c.f8;
   const int esz = f8 ? 1 : 2;
   if (!make_map_esz(&a->tm_q, c.q, total, c.H, c.d, esz) || !make_map_esz(&a->tm_k, c.k, total, c.H, c.d, esz) ||
-      !make_map_esz(&a->tm_v, c.v, total, c.H, c.d, esz))
+      !make_map_esz(&a->tm_v, c.v, total, c.H, c.d, esz) ||
+      (pl.pair && !make_map_rows64(&a->tm_k2, c.k, total, c.H, c.d)))
     return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled rejected the Q/K/V views");
+  a->pair = pl.pair;
   const bool varlen = c.cu_seqlens != nullptr;
   a->p.o = static_cast<__nv_bfloat16*>(c.o);
   a->p.lse = c.lse;
@@ -274,7 +293,7 @@ attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total
   a->p.B = c.B;
   a->p.H = c.H;
   a->p.N = c.N;
-  a->p.T = static_cast<int>(pl.T256);
+  a->p.T = static_cast<int>(pl.T);
   a->p.total = static_cast<int>(total);
   // The E4M3 scales of Q and K fold into the score scale; V's into 1/l.  One
   // rounding to fp32, from a double product.
@@ -292,9 +311,17 @@ attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total
   a->p.wr = pl.win_r;
   // Dense unmasked launches may split their last wave into half items (see the
   // kernel), so up to twice as many CTAs can be useful there.
-  const int64_t useful = (!varlen && pl.mask == attn::kMaskNone) ? 2 * pl.items_bound : pl.items_bound;
-  a->grid = static_cast<int>(useful < sms ? useful : sms);
-  a->smem = attn::fwd_smem_bytes(c.d, c.B, static_cast<int>(pl.T256), varlen ? 1 : 0, f8 ? 1 : 0);
+  a->smem = attn::fwd_smem_bytes(c.d, c.B, static_cast<int>(pl.T), varlen ? 1 : 0, f8 ? 1 : 0, pl.pair);
+  if (pl.pair) {
+    // Two CTAs per item; as many clusters as fit at once (SMs left over in a GPC
+    // of odd SM count cannot hold a cluster).
+    const int64_t fit = pair_clusters > 0 ? pair_clusters : sms / 2;
+    const int64_t clusters = pl.items_bound < fit ? pl.items_bound : fit;
+    a->grid = static_cast<int>(2 * clusters);
+  } else {
+    const int64_t useful = (!varlen && pl.mask == attn::kMaskNone) ? 2 * pl.items_bound : pl.items_bound;
+    a->grid = static_cast<int>(useful < sms ? useful : sms);
+  }
   return ATTN_OK;
 }
 
@@ -336,7 +363,12 @@ attn_status_t fwd_impl(const attn_internal::FwdCall& c, int64_t total_hint, attn
   }
   attn::FwdLaunch a;
   unsigned* work = work_slot(dev, cs);
-  st = attn_internal::fill_fwd_launch(c, pl, total, dev->sms, dev->err, work, &a);
+  if (pl.pair && dev->pair_clusters < 0) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    dev->pair_clusters = attn::fwd_pair_max_clusters(
+        attn::fwd_smem_bytes(128, c.B, static_cast<int>(pl.T), c.cu_seqlens ? 1 : 0, 0, 1));
+  }
+  st = attn_internal::fill_fwd_launch(c, pl, total, dev->sms, dev->pair_clusters, dev->err, work, &a);
   if (st != ATTN_OK) return st;
   return attn_internal::launch_planned_fwd(c, pl, a, stream);
 }

@@ -79,17 +79,22 @@ enum WaitSite {
   kSiteDrain, kSiteBadLen, kSiteItemFull, kSiteItemEmpty
 };
 
-template <int D, bool F8>
+// PAIR: a CTA pair runs tcgen05.mma.cta_group::2 (M = 256 rows per product, 128 in
+// each CTA); each CTA keeps its own 128 query rows per sub-tile and half of every
+// K/V tile (keys 64r..64r+63 of K, head-dim columns 64r..64r+63 of V for rank r),
+// so a ring slot is half a tile.
+template <int D, bool F8, bool PAIR = false>
 struct Layout {
   static constexpr int ESZ = F8 ? 1 : 2;              // bytes per element (E4M3 / bf16)
   static constexpr int TILE = kBM * D * ESZ;          // bytes of one 128 x D tile
   static constexpr int CHUNK = kBM * 128;             // one 128-byte-wide swizzle chunk
   static constexpr int NCHUNK = TILE / CHUNK;
   static constexpr int KSTEP = 32 / ESZ;              // elements per MMA K step (32 bytes)
-  static constexpr int NSTAGE = (TILE <= 16384) ? 8 : 4;  // K/V ring slots
+  static constexpr int SLOT = PAIR ? TILE / 2 : TILE; // bytes of one K/V ring slot
+  static constexpr int NSTAGE = (SLOT <= 16384) ? 8 : 4;  // K/V ring slots
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE;
-  static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE;
+  static constexpr int BAR_OFF = KV_OFF + NSTAGE * SLOT;
   // barrier indices
   // B_PFULL + kPSplit*s + h: part h of P~ of sub-tile s is in TMEM
   static constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 4,
@@ -101,8 +106,9 @@ struct Layout {
   static constexpr int TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
 };
 
-// A work item: query rows [row_base, row_base + 256) of one (sequence, head) as
-// two 128-row sub-tiles, or only the first sub-tile when `two` is false.
+// A work item: query rows [row_base, row_base + 2 * SUB) of one (sequence, head) as
+// two sub-tiles of SUB rows (SUB = 128; a CTA pair: 256, 128 per CTA), or only the
+// first sub-tile when `two` is false.
 struct Item {
   int b, h, seq_start, L, row_base;
   bool two;
@@ -133,6 +139,7 @@ struct Sched {
   int count;          // number of list positions
   int nbulk;          // items in the bulk
   int gtail;          // first tail group
+  int ishift;         // log2 of the query rows of an item (8: 256 rows; a CTA pair: 9)
 
   __device__ __forceinline__ int seq_T(int i, int& b, int& start, int& L) const {
     if (cu == nullptr) {
@@ -144,7 +151,7 @@ struct Sched {
     b = order[i];
     start = __ldg(cu + b);
     L = __ldg(cu + b + 1) - start;
-    return ceil_div(L, 2 * kBM);
+    return (L + (1 << ishift) - 1) >> ishift;
   }
 
   // SPLIT: the launch may hold half items (dense non-causal only).
@@ -195,18 +202,19 @@ struct Sched {
     const int i = g / H;
     it.h = g - i * H;
     seq_T(i, it.b, it.seq_start, it.L);
-    it.row_base = t * 2 * kBM + ((SPLIT && sub > 0) ? kBM : 0);
+    it.row_base = (t << ishift) + ((SPLIT && sub > 0) ? kBM : 0);
     it.two = !SPLIT || sub < 0;
     return it;
   }
 };
 
 
-// The mask hook, one compile-time functor per MaskKind.  For the 128 query rows
-// [row0, row0 + 128) of a sequence of length L:
-//   tiles()   the key tiles [lo, hi) holding a key visible to some row; the tiles
-//             outside are skipped, not loaded;
-//   partial() whether key tile kb (its first key) may hide a key from some row;
+// The mask hook, one compile-time functor per MaskKind.  For query rows of a
+// sequence of length L:
+//   tiles()   the key tiles [lo, hi) holding a key visible to some row of
+//             [row0, row0 + nrows); the tiles outside are skipped, not loaded;
+//   partial() whether key tile kb (its first key) may hide a key from some row of
+//             the 128 rows [row0, row0 + 128);
 //   cols()    the visible columns [c_lo, c_hi) of that tile for query row q.
 // Causal is the lower triangle of "FlashAttention 1-4 详解", 其他优化 (tiles above
 // the diagonal skipped).  The window is this library's instance of the
@@ -215,15 +223,15 @@ struct Sched {
 template <int MASK>
 struct MaskFn {
   int wl, wr;  // kMaskWindow only; both >= 0 and below 2^30
-  __device__ __forceinline__ void tiles(int row0, int L, int& lo, int& hi) const {
+  __device__ __forceinline__ void tiles(int row0, int nrows, int L, int& lo, int& hi) const {
     const int all = ceil_div(L, kBN);
     lo = 0;
     hi = all;
     if (MASK == kMaskCausal) {
-      hi = min(row0 / kBN + 1, all);  // up to and including the diagonal tile
+      hi = min((row0 + nrows - 1) / kBN + 1, all);  // up to and including the last row's diagonal tile
     } else if (MASK == kMaskWindow) {
       lo = max(row0 - wl, 0) / kBN;
-      hi = ceil_div(min(row0 + kBM + wr, L), kBN);
+      hi = ceil_div(min(row0 + nrows + wr, L), kBN);
     }
   }
   __device__ __forceinline__ bool partial(int kb, int row0, int L) const {
@@ -243,25 +251,25 @@ struct MaskFn {
   }
 };
 
-// Key tiles [lo, hi) that sub-tile s of an item processes (empty when its rows are
-// all past L, or for the missing second sub-tile of a half item).
-template <int MASK>
+// Key tiles [lo, hi) that sub-tile s (SUB rows) of an item processes (empty when
+// its rows are all past L, or for the missing second sub-tile of a half item).
+template <int MASK, int SUB = kBM>
 __device__ __forceinline__ void kv_range(const Item& it, int s, const MaskFn<MASK>& mk, int& lo,
                                          int& hi) {
   lo = hi = 0;
   if (s == 1 && !it.two) return;
-  const int row0 = it.row_base + s * kBM;
+  const int row0 = it.row_base + s * SUB;
   if (row0 >= it.L) return;
-  mk.tiles(row0, it.L, lo, hi);
+  mk.tiles(row0, SUB, it.L, lo, hi);
 }
 
 // Key tiles of the whole item: the union of its sub-tiles' ranges (sub-tile 0 is
 // never empty and its range starts no later than sub-tile 1's).
-template <int MASK>
+template <int MASK, int SUB = kBM>
 __device__ __forceinline__ void item_range(const Item& it, const MaskFn<MASK>& mk, int& lo, int& n) {
   int lo0, hi0, lo1, hi1;
-  kv_range<MASK>(it, 0, mk, lo0, hi0);
-  kv_range<MASK>(it, 1, mk, lo1, hi1);
+  kv_range<MASK, SUB>(it, 0, mk, lo0, hi0);
+  kv_range<MASK, SUB>(it, 1, mk, lo1, hi1);
   lo = lo0;
   n = (hi1 > hi0 ? hi1 : hi0) - lo0;
 }
@@ -280,13 +288,15 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 //   order[B] | gstart[B+1] | off[T+1] | cnt[T+1] | tstart[T]
 __host__ __device__ constexpr int varlen_table_ints(int B, int T) { return 2 * B + 3 * T + 3; }
 
-// Builds the varlen list tables (one warp): sequences sorted by tile-pair count
-// (descending, stable counting sort), the items before each sorted sequence, and
+// Builds the varlen list tables (one warp): sequences sorted by item count (items of
+// 2^ishift query rows; descending, stable counting sort), the items before each
+// sorted sequence, and
 // the tail of the list (the last groups holding at least `tail_items` items, see
 // Sched).  Writes gtail and nbulk; returns the number of items, or -1 if cu[0] !=
-// 0, cu[B] != total, or some length is negative or exceeds T*256.
+// 0, cu[B] != total, or some length is negative or exceeds T items.
 __device__ int build_varlen_tables(const int* cu, int B, int H, int T, int total, int tail_items,
-                                   int* tab, int lane, int* gtail_out, int* nbulk_out) {
+                                   int ishift, int* tab, int lane, int* gtail_out, int* nbulk_out) {
+  auto items_of = [&](int L) { return (L + (1 << ishift) - 1) >> ishift; };
   int* order = tab;
   int* gstart = order + B;
   int* off = gstart + B + 1;
@@ -297,7 +307,7 @@ __device__ int build_varlen_tables(const int* cu, int B, int H, int T, int total
   int bad = (lane == 0 && (__ldg(cu) != 0 || __ldg(cu + B) != total)) ? 1 : 0;
   for (int b = lane; b < B; b += 32) {
     const int L = __ldg(cu + b + 1) - __ldg(cu + b);
-    const int nt = L < 0 ? 0 : ceil_div(L, 2 * kBM);
+    const int nt = L < 0 ? 0 : items_of(L);
     if (L < 0 || nt > T) { bad = 1; continue; }
     atomicAdd(&off[nt], 1);
   }
@@ -322,7 +332,7 @@ __device__ int build_varlen_tables(const int* cu, int B, int H, int T, int total
   for (int base = 0; base < B; base += 32) {
     const int b = base + lane;
     int key = -1;
-    if (b < B) key = ceil_div(__ldg(cu + b + 1) - __ldg(cu + b), 2 * kBM);
+    if (b < B) key = items_of(__ldg(cu + b + 1) - __ldg(cu + b));
     const uint32_t same = __match_any_sync(0xffffffffu, key);
     const int rank = __popc(same & lt_mask);
     if (b < B) order[off[key] + rank] = b;
@@ -337,7 +347,7 @@ __device__ int build_varlen_tables(const int* cu, int B, int H, int T, int total
     int v = 0;
     if (i < B) {
       const int b = order[i];
-      v = H * ceil_div(__ldg(cu + b + 1) - __ldg(cu + b), 2 * kBM);
+      v = H * items_of(__ldg(cu + b + 1) - __ldg(cu + b));
     }
     const int incl = warp_incl_scan(v, lane);
     if (i < B) gstart[i] = carry + incl - v;
@@ -395,14 +405,26 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64
 // F8: Q, K, V are E4M3 with per-tensor scales (S = Q K^T and O += P~ V with
 // tcgen05.mma kind::f8f6f4, P~ rounded to E4M3; "FlashAttention 1-4 详解", 其他优化:
 // FP8 tensor cores for the forward's matrix products).
-template <int D, int MASK, int POLY, bool F8>
+// PAIR: the launch runs in clusters of two CTAs that share every item ("FlashAttention
+// V4 deep-dive", section 3.3: 2-CTA MMA; FA-4 summary items [13][14]).  An item is
+// 512 query rows, two sub-tiles of 256 rows with 128 in each CTA.  The leader (rank
+// 0) claims items and issues every tcgen05.mma.cta_group::2 (M = 256) for both CTAs;
+// each CTA loads its own query rows and half of each K/V tile (K by keys, V by
+// head-dim columns) from this GPU's memory, with no multicast, so a CTA moves and
+// stores half the K/V bytes of the single-CTA kernel; the softmax warps of both CTAs
+// work on their own rows and release P~ to the leader.  tm_k2 views K with 64-row
+// boxes (the K halves); it is unused otherwise.
+template <int D, int MASK, int POLY, bool F8, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Lay = Layout<D, F8>;
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k2,
+               const FwdParams p) {
+  using Lay = Layout<D, F8, PAIR>;
   static_assert(!F8 || D == 128, "E4M3 path: one 128-byte row per head");
+  static_assert(!PAIR || (D == 128 && !F8), "CTA pairs: bf16, d = 128");
   constexpr int NS = Lay::NSTAGE;
-  constexpr bool SPLIT = MASK == kMaskNone;  // the launch may hold half items
+  constexpr bool SPLIT = MASK == kMaskNone && !PAIR;  // the launch may hold half items
+  constexpr int SUB = PAIR ? 2 * kBM : kBM;            // query rows of a sub-tile (pair-wide)
   static_assert(POLY >= 0 && POLY <= 8, "pairs per 8");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -416,17 +438,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* tab = reinterpret_cast<int*>(smem + Lay::TABLE_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tail_items = 2 * static_cast<int>(gridDim.x);
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0: the pair's leader (or a lone CTA)
+  const bool leader = rank == 0;
+  // CTAs (pairs) that claim items; the list's tail holds two items per claimer.
+  const int claimers = PAIR ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
+  const int tail_items = 2 * claimers;
+  // The leader's copy of a barrier, as a shared::cluster address (pair mode).
+  auto lbar = [&](int i) -> uint32_t { return PAIR ? mapa_shared(bar(i), 0) : bar(i); };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Lay::B_QFULL), 1);
     mbar_init(bar(Lay::B_QEMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Lay::B_SFULL + s), 1);
-      for (int h = 0; h < kPSplit; ++h) mbar_init(bar(Lay::B_PFULL + kPSplit * s + h), 4);
+      // the 4 softmax warps of the sub-tile (of both CTAs of a pair) release P~
+      for (int h = 0; h < kPSplit; ++h) mbar_init(bar(Lay::B_PFULL + kPSplit * s + h), PAIR ? 8 : 4);
       mbar_init(bar(Lay::B_OFULL + s), 1);
       mbar_init(bar(Lay::B_ITEMF + s), 1);  // the producer publishes a claimed position
-      mbar_init(bar(Lay::B_ITEME + s), 9);  // the MMA warp and the 8 softmax warps read it
+      // read by the MMA warp and the 8 softmax warps (a pair: and the follower's
+      // producer and 8 softmax warps)
+      mbar_init(bar(Lay::B_ITEME + s), PAIR ? 18 : 9);
     }
     mbar_init(bar(Lay::B_DRAIN), 1);
     for (int i = 0; i < NS; ++i) {
@@ -437,8 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 9) {
-    tmem_alloc(sb + Lay::MISC_OFF, 512);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(sb + Lay::MISC_OFF, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(sb + Lay::MISC_OFF, 512);
+      tmem_relinquish();
+    }
   }
   if (warp == 8) {
     int count, gtail, nbulk;
@@ -450,8 +486,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       gtail = groups - k;
       nbulk = gtail * p.T;
     } else {
-      count = build_varlen_tables(p.cu_seqlens, p.B, p.H, p.T, p.total, tail_items, tab, lane, &gtail,
-                                  &nbulk);
+      count = build_varlen_tables(p.cu_seqlens, p.B, p.H, p.T, p.total, tail_items, PAIR ? 9 : 8, tab,
+                                  lane, &gtail, &nbulk);
       if (count < 0) {
         count = gtail = nbulk = 0;
         if (lane == 0 && p.err) atomicCAS(p.err, 0, 1 | (kSiteBadLen << 8));
@@ -466,6 +502,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if constexpr (PAIR) {  // both CTAs' barriers exist before either arrives on the other's
+    cluster_arrive();
+    cluster_wait();
+  }
 
   const uint32_t tmem = misc[0];
   Sched sch;
@@ -477,14 +517,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   sch.pairs = static_cast<int>(misc[2]);
   sch.gtail = static_cast<int>(misc[3]);
   sch.nbulk = static_cast<int>(misc[4]);
+  sch.ishift = PAIR ? 9 : 8;
   // Dense non-causal items all cost the same: when the last wave would leave
   // CTAs idle, its items are split into 128-row half items so it spreads over
   // more SMs (a half item runs without a ping-pong partner, but the wave is
   // shorter).  Causal and varlen lists end with their shortest items.
   sch.split = 0;
   if (SPLIT && p.cu_seqlens == nullptr) {
-    const int rem = sch.pairs % static_cast<int>(gridDim.x);
-    if (rem > 0 && 2 * rem <= static_cast<int>(gridDim.x)) sch.split = rem;
+    const int rem = sch.pairs % claimers;
+    if (rem > 0 && 2 * rem <= claimers) sch.split = rem;
   }
   sch.count = sch.pairs + sch.split;
   WaitCtl wc;
@@ -497,14 +538,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Consumer roles (the MMA warp, the softmax warps): the k-th list position this
   // CTA claimed, from the queue (one arrival per warp frees the entry); -1 ends
   // the list, and so does an expired wait.
+  // In a pair every entry is published to both CTAs and freed on the leader.
   auto take_item = [&](int k) -> int {
     const int e = k & 1;
-    if (!__all_sync(0xffffffffu, mbar_wait(bar(Lay::B_ITEMF + e), (k >> 1) & 1, wc,
-                                           timeout_code(kSiteItemFull))))
+    if (!__all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_ITEMF + e), (k >> 1) & 1, wc,
+                                                 timeout_code(kSiteItemFull))))
       return -1;
     const int idx = queue[e];
     __syncwarp();
-    if (lane == 0) mbar_arrive(bar(Lay::B_ITEME + e));
+    if (lane == 0) {
+      if (PAIR && !leader) mbar_arrive_remote(lbar(Lay::B_ITEME + e));
+      else mbar_arrive(bar(Lay::B_ITEME + e));
+    }
     return idx;
   };
 
@@ -525,10 +570,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (idx < 0) break;
       const Item it = sch.template decode<SPLIT>(idx);
       const int b = it.b, h = it.h, seq_start = it.seq_start, L = it.L;
-      int jlo, jhi;
-      kv_range<MASK>(it, s, mk, jlo, jhi);
+      int jlo, jhi;  // the sub-tile's key tiles (of both CTAs of a pair)
+      kv_range<MASK, SUB>(it, s, mk, jlo, jhi);
       if (jhi <= jlo) continue;
-      const int row0 = it.row_base + s * kBM;
+      const int row0 = it.row_base + s * SUB + static_cast<int>(rank) * kBM;  // this CTA's rows
       const int q_row = row0 + r;
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
@@ -664,7 +709,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // and fenced before the warp converges; lane 0 then releases them.
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(Lay::B_PFULL + kPSplit * s + half));
+          if (lane == 0) {
+            if (PAIR && !leader) mbar_arrive_remote(lbar(Lay::B_PFULL + kPSplit * s + half));
+            else mbar_arrive(bar(Lay::B_PFULL + kPSplit * s + half));
+          }
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       }
@@ -716,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Whole warp walks the loop and waits; one elected lane issues the copies.
     if (elect_one()) {
       tma_prefetch_map(&tm_q);
-      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(PAIR ? &tm_k2 : &tm_k);
       tma_prefetch_map(&tm_v);
     }
     __syncwarp();
@@ -726,26 +774,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     int n_items = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      // Claim the next list position once its queue entry is free, and publish it.
+      // Claim the next list position once its queue entry is free, and publish it
+      // (to both CTAs of a pair; the follower's producer takes it like the other roles).
       const int e = k & 1;
-      if (k >= 2) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_ITEME + e), ((k >> 1) - 1) & 1, wc,
-                                               timeout_code(kSiteItemEmpty)));
-        if (!ok) break;
-      }
       int idx = -1;
-      if (lane == 0) {
-        const unsigned c = atomicAdd(p.work, 1u);
-        if (c < static_cast<unsigned>(sch.count)) idx = static_cast<int>(c);
-        queue[e] = idx;
-        mbar_arrive(bar(Lay::B_ITEMF + e));
+      if (PAIR && !leader) {
+        idx = take_item(k);
+      } else {
+        if (k >= 2) {
+          ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_ITEME + e), ((k >> 1) - 1) & 1, wc,
+                                                       timeout_code(kSiteItemEmpty)));
+          if (!ok) break;
+        }
+        if (lane == 0) {
+          const unsigned c = atomicAdd(p.work, 1u);
+          if (c < static_cast<unsigned>(sch.count)) idx = static_cast<int>(c);
+          queue[e] = idx;
+          mbar_arrive(bar(Lay::B_ITEMF + e));
+          if constexpr (PAIR) {
+            const uint32_t qaddr = sb + Lay::MISC_OFF + 4 * (8 + e);
+            st_shared_remote_u32(mapa_shared(qaddr, 1), static_cast<uint32_t>(idx));
+            mbar_arrive_remote(mapa_shared(bar(Lay::B_ITEMF + e), 1));  // release: orders the store
+          }
+        }
+        idx = __shfl_sync(0xffffffffu, idx, 0);
       }
-      idx = __shfl_sync(0xffffffffu, idx, 0);
       if (idx < 0) break;
       const Item it = sch.template decode<SPLIT>(idx);
       const int h = it.h, seq_start = it.seq_start;
       int jlo, nkv;
-      item_range<MASK>(it, mk, jlo, nkv);
+      item_range<MASK, SUB>(it, mk, jlo, nkv);
       if (k > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QEMPTY), qe_phase, wc, timeout_code(kSiteQEmpty)));
         if (!ok) break;
@@ -755,17 +813,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // consumers' waits run out.
       const bool withhold = p.test_fault == 1 && k == 0;
       if (!withhold && elect_one()) {
-        mbar_arrive_expect_tx(bar(Lay::B_QFULL), 2 * Lay::TILE);
+        // Each CTA loads its own query rows; the leader counts the pair's bytes.
+        if (leader) mbar_arrive_expect_tx(bar(Lay::B_QFULL), (PAIR ? 4 : 2) * Lay::TILE);
 #pragma unroll
-        for (int s = 0; s < 2; ++s)
+        for (int s = 0; s < 2; ++s) {
+          const int qr = seq_start + it.row_base + s * SUB + static_cast<int>(rank) * kBM;
 #pragma unroll
-          for (int c = 0; c < Lay::NCHUNK; ++c)
-            tma_load_3d(sb + Lay::Q_OFF + s * Lay::TILE + c * Lay::CHUNK, &tm_q, bar(Lay::B_QFULL),
-                        c * (128 / Lay::ESZ), h, seq_start + it.row_base + s * kBM, pol_q);
+          for (int c = 0; c < Lay::NCHUNK; ++c) {
+            const uint32_t dst = sb + Lay::Q_OFF + s * Lay::TILE + c * Lay::CHUNK;
+            if constexpr (PAIR) tma_load_3d_pair(dst, &tm_q, lbar(Lay::B_QFULL), c * 64, h, qr, pol_q);
+            else tma_load_3d(dst, &tm_q, bar(Lay::B_QFULL), c * (128 / Lay::ESZ), h, qr, pol_q);
+          }
+        }
       }
       __syncwarp();
       if (!withhold) ++n_items;
       for (int j = 0; j < nkv && ok; ++j) {
+        const int key0 = seq_start + (jlo + j) * kBN;
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
           const uint32_t slot = n_ld % NS;
@@ -775,33 +839,60 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
           }
           if (elect_one()) {
-            mbar_arrive_expect_tx(bar(Lay::B_KVFULL + slot), Lay::TILE);
+            const uint32_t dst = sb + Lay::KV_OFF + slot * Lay::SLOT;
+            if constexpr (PAIR) {
+              // K: keys 64*rank..+63 (two 64-row boxes, one per 64 head-dim columns);
+              // V: all 128 keys, head-dim columns 64*rank..+63 (one box).
+              if (leader) mbar_arrive_expect_tx(bar(Lay::B_KVFULL + slot), 2 * Lay::SLOT);
+              if (which == 0) {
 #pragma unroll
-            for (int c = 0; c < Lay::NCHUNK; ++c)
-              tma_load_3d(sb + Lay::KV_OFF + slot * Lay::TILE + c * Lay::CHUNK, which ? &tm_v : &tm_k,
-                          bar(Lay::B_KVFULL + slot), c * (128 / Lay::ESZ), h,
-                          seq_start + (jlo + j) * kBN, pol_kv);
+                for (int c = 0; c < 2; ++c)
+                  tma_load_3d_pair(dst + c * (Lay::SLOT / 2), &tm_k2, lbar(Lay::B_KVFULL + slot), c * 64, h,
+                                   key0 + static_cast<int>(rank) * 64, pol_kv);
+              } else {
+                tma_load_3d_pair(dst, &tm_v, lbar(Lay::B_KVFULL + slot), static_cast<int>(rank) * 64, h,
+                                 key0, pol_kv);
+              }
+            } else {
+              mbar_arrive_expect_tx(bar(Lay::B_KVFULL + slot), Lay::TILE);
+#pragma unroll
+              for (int c = 0; c < Lay::NCHUNK; ++c)
+                tma_load_3d(dst + c * Lay::CHUNK, which ? &tm_v : &tm_k, bar(Lay::B_KVFULL + slot),
+                            c * (128 / Lay::ESZ), h, key0, pol_kv);
+            }
           }
           __syncwarp();
           ++n_ld;
         }
       }
     }
-    // Drain: every issued copy must have landed before the CTA may exit.
-    const uint32_t first = n_ld > static_cast<uint32_t>(NS) ? n_ld - NS : 0u;
-    for (uint32_t n = first; n < n_ld; ++n)
-      drain_wait(bar(Lay::B_KVFULL + n % NS), (n / NS) & 1u, kDrainLimitNs);
-    if (n_items > 0) drain_wait(bar(Lay::B_QFULL), (n_items - 1) & 1u, kDrainLimitNs);
-  } else {
+    // Drain: every issued copy must have landed before the CTA may exit (a pair's
+    // copies all complete on the leader's barriers; the leader drains them, and
+    // the pair waits for each other before exiting).
+    if (leader) {
+      const uint32_t first = n_ld > static_cast<uint32_t>(NS) ? n_ld - NS : 0u;
+      for (uint32_t n = first; n < n_ld; ++n)
+        drain_wait(bar(Lay::B_KVFULL + n % NS), (n / NS) & 1u, kDrainLimitNs);
+      if (n_items > 0) drain_wait(bar(Lay::B_QFULL), (n_items - 1) & 1u, kDrainLimitNs);
+    }
+  } else if (leader) {
     // ---------------------------------------------------------------- MMA
+    // (a pair's follower has no MMA role: the leader issues the pair's products)
     // The whole warp walks the loop and waits; one elected lane issues each MMA
     // and commit.  Issue order per key tile j (ping-pong of the two sub-tiles):
     //   PV(0, j-1), S(0, j), PV(1, j-1), S(1, j)
     // each only where tile j (j-1) lies in that sub-tile's key range.
     // S(s, j) overwrites P(s, j-1) in TMEM, which PV(s, j-1) read just before; the
     // tensor pipe executes one thread's MMAs in issue order.
-    constexpr uint32_t idesc_s = F8 ? idesc_e4m3_f32(kBM, kBN, 0, 0) : idesc_bf16_f32(kBM, kBN, 0, 0);
-    constexpr uint32_t idesc_o = F8 ? idesc_e4m3_f32(kBM, D, 0, 1) : idesc_bf16_f32(kBM, D, 0, 1);
+    constexpr int M = PAIR ? 2 * kBM : kBM;  // rows of one product (a pair: 128 in each CTA)
+    constexpr uint32_t idesc_s = F8 ? idesc_e4m3_f32(M, kBN, 0, 0) : idesc_bf16_f32(M, kBN, 0, 0);
+    constexpr uint32_t idesc_o = F8 ? idesc_e4m3_f32(M, D, 0, 1) : idesc_bf16_f32(M, D, 0, 1);
+    // Commit to this CTA's barrier, or to the barrier at the same offset in both
+    // CTAs of a pair.
+    auto commit = [&](int i) {
+      if constexpr (PAIR) tc_commit_pair(bar(i), 0x3);
+      else tc_commit(bar(i));
+    };
     const uint32_t tS0 = tmem + Lay::TM_S0, tS1 = tmem + Lay::TM_S1;
     const uint32_t tO0 = tmem + Lay::TM_O0, tO1 = tmem + Lay::TM_O1;
     uint32_t n_ld = 0, q_phase = 0, p_phase0 = 0, p_phase1 = 0;
@@ -811,10 +902,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (idx < 0) break;
       const Item it = sch.template decode<SPLIT>(idx);
       int jlo, nkv, lo0, hi0, lo1, hi1;
-      item_range<MASK>(it, mk, jlo, nkv);
-      kv_range<MASK>(it, 0, mk, lo0, hi0);
-      kv_range<MASK>(it, 1, mk, lo1, hi1);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QFULL), q_phase, wc, timeout_code(kSiteQFull)));
+      item_range<MASK, SUB>(it, mk, jlo, nkv);
+      kv_range<MASK, SUB>(it, 0, mk, lo0, hi0);
+      kv_range<MASK, SUB>(it, 1, mk, lo1, hi1);
+      ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_QFULL), q_phase, wc, timeout_code(kSiteQFull)));
       if (!ok) break;
       q_phase ^= 1u;
       tc_fence_after();
@@ -824,11 +915,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t nV = nK - 1u;        // ... and of V_{j-1}
         const uint32_t slotK = nK % NS, slotV = nV % NS;
         if (jj < nkv)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KVFULL + slotK), (nK / NS) & 1u, wc,
-                                                 timeout_code(kSiteKvFull)));
+          ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_KVFULL + slotK), (nK / NS) & 1u, wc,
+                                                       timeout_code(kSiteKvFull)));
         if (ok && jj > 0)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KVFULL + slotV), (nV / NS) & 1u, wc,
-                                                 timeout_code(kSiteKvFull)));
+          ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_KVFULL + slotV), (nV / NS) & 1u, wc,
+                                                       timeout_code(kSiteKvFull)));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -837,7 +928,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int los = s ? lo1 : lo0, his = s ? hi1 : hi0;
           if (ok && jj > 0 && j - 1 >= los && j - 1 < his) {
             uint32_t& ph = s ? p_phase1 : p_phase0;
-            const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::TILE;
+            const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::SLOT;
             constexpr int NK = kBN / Lay::KSTEP;  // PV K steps per key tile
             // Each part of P~ is multiplied as soon as the softmax warps release it.
             // One K step: KSTEP keys = 32 bytes of a P~ row (8 TMEM columns) and
@@ -845,16 +936,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             static_assert(NK % kPSplit == 0, "K steps per part");
 #pragma unroll
             for (int half = 0; half < kPSplit && ok; ++half) {
-              ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_PFULL + kPSplit * s + half), ph, wc,
-                                                     timeout_code(kSitePFull)));
+              ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_PFULL + kPSplit * s + half), ph, wc,
+                                                           timeout_code(kSitePFull)));
               if (!ok) break;
               tc_fence_after();
 #pragma unroll
               for (int kk = half * NK / kPSplit; kk < (half + 1) * NK / kPSplit; ++kk) {
                 if (elect_one()) {
+                  // V (a pair: this CTA's 64 head-dim columns of it) is MN-major.
                   const uint64_t dv = sdesc_sw128(vbase + kk * Lay::KSTEP * 128, Lay::CHUNK, 1024);
                   const uint32_t acc = (j - 1 > los || kk > 0) ? 1u : 0u;
-                  if constexpr (F8) mma_ts_f8(tO, tS + kk * 8, dv, idesc_o, acc);
+                  if constexpr (PAIR) mma_ts_pair(tO, tS + kk * 8, dv, idesc_o, acc);
+                  else if constexpr (F8) mma_ts_f8(tO, tS + kk * 8, dv, idesc_o, acc);
                   else mma_ts(tO, tS + kk * 8, dv, idesc_o, acc);
                 }
                 __syncwarp();
@@ -863,43 +956,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) {
               ph ^= 1u;
               if (j == his) {
-                if (elect_one()) tc_commit(bar(Lay::B_OFULL + s));
+                if (elect_one()) commit(Lay::B_OFULL + s);
                 __syncwarp();
               }
             }
           }
           if (ok && j >= los && j < his) {
             const uint32_t qbase = sb + Lay::Q_OFF + s * Lay::TILE;
-            const uint32_t kbase = sb + Lay::KV_OFF + slotK * Lay::TILE;
+            const uint32_t kbase = sb + Lay::KV_OFF + slotK * Lay::SLOT;
+            // K's rows (a pair: this CTA's 64 keys) in 128-byte chunks of head dims.
+            constexpr int KCHUNK = PAIR ? Lay::SLOT / 2 : Lay::CHUNK;
 #pragma unroll
             for (int kk = 0; kk < D / Lay::KSTEP; ++kk) {
               const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+              const uint32_t offk = (kk >> 2) * KCHUNK + (kk & 3) * 32;
               if (elect_one()) {
                 const uint64_t da = sdesc_sw128(qbase + off, 16, 1024);
-                const uint64_t db = sdesc_sw128(kbase + off, 16, 1024);
-                if constexpr (F8) mma_ss_f8(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
+                const uint64_t db = sdesc_sw128(kbase + offk, 16, 1024);
+                if constexpr (PAIR) mma_ss_pair(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
+                else if constexpr (F8) mma_ss_f8(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
                 else mma_ss(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
               }
               __syncwarp();
             }
-            if (elect_one()) tc_commit(bar(Lay::B_SFULL + s));
+            if (elect_one()) commit(Lay::B_SFULL + s);
             __syncwarp();
           }
         }
         if (!ok) break;
         if (elect_one()) {
-          if (jj < nkv) tc_commit(bar(Lay::B_KVEMPTY + slotK));
-          if (jj > 0) tc_commit(bar(Lay::B_KVEMPTY + slotV));
+          if (jj < nkv) commit(Lay::B_KVEMPTY + slotK);
+          if (jj > 0) commit(Lay::B_KVEMPTY + slotV);
           // The query tiles are free after the item's last S product (an item
           // without key tiles -- an empty half item -- frees them at once).
-          if (jj == (nkv > 0 ? nkv - 1 : 0)) tc_commit(bar(Lay::B_QEMPTY));
+          if (jj == (nkv > 0 ? nkv - 1 : 0)) commit(Lay::B_QEMPTY);
         }
         __syncwarp();
       }
       n_ld += 2u * nkv;
     }
     // Drain: every MMA issued by this warp completes before TMEM is freed.
-    if (elect_one()) tc_commit(bar(Lay::B_DRAIN));
+    if (elect_one()) {
+      if constexpr (PAIR) tc_commit_pair(bar(Lay::B_DRAIN), 0x1);
+      else tc_commit(bar(Lay::B_DRAIN));
+    }
     __syncwarp();
     if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, kDrainLimitNs)) && lane == 0 && p.err)
       atomicCAS(p.err, 0, timeout_code(kSiteDrain));
@@ -907,8 +1007,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) {  // neither CTA of a pair leaves while the other may still use its memory
+    cluster_arrive();
+    cluster_wait();
+  }
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, 512);
+  if (warp == 9) {
+    if constexpr (PAIR) tmem_dealloc_pair(tmem, 512);
+    else tmem_dealloc(tmem, 512);
+  }
   // The last CTA to finish returns the claim counter to zero for the next launch
   // that uses it: every CTA's producer has made its last claim before its CTA
   // counts itself finished here.
@@ -921,23 +1028,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool F8>
-constexpr int smem_bytes_fixed() { return 1024 + Layout<D, F8>::TABLE_OFF; }
+template <int D, bool F8, bool PAIR = false>
+constexpr int smem_bytes_fixed() { return 1024 + Layout<D, F8, PAIR>::TABLE_OFF; }
 
 }  // namespace
 
-int fwd_smem_bytes(int D, int B, int T, int varlen, int fp8) {
-  const int fixed = fp8 ? smem_bytes_fixed<128, true>()
-                        : (D == 128 ? smem_bytes_fixed<128, false>() : smem_bytes_fixed<64, false>());
+int fwd_smem_bytes(int D, int B, int T, int varlen, int fp8, int pair) {
+  const int fixed = pair ? smem_bytes_fixed<128, false, true>()
+                         : fp8 ? smem_bytes_fixed<128, true>()
+                               : (D == 128 ? smem_bytes_fixed<128, false>() : smem_bytes_fixed<64, false>());
   return fixed + (varlen ? varlen_table_ints(B, T) * 4 : 0);
 }
 
-template <int D, int MASK, int POLY, bool F8 = false>
+template <int D, int MASK, int POLY, bool F8 = false, bool PAIR = false>
 static cudaError_t launch_t(const FwdLaunch& a, cudaStream_t st) {
-  auto kern = fwd_kernel<D, MASK, POLY, F8>;
+  auto kern = fwd_kernel<D, MASK, POLY, F8, PAIR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem);
   if (e != cudaSuccess) return e;
-  kern<<<a.grid, kThreads, a.smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.p);
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = a.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, a.tm_q, a.tm_k, a.tm_v, a.tm_k2, a.p);
+    if (e != cudaSuccess) return e;
+  } else {
+    kern<<<a.grid, kThreads, a.smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_k2, a.p);
+  }
   return cudaGetLastError();
 }
 
@@ -956,6 +1081,11 @@ static cudaError_t launch_m(const FwdLaunch& a, MaskKind mask, int poly, cudaStr
 }
 
 cudaError_t launch_fwd(const FwdLaunch& a, int D, MaskKind mask, int poly, int fp8, cudaStream_t st) {
+  if (a.pair) {  // CTA pairs: bf16, d = 128, exponentials on MUFU
+    if (mask == kMaskCausal) return launch_t<128, kMaskCausal, 0, false, true>(a, st);
+    if (mask == kMaskWindow) return launch_t<128, kMaskWindow, 0, false, true>(a, st);
+    return launch_t<128, kMaskNone, 0, false, true>(a, st);
+  }
   if (fp8) {  // E4M3: d = 128; exponentials all on MUFU or 2 of every 8 pairs on the FMA pipe
     if (poly == 2) {
       if (mask == kMaskCausal) return launch_t<128, kMaskCausal, 2, true>(a, st);
@@ -967,6 +1097,26 @@ cudaError_t launch_fwd(const FwdLaunch& a, int D, MaskKind mask, int poly, int f
     return launch_t<128, kMaskNone, 0, true>(a, st);
   }
   return D == 128 ? launch_m<128>(a, mask, poly, st) : launch_m<64>(a, mask, poly, st);
+}
+
+int fwd_pair_max_clusters(int smem) {
+  // Clusters of two CTAs of this kernel (causal, MUFU exponentials) that fit at once.
+  auto kern = fwd_kernel<128, kMaskCausal, 0, false, true>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return 0;
+  return n;
 }
 
 }  // namespace attn

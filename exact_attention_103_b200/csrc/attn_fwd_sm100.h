@@ -21,7 +21,7 @@ struct FwdParams {
   float* lse;            // dense [B, H, N]; varlen [H, total]
   const int* cu_seqlens; // device int32[B+1] or null (dense)
   int B, H, N;
-  int T;                 // ceil(N / 256): query tile-pairs of the longest sequence
+  int T;                 // items of the longest sequence: ceil(N / 256) (CTA pairs: / 512)
   int total;             // packed tokens (dense: B*N)
   float scale_log2;      // scale * log2(e)
   float tau;             // conditional-rescale threshold, log2 units
@@ -39,14 +39,19 @@ struct FwdParams {
 
 struct FwdLaunch {
   // 3-D maps {D, H, total} with 128-byte swizzle; box {64, 1, 128} for bf16 and
-  // {128, 1, 128} for E4M3 (one 128-byte row either way)
-  CUtensorMap tm_q, tm_k, tm_v;
+  // {128, 1, 128} for E4M3 (one 128-byte row either way); tm_k2: K with box
+  // {64, 1, 64} (the K halves of CTA pairs; unused otherwise)
+  CUtensorMap tm_q, tm_k, tm_v, tm_k2;
   FwdParams p;
   int grid;
   int smem;
+  int pair;  // launch in clusters of two CTAs (tcgen05.mma.cta_group::2); grid even
 };
 
-int fwd_smem_bytes(int D, int B, int T, int varlen, int fp8);
+// T: items of the longest sequence (256 query rows each; CTA pairs: 512).
+int fwd_smem_bytes(int D, int B, int T, int varlen, int fp8, int pair);
+// Clusters of two CTAs of the pair kernel that fit on the device at once (0: none).
+int fwd_pair_max_clusters(int smem);
 // poly: exponentials per 8 column pairs on the FMA-pipe polynomial (0, 2 or 8).
 // fp8: E4M3 inputs (D = 128, poly = 0 only).
 cudaError_t launch_fwd(const FwdLaunch& a, int D, MaskKind mask, int poly, int fp8, cudaStream_t st);

@@ -35,16 +35,18 @@ struct FwdPlan {
   int test_fault, poly;
   attn::MaskKind mask;
   int win_l, win_r;
-  int64_t T256, items_bound, dense_tokens;
+  int pair;  // clusters of two CTAs (opts->cta_pair)
+  int64_t T, items_bound, dense_tokens;  // T: items of the longest sequence (256 or 512 rows)
 };
 
 // Checks every argument of a forward call on the host; touches no device state.
 attn_status_t plan_fwd(const FwdCall& c, FwdPlan* pl);
 // Builds the launch of a planned forward call over `total` packed tokens (dense:
 // B*N) on a device with `sms` SMs, the kernel recording errors in `err` and
-// claiming work items through the two zeroed words at `work` (device addresses).
-attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total, int sms, int* err,
-                              unsigned* work, attn::FwdLaunch* a);
+// claiming work items through the two zeroed words at `work` (device addresses);
+// pair_clusters: clusters of the CTA-pair kernel that fit at once (pair launches).
+attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total, int sms, int pair_clusters,
+                              int* err, unsigned* work, attn::FwdLaunch* a);
 attn_status_t launch_planned_fwd(const FwdCall& c, const FwdPlan& pl, const attn::FwdLaunch& a,
                                  attn_stream_t stream);
 // Looks up the driver's tensor-map encoder once per process.

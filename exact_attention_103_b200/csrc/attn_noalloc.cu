@@ -95,7 +95,7 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
   st = setup_device(&dev);
   if (st != ATTN_OK) return st;
   attn::FwdLaunch a;
-  st = attn_internal::fill_fwd_launch(c, pl, total, dev->sms, dev->scratch,
+  st = attn_internal::fill_fwd_launch(c, pl, total, dev->sms, 0, dev->scratch,
                                       reinterpret_cast<unsigned*>(dev->scratch + 2), &a);
   if (st != ATTN_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);

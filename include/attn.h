@@ -119,7 +119,15 @@ ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, voi
  *      units).  0 (the default, all MUFU), 2 or 8; other values are rejected
  *      (ATTN_ERR_INVALID_ARG).  The polynomial has a relative error below 7.5e-5,
  *      under half a bf16 ulp, so the results differ from the MUFU path only by
- *      the rounding of P~. */
+ *      the rounding of P~.
+ *  cta_pair: nonzero runs the forward in clusters of two CTAs on neighbouring SMs
+ *      that share each item of 512 query rows ("FlashAttention V4 deep-dive",
+ *      section 3.3, 2-CTA MMA; FA-4 summary [13][14]): the pair's leader issues
+ *      tcgen05.mma.cta_group::2 products of 256 rows, and each CTA loads its own
+ *      query rows and half of every K/V tile (no multicast), halving each SM's
+ *      K/V traffic.  bf16 inputs, d = 128, exp_poly_per8 = 0 (else
+ *      ATTN_ERR_UNSUPPORTED).  Results equal the single-CTA path's up to the order
+ *      of fp32 accumulation inside the products. */
 typedef struct {
   float rescale_threshold;
   unsigned long long* stats;
@@ -130,6 +138,7 @@ typedef struct {
   int window_left;
   int window_right;
   int exp_poly_per8;
+  int cta_pair;
 } attn_fwd_opts_t;
 
 /* attn_fwd with options (opts may be NULL = defaults). */

@@ -151,3 +151,17 @@ def test_missing_library_fails_loudly():
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT,
                        timeout=300)
     assert r.stdout.strip() == "raised True", r.stdout + r.stderr
+
+
+def test_cta_pair_limits(lib):
+    """CTA pairs run bf16, d = 128, all-MUFU exponentials only."""
+    for d, poly in ((64, 0), (128, 2)):
+        opts = ea.FwdOpts(-1.0, None, 0, 0, 0, 0, 0, 0, poly, 1)
+        st = lib.attn_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, d, 0, 0.1, None,
+                             ctypes.byref(opts), None)
+        assert st == ea.ATTN_ERR_UNSUPPORTED, (d, poly)
+        assert "cta_pair" in ea.last_error()
+    opts = ea.FwdOpts(-1.0, None, 0, 0, 0, 0, 0, 0, 0, 1)
+    st = lib.attn_fwd_e4m3(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0, 0.1, 1.0, 1.0, 1.0, None,
+                           ctypes.byref(opts), None)
+    assert st == ea.ATTN_ERR_UNSUPPORTED

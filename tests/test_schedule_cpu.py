@@ -22,15 +22,15 @@ def ceil_div(a, b):
     return (a + b - 1) // b
 
 
-def build_varlen_tables(cu, B, H, T, total, tail_items):
+def build_varlen_tables(cu, B, H, T, total, tail_items, ishift=8):
     """Twin of build_varlen_tables: returns (order, gstart, tstart, items, gtail, nbulk)
-    or None for an invalid cu_seqlens."""
+    or None for an invalid cu_seqlens (items of 2^ishift query rows)."""
     if cu[0] != 0 or cu[B] != total:
         return None
     nts = []
     for b in range(B):
         L = cu[b + 1] - cu[b]
-        nt = 0 if L < 0 else ceil_div(L, 2 * BM)
+        nt = 0 if L < 0 else ceil_div(L, 1 << ishift)
         if L < 0 or nt > T:
             return None
         nts.append(nt)
@@ -69,10 +69,13 @@ def build_varlen_tables(cu, B, H, T, total, tail_items):
 class Sched:
     """Twin of the kernel's Sched (list parameters and decode)."""
 
-    def __init__(self, B, H, N, grid, cu=None, split_ok=False):
+    def __init__(self, B, H, N, grid, cu=None, split_ok=False, pair=False):
         self.B, self.H, self.N, self.cu = B, H, N, cu
-        self.T = ceil_div(N, 2 * BM)
-        tail_items = 2 * grid
+        self.ishift = 9 if pair else 8  # CTA pairs: items of 512 rows
+        self.T = ceil_div(N, 1 << self.ishift)
+        claimers = grid // 2 if pair else grid
+        tail_items = 2 * claimers
+        grid = claimers
         if cu is None:
             groups = B * H
             k = min(ceil_div(tail_items, self.T), groups)
@@ -80,11 +83,11 @@ class Sched:
             self.gtail = groups - k
             self.nbulk = self.gtail * self.T
         else:
-            r = build_varlen_tables(cu, B, H, self.T, cu[B], tail_items)
+            r = build_varlen_tables(cu, B, H, self.T, cu[B], tail_items, self.ishift)
             assert r is not None
             self.order, self.gstart, self.tstart, self.pairs, self.gtail, self.nbulk = r
         self.split = 0
-        if split_ok and cu is None:
+        if split_ok and cu is None and not pair:
             rem = self.pairs % grid
             if rem > 0 and 2 * rem <= grid:
                 self.split = rem
@@ -95,7 +98,7 @@ class Sched:
             return i, i * self.N, self.N, self.T
         b = self.order[i]
         L = self.cu[b + 1] - self.cu[b]
-        return b, self.cu[b], L, ceil_div(L, 2 * BM)
+        return b, self.cu[b], L, ceil_div(L, 1 << self.ishift)
 
     def decode(self, idx):
         """(b, h, row_base, two, t) of list position idx."""
@@ -142,21 +145,23 @@ class Sched:
         i = g // H
         h = g - i * H
         b, _, L, _ = self.seq(i)
-        row_base = t * 2 * BM + (BM if (sub > 0) else 0)
+        row_base = (t << self.ishift) + (BM if (sub > 0) else 0)
         two = sub < 0
         return b, h, row_base, two, t
 
 
 def _coverage(s, lengths):
     seen = {}
+    blocks = (1 << s.ishift) // (2 * BM)  # 128-row blocks of a sub-tile (a pair: one per CTA)
     for idx in range(s.count):
         b, h, row_base, two, _ = s.decode(idx)
         L = lengths[b]
         for st in ((0, 1) if two else (0,)):
-            row0 = row_base + st * BM
-            if row0 < L:  # a sub-tile past the sequence end does no work
-                key = (b, h, row0)
-                seen[key] = seen.get(key, 0) + 1
+            for blk in range(blocks):
+                row0 = row_base + (st * blocks + blk) * BM
+                if row0 < L:  # rows past the sequence end are not stored
+                    key = (b, h, row0)
+                    seen[key] = seen.get(key, 0) + 1
     expected = {(b, h, r) for b, L in enumerate(lengths) for h in range(s.H)
                 for r in range(0, L, BM)}
     assert set(seen) == expected, (len(set(seen)), len(expected))
@@ -227,3 +232,18 @@ def test_invalid_cu_seqlens_rejected():
     assert build_varlen_tables([1, 5, 9], 2, 1, 1, 9, 4) is None  # cu[0] != 0
     assert build_varlen_tables([0, 5, 9], 2, 1, 1, 10, 4) is None  # cu[B] != total
     assert build_varlen_tables([0, 600], 1, 1, 2, 600, 4) is None  # longer than T*256
+
+
+@pytest.mark.parametrize("grid", [148, 144, 2])
+def test_pair_lists_cover_every_block_once(grid):
+    """CTA pairs (items of 512 rows, claimed by one CTA of each pair): the dense and
+    packed benchmark workloads and random packed batches."""
+    _coverage(Sched(2, 16, 8192, grid, pair=True), [8192] * 2)
+    _coverage(Sched(4, 16, 2048, grid, pair=True), [2048] * 4)
+    _coverage(Sched(3, 5, 700, grid, pair=True), [700] * 3)
+    w = ai.VARLEN
+    _coverage(Sched(w.B, w.H, w.N, grid, cu=w.cu_seqlens(), pair=True), w.seq_lengths())
+    rng = random.Random(12)
+    for _ in range(20):
+        lengths = [rng.randint(0, 3000) for _ in range(rng.choice([1, 4, 30]))]
+        _coverage(Sched(len(lengths), 3, max(max(lengths), 1), grid, cu=_cu(lengths), pair=True), lengths)
