@@ -369,17 +369,22 @@ def run_ours(args, rank, world, local):
 
     # One untimed launch with the kernel's counters on: how often the conditional
     # rescale fired (the counters are not kept under a sliding window).
+    # Also at tau = 0 (rescale whenever a row's maximum grows: the rule the pages'
+    # skip-rate figure compares against).
     rescale = None
     if w.window is None:
-        counters = torch.zeros(2, dtype=torch.int64, device=dev)
-        ea.fwd(q, k, v, causal=w.causal, scale=scale, cu_seqlens=cu, max_seqlen=max_len,
-               out=out, lse=lse, exp_poly_per8=args.exp_poly_per8, e4m3_scales=f8,
-               stats=counters, cta_pair=args.cta_pair)
-        ea.get_device_status()
-        rescaled, row_tiles = (int(x) for x in counters.cpu())
-        rescale = {"rows_rescaled": rescaled, "row_tiles_after_first": row_tiles,
-                   "skip_rate": (1.0 - rescaled / row_tiles) if row_tiles else None,
-                   "tau_log2": 4.0 if w.e4m3 else 8.0}
+        rescale = {}
+        for tau in (None, 0.0):
+            counters = torch.zeros(2, dtype=torch.int64, device=dev)
+            ea.fwd(q, k, v, causal=w.causal, scale=scale, cu_seqlens=cu, max_seqlen=max_len,
+                   out=out, lse=lse, exp_poly_per8=args.exp_poly_per8, e4m3_scales=f8,
+                   stats=counters, cta_pair=args.cta_pair, rescale_threshold=tau)
+            ea.get_device_status()
+            rescaled, row_tiles = (int(x) for x in counters.cpu())
+            key = "default" if tau is None else "tau0"
+            rescale[key] = {"tau_log2": (4.0 if w.e4m3 else 8.0) if tau is None else tau,
+                            "rows_rescaled": rescaled, "row_tiles_after_first": row_tiles,
+                            "skip_rate": (1.0 - rescaled / row_tiles) if row_tiles else None}
     achieved = flops / (statistics.mean(times) / 1e3) / 1e12  # per launch, this rank
     clk = clocks.summary()
     # The denominator: the measured cuBLAS bf16 peak as a burst, or its sustained
