@@ -1,4 +1,4 @@
-"""The forward kernel's FMA-pipe exponential (exp2_poly in attn_fwd_sm100.cu, with
+"""The forward kernel's FMA-pipe exponential (exp2_poly and exp2_poly_x2 in softmax_math.cuh, with
 the coefficients of csrc/exp2_poly.h) emulated step by step in float32 on the CPU
 and checked against 2^x: the relative error stays within the bound the header
 states, over the whole range the kernel feeds it (P~ arguments up to the rescale
