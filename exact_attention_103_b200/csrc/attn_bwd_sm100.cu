@@ -19,9 +19,21 @@
 // elected lane issues).  The MMA warps issue their products in a software-
 // pipelined order so the next tile's exponentials overlap the current tile's
 // products (dK/dV: dV(n), S^T(n+1), dK(n), dP^T(n+1); dQ: dQ(j), dP(j+1), S(j+2)
-// with S double-buffered).  MASK selects the visibility rule of the forward's mask
-// hook: none, causal, or the sliding window (only the tiles the window reaches are
-// visited).  Every wait is bounded as in the forward kernel.
+// with S double-buffered).  Streamed tiles sit in single-tile ring slots, each
+// released as soon as its last product has read it (dK/dV: dO after dV, Q after
+// dK; dQ: V after dP, K after dQ), so the next copies start early.
+//
+// In the dK/dV kernel the per-query LSE and D vary along the TMEM columns, the
+// same for every thread of a warp.  Rather than broadcast them across lanes, the
+// kernel lets the tensor core subtract them: S^T and dP^T get one more K-step of
+// 16 in which A is a constant tile of ones and B holds -LSE/scale (resp. -D) of
+// each query, split into three bf16 terms (hi + mid + lo, exact to ~2^-24 of the
+// value), so TMEM receives S^T - LSE/scale and dP^T - D directly.  Queries past
+// the sequence end get -inf (P = 0).
+//
+// MASK selects the visibility rule of the forward's mask hook: none, causal, or
+// the sliding window (only the tiles the window reaches are visited).  Every wait
+// is bounded as in the forward kernel.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -40,31 +52,94 @@ __host__ __device__ constexpr int timeout_code(int site) { return 4 | (site << 8
 enum BwdSite { kSiteKv = 32, kSiteStageFull, kSiteStageEmpty, kSiteS, kSiteP, kSiteDs, kSiteAcc,
                kSiteDrain, kSiteBadLen };
 
+// Shared memory of the dK/dV kernel (offsets from a 1024-aligned base): resident
+// K_j (A0) and V_j (A1); ONES, the A operand of the extra K-step; two Q slots and
+// two dO slots, each a tile followed by its 128 x 16 extra-step operand (XTRA).
 template <int D>
-struct BwdLayout {
+struct DkdvLayout {
   static constexpr int TILE = kTile * D * 2;
-  static constexpr int CHUNK = kTile * 128;
-  // smem: two resident tiles (A0, A1), then two ring stages of two tiles each,
-  // then per-stage vectors (128 LSE + 128 D floats), barriers, misc.
+  static constexpr int CHUNK = kTile * 128;  // 128 rows x 64 columns, 128-byte swizzle
+  static constexpr int XTRA = kTile * 32;    // 128 rows x 16 bf16, no swizzle
+  static constexpr int SLOT = TILE + XTRA;
+  static constexpr int NSLOT = 2;            // per operand (Q, dO)
   static constexpr int A0_OFF = 0;
   static constexpr int A1_OFF = TILE;
-  static constexpr int STAGE_OFF = 2 * TILE;
-  static constexpr int NSTAGE = 2;
-  static constexpr int VEC_OFF = STAGE_OFF + NSTAGE * 2 * TILE;
-  static constexpr int BAR_OFF = VEC_OFF + NSTAGE * 2 * kTile * 4;
-  // barrier indices
-  // B_S: S (or S^T) is in TMEM region A (B_S1: in region A', the dQ kernel's
-  // second score buffer); B_DP: dP (or dP^T) is in region B.
-  static constexpr int B_RES = 0, B_FULL = 1, B_EMPTY = 3, B_S = 5, B_P = 6, B_DS = 7, B_ACC = 8,
-                       B_DRAIN = 9, B_DP = 10, B_S1 = 11, NBARS = 12;
+  static constexpr int ONES_OFF = 2 * TILE;
+  static constexpr int Q_OFF = ONES_OFF + XTRA;
+  static constexpr int DO_OFF = Q_OFF + NSLOT * SLOT;
+  static constexpr int BAR_OFF = DO_OFF + NSLOT * SLOT;
+  // B_S: S^T in TMEM region A; B_DP: dP^T in region B; B_P / B_DS: P^T / dS^T
+  // written back by the eight elementwise warps.
+  static constexpr int B_RES = 0, B_QFULL = 1, B_QEMPTY = 3, B_OFULL = 5, B_OEMPTY = 7, B_S = 9,
+                       B_DP = 10, B_P = 11, B_DS = 12, B_ACC = 13, B_DRAIN = 14, NBARS = 15;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM = MISC_OFF + 64;
-  // TMEM columns: region A (S^T or S, then packed P^T), region B (dP^T or dP,
-  // then packed dS), accumulators.  The dQ kernel has one accumulator and uses
-  // the second one's columns as A', a second score buffer (128 columns).
-  static constexpr int TM_A = 0, TM_B = 128, TM_ACC0 = 256, TM_ACC1 = 256 + D, TM_A2 = 256 + D;
-  static_assert(TM_A2 + kTile <= 512, "A' fits in TMEM");
+  // TMEM columns: region A (S^T, then packed P^T), region B (dP^T, then packed
+  // dS^T), the dV and dK accumulators.
+  static constexpr int TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
+  static_assert(Q_OFF % 1024 == 0 && SLOT % 1024 == 0, "swizzled tiles stay 1024-aligned");
+  static_assert(1024 + SMEM <= 232448, "fits in shared memory");
 };
+
+// Shared memory of the dQ kernel: resident Q_i (A0) and dO_i (A1); three K slots
+// and two V slots.
+template <int D>
+struct DqLayout {
+  static constexpr int TILE = kTile * D * 2;
+  static constexpr int CHUNK = kTile * 128;
+  static constexpr int NK = 3, NV = 2;
+  static constexpr int A0_OFF = 0;
+  static constexpr int A1_OFF = TILE;
+  static constexpr int K_OFF = 2 * TILE;
+  static constexpr int V_OFF = K_OFF + NK * TILE;
+  static constexpr int BAR_OFF = V_OFF + NV * TILE;
+  // B_S / B_S1: S in TMEM region A / A'; B_DP: dP in region B; B_DS: dS written back.
+  static constexpr int B_RES = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 9, B_S = 11,
+                       B_S1 = 12, B_DP = 13, B_DS = 14, B_ACC = 15, B_DRAIN = 16, NBARS = 17;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int SMEM = MISC_OFF + 64;
+  // TMEM columns: region A (S), region B (dP, then packed dS), the dQ accumulator,
+  // region A' (the second score buffer).
+  static constexpr int TM_A = 0, TM_B = 128, TM_DQ = 256, TM_A2 = 256 + D;
+  static_assert(TM_A2 + kTile <= 512, "A' fits in TMEM");
+  static_assert(1024 + SMEM <= 232448, "fits in shared memory");
+};
+
+// Shared-memory matrix descriptor of a K-major operand without swizzling: core
+// matrices of 8 rows x 16 bytes stored contiguously (128 bytes), lbo bytes between
+// core matrices adjacent along K, sbo bytes between 8-row groups.
+__device__ __forceinline__ uint64_t sdesc_kmajor_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;  // descriptor version of this architecture; layout type 0 = no swizzle
+  return d;
+}
+// A descriptor advanced by `bytes` within the same operand (adds to the start
+// address field; shared-memory addresses stay below 2^18, so nothing carries out).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+// Byte offset of row r's first core-matrix row in a 128 x 16 operand of that layout
+// (lbo = 128, sbo = 256).
+__device__ __forceinline__ uint32_t xtra_row_off(int r) { return (r & 7) * 16 + (r >> 3) * 256; }
+
+// Orders this thread's generic-proxy shared-memory writes before later reads by
+// the tensor core (async proxy).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// -x as three bf16 terms whose sum is -x to ~2^-24 relative (x = +inf: -inf, 0, 0),
+// packed as the first four bf16 of an extra-step row: {t0, t1, t2, 0}.
+__device__ __forceinline__ uint2 neg_split3(float x) {
+  if (isinf(x)) return make_uint2(pack_bf16x2(-INFINITY, 0.f), 0u);
+  const float y = -x;
+  const float t0 = __bfloat162float(__float2bfloat16_rn(y));
+  const float r1 = y - t0;
+  const float t1 = __bfloat162float(__float2bfloat16_rn(r1));
+  const float t2 = r1 - t1;
+  return make_uint2(pack_bf16x2(t0, t1), pack_bf16x2(t2, 0.f));
+}
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
@@ -144,31 +219,19 @@ __device__ __forceinline__ void store_half_row(uint32_t t_acc, __nv_bfloat16* ds
   }
 }
 
-// Shared set-up of both main kernels: barriers, TMEM (512 columns), abort flag.
-// full_arrivals: arrivals that complete a ring stage (besides its bytes).
-template <int D>
-__device__ __forceinline__ uint32_t bwd_setup(uint8_t* smem, uint32_t sb, int warp, int full_arrivals) {
-  using Lay = BwdLayout<D>;
-  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
+// Shared set-up of both main kernels: barriers (counts from `counts`, NB of them),
+// TMEM (512 columns), abort flag.  Returns the TMEM base address.
+template <int NB>
+__device__ __forceinline__ uint32_t bwd_setup(uint8_t* smem, uint32_t sb, int bar_off, int misc_off,
+                                              int warp, const uint8_t (&counts)[NB]) {
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + misc_off);
   if (threadIdx.x == 0) {
-    auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
-    mbar_init(bar(Lay::B_RES), 1);
-    for (int s = 0; s < Lay::NSTAGE; ++s) {
-      mbar_init(bar(Lay::B_FULL + s), full_arrivals);
-      mbar_init(bar(Lay::B_EMPTY + s), 1);
-    }
-    mbar_init(bar(Lay::B_S), 1);
-    mbar_init(bar(Lay::B_S1), 1);
-    mbar_init(bar(Lay::B_DP), 1);
-    mbar_init(bar(Lay::B_P), 8);
-    mbar_init(bar(Lay::B_DS), 8);
-    mbar_init(bar(Lay::B_ACC), 1);
-    mbar_init(bar(Lay::B_DRAIN), 1);
+    for (int i = 0; i < NB; ++i) mbar_init(sb + bar_off + 8 * i, counts[i]);
     misc[1] = 0u;
     fence_barrier_init();
   }
   if (warp == 9) {
-    tmem_alloc(sb + Lay::MISC_OFF, 512);
+    tmem_alloc(sb + misc_off, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -220,17 +283,18 @@ __global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
 }
 
 // ------------------------------------------------------------------ dK, dV
-// CTA: key tile j of (b, h).  Resident: K_j (A0), V_j (A1).  Ring: (Q_i, dO_i).
-// Per query tile i:  S^T = K_j Q_i^T (TMEM A), dP^T = V_j dO_i^T (TMEM B);
-//   P^T = exp2(scale*log2e*S^T - LSE2_i) (causal: zero where query < key) -> A;
-//   dV += P^T dO_i;  dS^T = P^T o (dP^T - D_i) -> B;  dK += dS^T Q_i.
+// CTA: key tile j of (b, h).  Resident: K_j (A0), V_j (A1).  Streamed: Q_i, dO_i.
+// Per query tile i (extra K-step: see the file comment):
+//   S'^T = K_j Q_i^T - LSE_i/scale (TMEM A), dP'^T = V_j dO_i^T - D_i (TMEM B);
+//   P^T = exp2(scale*log2e * S'^T) (causal: zero where query < key) -> A;
+//   dV += P^T dO_i;  dS^T = P^T o dP'^T -> B;  dK += dS^T Q_i.
 // MASK: 0 none, 1 causal, 2 sliding window (see BwdParams::wl, wr).
 template <int D, int MASK>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p) {
-  using Lay = BwdLayout<D>;
+  using Lay = DkdvLayout<D>;
   BwdItem it;
   constexpr bool CAUSAL = MASK == 1;
   if (!decode_block(p, true, CAUSAL, it)) return;  // uniform for the CTA
@@ -240,7 +304,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t tmem = bwd_setup<D>(smem, sb, warp, 2);  // copies + query vectors
+  // The extra-step operands: ONES = {1, 1, 1, 0, ...} in every row; the slots'
+  // operands are zero beyond their first four columns (the producer writes only
+  // those).
+  {
+    uint4* z = reinterpret_cast<uint4*>(smem + Lay::ONES_OFF);
+    const uint32_t one2 = pack_bf16x2(1.f, 1.f), one0 = pack_bf16x2(1.f, 0.f);
+    for (int u = threadIdx.x; u < Lay::XTRA / 16; u += kThreads) {
+      // 16-byte unit u: core-matrix row (u & 7) of row group (u >> 4); units with
+      // bit 3 set hold K columns 8..15
+      z[u] = ((u >> 3) & 1) ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(one2, one0, 0u, 0u);
+    }
+    for (int s2 = 0; s2 < 2 * Lay::NSLOT; ++s2) {
+      uint4* x = reinterpret_cast<uint4*>(smem + Lay::Q_OFF + s2 * Lay::SLOT + Lay::TILE);
+      for (int u = threadIdx.x; u < Lay::XTRA / 16; u += kThreads) x[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
+  const uint8_t counts[Lay::NBARS] = {1, 2, 2, 1, 1, 2, 2, 1, 1, 1, 1, 8, 8, 1, 1};
+  const uint32_t tmem = bwd_setup<Lay::NBARS>(smem, sb, Lay::BAR_OFF, Lay::MISC_OFF, warp, counts);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
   WaitCtl wc;
   wc.abort = reinterpret_cast<volatile uint32_t*>(misc + 1);
@@ -257,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     i_end = min(ntiles, (j * kTile + kTile - 1 + p.wl) / kTile + 1);
   }
   const int nq = i_end - i_first;
-  float* vec = reinterpret_cast<float*>(smem + Lay::VEC_OFF);
+  auto q_slot = [&](int n) -> uint32_t { return sb + Lay::Q_OFF + (n & 1) * Lay::SLOT; };
+  auto o_slot = [&](int n) -> uint32_t { return sb + Lay::DO_OFF + (n & 1) * Lay::SLOT; };
 
   if (warp < 8) {
     // ---------------------------------------------------- elementwise work
@@ -271,20 +354,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_phase = 0, dp_phase = 0;
     bool ok = true;
     for (int n = 0; n < nq && ok; ++n) {
-      const int i = i_first + n, st = n & 1;
+      const int i = i_first + n;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_S), s_phase, wc, timeout_code(kSiteS)));
       if (!ok) break;
       s_phase ^= 1u;
       tc_fence_after();
-      // The 64 query columns' LSE2 and D (written before S^T(n) was issued): lane l
-      // holds entries 2l, 2l+1 and the warp broadcasts them by shuffles.
-      const float2 my_l = reinterpret_cast<const float2*>(vec + st * 2 * kTile + 64 * hf)[lane];
-      const float2 my_d = reinterpret_cast<const float2*>(vec + st * 2 * kTile + kTile + 64 * hf)[lane];
       uint32_t sv[64];
       tmem_ld_x64(tA, sv);
       // P^T for this thread's 64 query columns (causal diagonal tile: a query
-      // sees the key only if query >= key; rows past the sequence have LSE2 = +inf).
-      // Window: query q = qb + c sees this key iff key - wr <= q <= key + wl.
+      // sees the key only if query >= key).  Window: query q = qb + c sees this
+      // key iff key - wr <= q <= key + wl.
       int lim = (CAUSAL && i == j) ? r - 64 * hf : -1;  // columns < lim are masked
       int lim_hi = 64;                                   // columns > lim_hi are masked
       if (MASK == 2) {
@@ -293,13 +372,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         lim_hi = key + p.wl - qb;
       }
       float pv[64];
-      uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const float lc = __shfl_sync(0xffffffffu, (c & 1) ? my_l.y : my_l.x, c >> 1);
-        const float e = fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lc));
+        const float e = fast_exp2(__uint_as_float(sv[c]) * sl);
         pv[c] = (c < lim || (MASK == 2 && c > lim_hi)) ? 0.f : e;
       }
+      uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
       tmem_st_x32(tA, pk);
@@ -316,10 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int c0 = 32 * q2 + 2 * c;
-          const float d0 = __shfl_sync(0xffffffffu, my_d.x, c0 >> 1);
-          const float d1 = __shfl_sync(0xffffffffu, my_d.y, c0 >> 1);
-          pk[16 * q2 + c] = pack_bf16x2(pv[c0] * (__uint_as_float(dv[2 * c]) - d0),
-                                        pv[c0 + 1] * (__uint_as_float(dv[2 * c + 1]) - d1));
+          pk[16 * q2 + c] = pack_bf16x2(pv[c0] * __uint_as_float(dv[2 * c]),
+                                        pv[c0 + 1] * __uint_as_float(dv[2 * c + 1]));
         }
       }
       tmem_st_x32(tB, pk);
@@ -330,8 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool store = key < it.L;
       const int64_t row = (static_cast<int64_t>(it.seq_start + key) * p.H + it.h) * D + (D / 2) * hf;
-      const uint32_t t_dv = tmem + lane_bits + Lay::TM_ACC0 + (D / 2) * hf;
-      const uint32_t t_dk = tmem + lane_bits + Lay::TM_ACC1 + (D / 2) * hf;
+      const uint32_t t_dv = tmem + lane_bits + Lay::TM_DV + (D / 2) * hf;
+      const uint32_t t_dk = tmem + lane_bits + Lay::TM_DK + (D / 2) * hf;
       store_half_row<D>(t_dv, p.dv + row, 1.f, store);
       store_half_row<D>(t_dk, p.dk + row, p.scale, store);
     }
@@ -350,87 +426,101 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+    const float l_to_s = kLog2e / p.scale_log2;  // LSE -> the same units as K Q^T (1/scale)
     bool ok = true;
     for (int n = 0; n < nq && ok; ++n) {
-      const int i = i_first + n, st = n & 1;
-      // Per-query vectors of this tile: LSE in log2 units (+inf past the
-      // sequence, so P = 0 there) and D.  Read into registers before the stage is
-      // free, so their latency overlaps the wait and the copies.
-      float lv[kTile / 32], dv[kTile / 32];
+      const int i = i_first + n;
+      // The extra-step rows of this query tile: lane l writes rows 4l..4l+3 (read
+      // into registers before the slots are free, so the latency overlaps the waits).
+      uint2 xl[4], xd[4];
 #pragma unroll
-      for (int u = 0; u < kTile / 32; ++u) {
-        const int qrow = i * kTile + 32 * u + lane;
+      for (int u = 0; u < 4; ++u) {
+        const int qrow = i * kTile + 4 * lane + u;
         const bool in = qrow < it.L;
         const int64_t vi = vec_index(p, it.b, it.h, it.seq_start, in ? qrow : 0);
-        lv[u] = in ? __ldg(p.lse + vi) * kLog2e : INFINITY;
-        dv[u] = in ? __ldg(p.dpre + vi) : 0.f;
+        xl[u] = neg_split3(in ? __ldg(p.lse + vi) * l_to_s : INFINITY);
+        xd[u] = neg_split3(in ? __ldg(p.dpre + vi) : 0.f);
       }
-      if (n >= Lay::NSTAGE) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_EMPTY + st), ((n >> 1) - 1) & 1u, wc,
+      // Each slot's barrier counts two arrivals: the copies' (with their bytes)
+      // and the warp's, after it has written the extra-step rows.
+      auto fill = [&](uint32_t slot, uint32_t full, const CUtensorMap* tm, const uint2 (&x)[4]) {
+        if (elect_one()) {
+          mbar_arrive_expect_tx(full, Lay::TILE);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(slot + c * Lay::CHUNK, tm, full, c * 64, it.h, it.seq_start + i * kTile, pol_ring);
+        }
+        uint8_t* xs = smem + (slot - sb) + Lay::TILE;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint2*>(xs + xtra_row_off(4 * lane + u)) = x[u];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(full);
+      };
+      const int sl2 = n & 1;
+      if (n >= Lay::NSLOT) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QEMPTY + sl2), ((n >> 1) - 1) & 1u, wc,
                                                timeout_code(kSiteStageEmpty)));
         if (!ok) break;
       }
-      // The stage's barrier counts two arrivals: the copies' (with their bytes)
-      // and the warp's, after it has written the vectors.
-      if (elect_one()) {
-        mbar_arrive_expect_tx(bar(Lay::B_FULL + st), 2 * Lay::TILE);
-        const uint32_t base = sb + Lay::STAGE_OFF + st * 2 * Lay::TILE;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(base + c * Lay::CHUNK, &tm_q, bar(Lay::B_FULL + st), c * 64, it.h,
-                      it.seq_start + i * kTile, pol_ring);
-          tma_load_3d(base + Lay::TILE + c * Lay::CHUNK, &tm_do, bar(Lay::B_FULL + st), c * 64, it.h,
-                      it.seq_start + i * kTile, pol_ring);
-        }
+      fill(q_slot(n), bar(Lay::B_QFULL + sl2), &tm_q, xl);
+      if (n >= Lay::NSLOT) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_OEMPTY + sl2), ((n >> 1) - 1) & 1u, wc,
+                                               timeout_code(kSiteStageEmpty)));
+        if (!ok) break;
       }
-      float* v = vec + st * 2 * kTile;
-#pragma unroll
-      for (int u = 0; u < kTile / 32; ++u) {
-        v[32 * u + lane] = lv[u];
-        v[kTile + 32 * u + lane] = dv[u];
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(Lay::B_FULL + st));
+      fill(o_slot(n), bar(Lay::B_OFULL + sl2), &tm_do, xd);
     }
     // Drain: copies still in flight must land before the CTA exits.
     drain_wait(bar(Lay::B_RES), 0u, kDrainLimitNs);
-    for (int n = (nq > Lay::NSTAGE ? nq - Lay::NSTAGE : 0); n < nq; ++n)
-      drain_wait(bar(Lay::B_FULL + (n & 1)), (n >> 1) & 1u, kDrainLimitNs);
+    for (int n = (nq > Lay::NSLOT ? nq - Lay::NSLOT : 0); n < nq; ++n) {
+      drain_wait(bar(Lay::B_QFULL + (n & 1)), (n >> 1) & 1u, kDrainLimitNs);
+      drain_wait(bar(Lay::B_OFULL + (n & 1)), (n >> 1) & 1u, kDrainLimitNs);
+    }
   } else {
     // ---------------------------------------------------------------- MMA
+    // Each product's K-steps are issued back to back by one elected lane, with
+    // descriptors built once and advanced by compile-time offsets.
     constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0, 0);
     constexpr uint32_t idesc_acc = idesc_bf16_f32(kTile, D, 0, 1);
     const uint32_t tA = tmem + Lay::TM_A, tB = tmem + Lay::TM_B;
-    const uint32_t tdV = tmem + Lay::TM_ACC0, tdK = tmem + Lay::TM_ACC1;
+    const uint32_t tdV = tmem + Lay::TM_DV, tdK = tmem + Lay::TM_DK;
+    const uint64_t ones = sdesc_kmajor_plain(sb + Lay::ONES_OFF, 128, 256);
+    const uint64_t dK0 = sdesc_sw128(sb + Lay::A0_OFF, 16, 1024), dV0 = sdesc_sw128(sb + Lay::A1_OFF, 16, 1024);
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_RES), 0, wc, timeout_code(kSiteKv)));
     uint32_t p_phase = 0, ds_phase = 0;
-    auto stage_q = [&](int n) -> uint32_t { return sb + Lay::STAGE_OFF + (n & 1) * 2 * Lay::TILE; };
-    // S^T = K Q_n^T into region A (A and B K-major from shared memory).
-    auto issue_st = [&](int n) {
-      const uint32_t qb = stage_q(n);
+    auto wait_full = [&](int b0, int n) -> bool {
+      const bool r = __all_sync(0xffffffffu, mbar_wait(bar(b0 + (n & 1)), (n >> 1) & 1u, wc,
+                                                       timeout_code(kSiteStageFull)));
+      if (r) tc_fence_after();
+      return r;
+    };
+    // t = A (K_j or V_j, K-major) times the streamed tile's transpose (K-major), plus
+    // the extra step, into TMEM region t; commit to `done`.
+    auto issue_score = [&](uint32_t t, uint64_t a0, uint32_t slot, uint32_t done) {
+      if (elect_one()) {
+        const uint64_t b0 = sdesc_sw128(slot, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-        if (elect_one())
-          mma_ss(tA, sdesc_sw128(sb + Lay::A0_OFF + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
-        __syncwarp();
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+          mma_ss(t, desc_add(a0, off), desc_add(b0, off), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_ss(t, ones, sdesc_kmajor_plain(slot + Lay::TILE, 128, 256), idesc_s, 1u);
+        tc_commit(done);
       }
-      if (elect_one()) tc_commit(bar(Lay::B_S));
       __syncwarp();
     };
-    // dP^T = V dO_n^T into region B.
-    auto issue_dpt = [&](int n) {
-      const uint32_t dob = stage_q(n) + Lay::TILE;
+    // acc += (packed bf16 from TMEM region ta) times the streamed tile (MN-major);
+    // commit to `done` (the tile's slot is then free).
+    auto issue_acc = [&](uint32_t acc, uint32_t ta, uint32_t slot, bool first, uint32_t done) {
+      if (elect_one()) {
+        const uint64_t b0 = sdesc_sw128(slot, Lay::CHUNK, 1024);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-        if (elect_one())
-          mma_ss(tB, sdesc_sw128(sb + Lay::A1_OFF + off, 16, 1024), sdesc_sw128(dob + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
-        __syncwarp();
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(acc, ta + packed_col(kk), desc_add(b0, kk * 2048), idesc_acc, (!first || kk > 0) ? 1u : 0u);
+        tc_commit(done);
       }
-      if (elect_one()) tc_commit(bar(Lay::B_DP));
       __syncwarp();
     };
     // Software pipeline over query tiles: per tile n the tensor pipe runs
@@ -438,52 +528,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     // so the elementwise work on tile n+1 (exponentials) overlaps dK(n) and
     // dP^T(n+1), and dS of tile n overlaps dV(n) and S^T(n+1).  Region A is
     // rewritten by S^T(n+1) only after dV(n) has read P^T(n) (one issuing thread:
-    // in order), region B by dP^T(n+1) only after dK(n) has read dS^T(n).
+    // in order), region B by dP^T(n+1) only after dK(n) has read dS^T(n).  dO(n)'s
+    // slot is released after dV(n), Q(n)'s after dK(n).
     if (ok && nq > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL), 0u, wc, timeout_code(kSiteStageFull)));
-      if (ok) {
-        tc_fence_after();
-        issue_st(0);
-        issue_dpt(0);
-      }
+      ok = wait_full(Lay::B_QFULL, 0);
+      if (ok) issue_score(tA, dK0, q_slot(0), bar(Lay::B_S));
+      if (ok) ok = wait_full(Lay::B_OFULL, 0);
+      if (ok) issue_score(tB, dV0, o_slot(0), bar(Lay::B_DP));
     }
     for (int n = 0; n < nq && ok; ++n) {
-      const int st = n & 1;
-      const uint32_t qb = stage_q(n), dob = qb + Lay::TILE;
+      const int sl2 = n & 1;
       // dV += P^T dO (A = P^T from TMEM, B = dO MN-major).
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_P), p_phase, wc, timeout_code(kSiteP)));
       if (!ok) break;
       p_phase ^= 1u;
       tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk) {
-        if (elect_one())
-          mma_ts(tdV, tA + packed_col(kk), sdesc_sw128(dob + kk * 2048, Lay::CHUNK, 1024), idesc_acc,
-                 (n > 0 || kk > 0) ? 1u : 0u);
-        __syncwarp();
-      }
+      issue_acc(tdV, tA, o_slot(n), n == 0, bar(Lay::B_OEMPTY + sl2));
       if (n + 1 < nq) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL + ((n + 1) & 1)), ((n + 1) >> 1) & 1u, wc,
-                                               timeout_code(kSiteStageFull)));
+        ok = wait_full(Lay::B_QFULL, n + 1);
         if (!ok) break;
-        tc_fence_after();
-        issue_st(n + 1);
+        issue_score(tA, dK0, q_slot(n + 1), bar(Lay::B_S));
       }
       // dK += dS^T Q (A = dS^T from TMEM, B = Q MN-major); scale applied at the end.
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DS), ds_phase, wc, timeout_code(kSiteDs)));
       if (!ok) break;
       ds_phase ^= 1u;
       tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk) {
-        if (elect_one())
-          mma_ts(tdK, tB + packed_col(kk), sdesc_sw128(qb + kk * 2048, Lay::CHUNK, 1024), idesc_acc,
-                 (n > 0 || kk > 0) ? 1u : 0u);
-        __syncwarp();
+      issue_acc(tdK, tB, q_slot(n), n == 0, bar(Lay::B_QEMPTY + sl2));
+      if (n + 1 < nq) {
+        ok = wait_full(Lay::B_OFULL, n + 1);
+        if (!ok) break;
+        issue_score(tB, dV0, o_slot(n + 1), bar(Lay::B_DP));
       }
-      if (elect_one()) tc_commit(bar(Lay::B_EMPTY + st));
-      __syncwarp();
-      if (n + 1 < nq) issue_dpt(n + 1);
     }
     if (elect_one()) {
       if (ok) tc_commit(bar(Lay::B_ACC));
@@ -500,8 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------- dQ
-// CTA: query tile i of (b, h).  Resident: Q_i (A0), dO_i (A1).  Ring: (K_j, V_j).
-// Per key tile j:  S = Q_i K_j^T (TMEM A), dP = dO_i V_j^T (TMEM B);
+// CTA: query tile i of (b, h).  Resident: Q_i (A0), dO_i (A1).  Streamed: K_j, V_j.
+// Per key tile j:  S = Q_i K_j^T (TMEM A or A'), dP = dO_i V_j^T (TMEM B);
 //   P = exp2(scale*log2e*S - LSE2_row) (causal: zero where key > query);
 //   dS = P o (dP - D_row) -> B;  dQ += dS K_j.  dQ is scaled at the end.
 template <int D, int MASK>
@@ -509,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p) {
-  using Lay = BwdLayout<D>;
+  using Lay = DqLayout<D>;
   BwdItem it;
   constexpr bool CAUSAL = MASK == 1;
   if (!decode_block(p, false, CAUSAL, it)) return;  // uniform for the CTA
@@ -519,7 +595,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sb + Lay::BAR_OFF + 8 * i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t tmem = bwd_setup<D>(smem, sb, warp, 1);
+  const uint8_t counts[Lay::NBARS] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 8, 1, 1};
+  const uint32_t tmem = bwd_setup<Lay::NBARS>(smem, sb, Lay::BAR_OFF, Lay::MISC_OFF, warp, counts);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
   WaitCtl wc;
   wc.abort = reinterpret_cast<volatile uint32_t*>(misc + 1);
@@ -535,7 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     j_end = min(ntiles, ceil_div(i * kTile + kTile + p.wr, kTile));
   }
   const int nk = j_end - j_first;
-
+  auto k_slot = [&](int j) -> uint32_t { return sb + Lay::K_OFF + (j % Lay::NK) * Lay::TILE; };
+  auto v_slot = [&](int j) -> uint32_t { return sb + Lay::V_OFF + (j % Lay::NV) * Lay::TILE; };
   if (warp < 8) {
     const int hf = warp >> 2, wq = warp & 3;
     const int r = wq * 32 + lane;
@@ -599,9 +677,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const int64_t row = (static_cast<int64_t>(it.seq_start + q_row) * p.H + it.h) * D + (D / 2) * hf;
-      store_half_row<D>(tmem + lane_bits + Lay::TM_ACC0 + (D / 2) * hf, p.dq + row, p.scale, in);
+      store_half_row<D>(tmem + lane_bits + Lay::TM_DQ + (D / 2) * hf, p.dq + row, p.scale, in);
     }
   } else if (warp == 8) {
+    // ------------------------------------------------------------ producer
     const uint64_t pol_res = l2_policy_evict_first();
     const uint64_t pol_ring = l2_policy_evict_last();
     if (elect_one()) {
@@ -615,109 +694,118 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+    auto load = [&](uint32_t slot, uint32_t full, const CUtensorMap* tm, int j) {
+      if (elect_one()) {
+        mbar_arrive_expect_tx(full, Lay::TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(slot + c * Lay::CHUNK, tm, full, c * 64, it.h, it.seq_start + (j_first + j) * kTile,
+                      pol_ring);
+      }
+      __syncwarp();
+    };
     bool ok = true;
     for (int j = 0; j < nk && ok; ++j) {
-      const int st = j & 1;
-      if (j >= Lay::NSTAGE) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_EMPTY + st), ((j >> 1) - 1) & 1u, wc,
+      const int ks = j % Lay::NK, vs = j % Lay::NV;
+      if (j >= Lay::NK) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KEMPTY + ks), ((j / Lay::NK) - 1) & 1u, wc,
                                                timeout_code(kSiteStageEmpty)));
         if (!ok) break;
       }
-      if (elect_one()) {
-        mbar_arrive_expect_tx(bar(Lay::B_FULL + st), 2 * Lay::TILE);
-        const uint32_t base = sb + Lay::STAGE_OFF + st * 2 * Lay::TILE;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(base + c * Lay::CHUNK, &tm_k, bar(Lay::B_FULL + st), c * 64, it.h,
-                      it.seq_start + (j_first + j) * kTile, pol_ring);
-          tma_load_3d(base + Lay::TILE + c * Lay::CHUNK, &tm_v, bar(Lay::B_FULL + st), c * 64, it.h,
-                      it.seq_start + (j_first + j) * kTile, pol_ring);
-        }
+      load(k_slot(j), bar(Lay::B_KFULL + ks), &tm_k, j);
+      if (j >= Lay::NV) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_VEMPTY + vs), ((j / Lay::NV) - 1) & 1u, wc,
+                                               timeout_code(kSiteStageEmpty)));
+        if (!ok) break;
       }
-      __syncwarp();
+      load(v_slot(j), bar(Lay::B_VFULL + vs), &tm_v, j);
     }
     drain_wait(bar(Lay::B_RES), 0u, kDrainLimitNs);
-    for (int j = (nk > Lay::NSTAGE ? nk - Lay::NSTAGE : 0); j < nk; ++j)
-      drain_wait(bar(Lay::B_FULL + (j & 1)), (j >> 1) & 1u, kDrainLimitNs);
+    for (int j = (nk > Lay::NK ? nk - Lay::NK : 0); j < nk; ++j)
+      drain_wait(bar(Lay::B_KFULL + j % Lay::NK), (j / Lay::NK) & 1u, kDrainLimitNs);
+    for (int j = (nk > Lay::NV ? nk - Lay::NV : 0); j < nk; ++j)
+      drain_wait(bar(Lay::B_VFULL + j % Lay::NV), (j / Lay::NV) & 1u, kDrainLimitNs);
   } else {
+    // ---------------------------------------------------------------- MMA
     constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0, 0);
     constexpr uint32_t idesc_acc = idesc_bf16_f32(kTile, D, 0, 1);
-    const uint32_t tB = tmem + Lay::TM_B, tdQ = tmem + Lay::TM_ACC0;
+    const uint32_t tB = tmem + Lay::TM_B, tdQ = tmem + Lay::TM_DQ;
+    const uint64_t dQ0 = sdesc_sw128(sb + Lay::A0_OFF, 16, 1024), dO0 = sdesc_sw128(sb + Lay::A1_OFF, 16, 1024);
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_RES), 0, wc, timeout_code(kSiteKv)));
     uint32_t ds_phase = 0;
-    auto stage_k = [&](int j) -> uint32_t { return sb + Lay::STAGE_OFF + (j & 1) * 2 * Lay::TILE; };
-    // S = Q K_j^T into region A (j even) or A' (j odd).
-    auto issue_s = [&](int j) {
-      const uint32_t kb = stage_k(j);
-      const uint32_t tS = tmem + ((j & 1) ? Lay::TM_A2 : Lay::TM_A);
+    auto wait_k = [&](int j) -> bool {
+      const bool r = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KFULL + j % Lay::NK), (j / Lay::NK) & 1u,
+                                                       wc, timeout_code(kSiteStageFull)));
+      if (r) tc_fence_after();
+      return r;
+    };
+    auto wait_v = [&](int j) -> bool {
+      const bool r = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_VFULL + j % Lay::NV), (j / Lay::NV) & 1u,
+                                                       wc, timeout_code(kSiteStageFull)));
+      if (r) tc_fence_after();
+      return r;
+    };
+    // t = A (Q_i or dO_i) times the streamed tile's transpose, both K-major, issued
+    // back to back by one elected lane; commit to `done` (and `done2`, if given).
+    auto issue_score = [&](uint32_t t, uint64_t a0, uint32_t slot, uint32_t done, uint32_t done2) {
+      if (elect_one()) {
+        const uint64_t b0 = sdesc_sw128(slot, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-        if (elect_one())
-          mma_ss(tS, sdesc_sw128(sb + Lay::A0_OFF + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
-        __syncwarp();
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+          mma_ss(t, desc_add(a0, off), desc_add(b0, off), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(done);
+        if (done2 != 0u) tc_commit(done2);
       }
-      if (elect_one()) tc_commit(bar((j & 1) ? Lay::B_S1 : Lay::B_S));
       __syncwarp();
     };
-    // dP = dO V_j^T into region B, with its own commit.
+    // S = Q K_j^T into region A (j even) or A' (j odd).
+    auto issue_s = [&](int j) {
+      issue_score(tmem + ((j & 1) ? Lay::TM_A2 : Lay::TM_A), dQ0, k_slot(j), bar((j & 1) ? Lay::B_S1 : Lay::B_S),
+                  0u);
+    };
+    // dP = dO V_j^T into region B, with its own commit; V_j's slot is then free.
     auto issue_dp = [&](int j) {
-      const uint32_t vb = stage_k(j) + Lay::TILE;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-        if (elect_one())
-          mma_ss(tB, sdesc_sw128(sb + Lay::A1_OFF + off, 16, 1024), sdesc_sw128(vb + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
-        __syncwarp();
-      }
-      if (elect_one()) tc_commit(bar(Lay::B_DP));
-      __syncwarp();
+      issue_score(tB, dO0, v_slot(j), bar(Lay::B_DP), bar(Lay::B_VEMPTY + j % Lay::NV));
     };
     // Per key tile j the tensor pipe runs dQ(j), dP(j+1), S(j+2): S(j+1) is
     // already in the other score buffer, so the exponentials of tile j+1 start as
     // soon as dS(j) is released.  The elementwise warps read S(j) and dP(j) before
     // releasing dS(j), and one thread issues every MMA in order, so dP(j+1)
     // overwrites region B only after dQ(j) has read dS(j), and S(j+2) reuses S(j)'s
-    // buffer only after that release.
-    auto wait_full = [&](int j) -> bool {
-      const bool r = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_FULL + (j & 1)), (j >> 1) & 1u, wc,
-                                                       timeout_code(kSiteStageFull)));
-      if (r) tc_fence_after();
-      return r;
-    };
+    // buffer only after that release.  K_j's slot is released after dQ(j).
     if (ok && nk > 0) {
-      ok = wait_full(0);
-      if (ok) {
-        issue_s(0);
-        issue_dp(0);
-      }
+      ok = wait_k(0);
+      if (ok) issue_s(0);
+      if (ok) ok = wait_v(0);
+      if (ok) issue_dp(0);
       if (ok && nk > 1) {
-        ok = wait_full(1);
+        ok = wait_k(1);
         if (ok) issue_s(1);
       }
     }
     for (int j = 0; j < nk && ok; ++j) {
-      const int st = j & 1;
-      const uint32_t kb = stage_k(j);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DS), ds_phase, wc, timeout_code(kSiteDs)));
       if (!ok) break;
       ds_phase ^= 1u;
       tc_fence_after();
       // dQ += dS K (A = dS from TMEM, B = K MN-major).
+      if (elect_one()) {
+        const uint64_t b0 = sdesc_sw128(k_slot(j), Lay::CHUNK, 1024);
 #pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk) {
-        if (elect_one())
-          mma_ts(tdQ, tB + packed_col(kk), sdesc_sw128(kb + kk * 2048, Lay::CHUNK, 1024), idesc_acc,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        __syncwarp();
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tdQ, tB + packed_col(kk), desc_add(b0, kk * 2048), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(Lay::B_KEMPTY + j % Lay::NK));
       }
-      if (elect_one()) tc_commit(bar(Lay::B_EMPTY + st));
       __syncwarp();
-      if (j + 1 < nk) issue_dp(j + 1);  // stage (j+1) was waited for before S(j+1)
+      if (j + 1 < nk) {
+        ok = wait_v(j + 1);
+        if (!ok) break;
+        issue_dp(j + 1);
+      }
       if (j + 2 < nk) {
-        ok = wait_full(j + 2);
+        ok = wait_k(j + 2);
         if (!ok) break;
         issue_s(j + 2);
       }
@@ -738,16 +826,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, int MASK>
 cudaError_t launch_main(const BwdLaunch& a, cudaStream_t st) {
-  const int smem = 1024 + BwdLayout<D>::SMEM;
+  const int smem1 = 1024 + DkdvLayout<D>::SMEM;
+  const int smem2 = 1024 + DqLayout<D>::SMEM;
   auto k1 = bwd_dkdv_kernel<D, MASK>;
   auto k2 = bwd_dq_kernel<D, MASK>;
-  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
   if (e != cudaSuccess) return e;
-  k1<<<a.grid, kThreads, smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.p);
+  k1<<<a.grid, kThreads, smem1, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k2<<<a.grid, kThreads, smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.p);
+  k2<<<a.grid, kThreads, smem2, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.p);
   return cudaGetLastError();
 }
 
