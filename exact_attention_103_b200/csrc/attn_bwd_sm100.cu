@@ -39,6 +39,7 @@
 
 #include "attn_bwd_sm100.h"
 #include "sm100_ptx.cuh"
+#include "softmax_math.cuh"
 
 namespace attn {
 
@@ -142,6 +143,29 @@ __device__ __forceinline__ uint2 neg_split3(float x) {
 }
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Pairs of exponentials (of every 8) computed on the FMA pipe by exp2_poly_x2
+// instead of MUFU ex2 (the exponential split of the forward kernel).
+#ifndef ATTN_BWD_POLY8
+#define ATTN_BWD_POLY8 0
+#endif
+constexpr int kBwdPoly8 = ATTN_BWD_POLY8;
+static_assert(kBwdPoly8 >= 0 && kBwdPoly8 <= 8, "pairs per 8");
+
+// y <- 2^y for 64 log2-domain arguments, two at a time.  MUFU ex2 gives 0 for
+// y = -inf; the polynomial clamps at 2^-125 (used only where such rows are masked
+// or never stored).
+__device__ __forceinline__ void exp2_cols(float (&y)[64]) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    if (((c >> 1) & 7) >= 8 - kBwdPoly8) {
+      exp2_poly_x2(y[c], y[c + 1]);
+    } else {
+      y[c] = fast_exp2(y[c]);
+      y[c + 1] = fast_exp2(y[c + 1]);
+    }
+  }
+}
 
 __device__ __forceinline__ int64_t vec_index(const BwdParams& p, int b, int h, int seq_start,
                                              int row) {
@@ -373,9 +397,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float pv[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float e = fast_exp2(__uint_as_float(sv[c]) * sl);
-        pv[c] = (c < lim || (MASK == 2 && c > lim_hi)) ? 0.f : e;
+      for (int c = 0; c < 64; c += 2)
+        fmul2_bc(pv[c], pv[c + 1], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl);
+      exp2_cols(pv);
+      // Only the diagonal tile (causal) and the window's edge tiles mask columns.
+      if (__any_sync(0xffffffffu, lim > 0 || (MASK == 2 && lim_hi < 63))) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c < lim || (MASK == 2 && c > lim_hi)) pv[c] = 0.f;
       }
       uint32_t pk[32];
 #pragma unroll
@@ -386,16 +415,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       dp_phase ^= 1u;
       tc_fence_after();
-      // dS^T = P^T o (dP^T - D), in two 32-column halves to bound registers.
+      // dS^T = P^T o (dP^T - D) (the subtraction done by the tensor core).
+      {
+        uint32_t dv[64];
+        tmem_ld_x64(tB, dv);
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
-        uint32_t dv[32];
-        tmem_ld_x32(tB + 32 * q2, dv);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int c0 = 32 * q2 + 2 * c;
-          pk[16 * q2 + c] = pack_bf16x2(pv[c0] * __uint_as_float(dv[2 * c]),
-                                        pv[c0 + 1] * __uint_as_float(dv[2 * c + 1]));
+        for (int c = 0; c < 32; ++c) {
+          float d0, d1;
+          ffma2_vb(d0, d1, __uint_as_float(dv[2 * c]), __uint_as_float(dv[2 * c + 1]), pv[2 * c],
+                   pv[2 * c + 1], 0.f);
+          pk[c] = pack_bf16x2(d0, d1);
         }
       }
       tmem_st_x32(tB, pk);
@@ -650,24 +679,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float pv[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float e = fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lse2));
-        pv[c] = (c < lim && (MASK != 2 || c >= lim_lo)) ? e : 0.f;
+      for (int c = 0; c < 64; c += 2)
+        ffma2_bc(pv[c], pv[c + 1], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl, -lse2);
+      exp2_cols(pv);
+      if (__any_sync(0xffffffffu, lim < 64 || (MASK == 2 && lim_lo > 0))) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (!(c < lim && (MASK != 2 || c >= lim_lo))) pv[c] = 0.f;
       }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DP), dp_phase, wc, timeout_code(kSiteS)));
       if (!ok) break;
       dp_phase ^= 1u;
       tc_fence_after();
       uint32_t pk[32];
+      {
+        uint32_t dv[64];
+        tmem_ld_x64(tB, dv);
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
-        uint32_t dv[32];
-        tmem_ld_x32(tB + 32 * q2, dv);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int c0 = 32 * q2 + 2 * c;
-          pk[16 * q2 + c] = pack_bf16x2(pv[c0] * (__uint_as_float(dv[2 * c]) - dd),
-                                        pv[c0 + 1] * (__uint_as_float(dv[2 * c + 1]) - dd));
+        for (int c = 0; c < 32; ++c) {
+          float d0, d1;
+          fsub2_bc(d0, d1, __uint_as_float(dv[2 * c]), __uint_as_float(dv[2 * c + 1]), dd);
+          ffma2_vb(d0, d1, d0, d1, pv[2 * c], pv[2 * c + 1], 0.f);
+          pk[c] = pack_bf16x2(d0, d1);
         }
       }
       tmem_st_x32(tB, pk);
