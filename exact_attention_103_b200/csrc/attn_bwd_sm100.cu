@@ -178,9 +178,16 @@ __device__ __forceinline__ int64_t vec_index(const BwdParams& p, int b, int h, i
 // the K-step kk of an MMA that reads them as its A operand starts here:
 __device__ __forceinline__ uint32_t packed_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
 
-// Block -> (sequence, head, tile) in longest-first order: for the key-tile
-// kernel (causal) small tile indices have the most query tiles; for the
-// query-tile kernel large indices have the most key tiles.
+// Block -> (sequence, head, tile).  Blocks are dealt in groups of kBwdGroup
+// (sequence, head) pairs, longest-first inside each group (for the key-tile kernel
+// (causal) small tile indices have the most query tiles; for the query-tile
+// kernel large indices have the most key tiles).  The CTAs running at any time
+// then belong to a few heads, whose streamed tiles (4 MB per head at N = 8192,
+// d = 128) stay in L2 while every CTA of the group reads them.
+#ifndef ATTN_BWD_GROUP
+#define ATTN_BWD_GROUP 8
+#endif
+constexpr int kBwdGroup = ATTN_BWD_GROUP;
 struct BwdItem {
   int b, h, tile, seq_start, L;
 };
@@ -192,8 +199,12 @@ struct BwdItem {
 __device__ __forceinline__ bool decode_block(const BwdParams& p, bool key_tiles, bool causal,
                                              BwdItem& it) {
   const int nbh = p.B * p.H;
-  const int idx = blockIdx.x;
-  const int rank = idx / nbh, bh = idx - rank * nbh;
+  const int idx = static_cast<int>(blockIdx.x);
+  const int G = nbh < kBwdGroup ? nbh : kBwdGroup;
+  const int grp = idx / (G * p.ntiles);
+  const int gsize = min(G, nbh - grp * G);  // the last group may be smaller
+  const int rem = idx - grp * G * p.ntiles;
+  const int rank = rem / gsize, bh = grp * G + (rem - rank * gsize);
   it.b = bh / p.H;
   it.h = bh - it.b * p.H;
   it.tile = (causal && !key_tiles) ? p.ntiles - 1 - rank : rank;

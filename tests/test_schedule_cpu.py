@@ -247,3 +247,34 @@ def test_pair_lists_cover_every_block_once(grid):
     for _ in range(20):
         lengths = [rng.randint(0, 3000) for _ in range(rng.choice([1, 4, 30]))]
         _coverage(Sched(len(lengths), 3, max(max(lengths), 1), grid, cu=_cu(lengths), pair=True), lengths)
+
+
+def bwd_decode(idx, nbh, ntiles, group):
+    """Twin of the backward's block order (decode_block in csrc/attn_bwd_sm100.cu):
+    blocks dealt in groups of `group` (sequence, head) pairs, by rank inside a group.
+    Returns (bh, rank)."""
+    G = min(nbh, group)
+    grp = idx // (G * ntiles)
+    gsize = min(G, nbh - grp * G)
+    rem = idx - grp * G * ntiles
+    rank = rem // gsize
+    return grp * G + (rem - rank * gsize), rank
+
+
+@pytest.mark.parametrize("nbh,ntiles", [(32, 64), (1, 1), (3, 5), (17, 9), (8, 64), (40, 3)])
+@pytest.mark.parametrize("group", [1, 4, 8, 16, 64])
+def test_bwd_block_order_is_a_bijection(nbh, ntiles, group):
+    """Every (sequence-head pair, tile rank) is dealt to exactly one block of the
+    nbh * ntiles grid; inside a group ranks do not decrease (longest work first);
+    the blocks running together span at most `group` pairs per rank sweep."""
+    seen = {}
+    prev = None
+    for idx in range(nbh * ntiles):
+        bh, rank = bwd_decode(idx, nbh, ntiles, group)
+        assert 0 <= bh < nbh and 0 <= rank < ntiles
+        seen[(bh, rank)] = seen.get((bh, rank), 0) + 1
+        grp = bh // min(nbh, group)
+        if prev is not None and prev[0] == grp:
+            assert rank >= prev[1]
+        prev = (grp, rank)
+    assert len(seen) == nbh * ntiles and all(v == 1 for v in seen.values())
