@@ -117,9 +117,6 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_plain(uint32_t saddr, uint32_t 
   d |= 1ull << 46;  // descriptor version of this architecture; layout type 0 = no swizzle
   return d;
 }
-// A descriptor advanced by `bytes` within the same operand (adds to the start
-// address field; shared-memory addresses stay below 2^18, so nothing carries out).
-__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 // Byte offset of row r's first core-matrix row in a 128 x 16 operand of that layout
 // (lbo = 128, sbo = 256).
 __device__ __forceinline__ uint32_t xtra_row_off(int r) { return (r & 7) * 16 + (r >> 3) * 256; }

@@ -940,18 +940,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                            timeout_code(kSitePFull)));
               if (!ok) break;
               tc_fence_after();
+              // The part's K steps are issued back to back by one elected lane.
+              if (elect_one()) {
+                // V (a pair: this CTA's 64 head-dim columns of it) is MN-major.
+                const uint64_t dv0 = sdesc_sw128(vbase, Lay::CHUNK, 1024);
 #pragma unroll
-              for (int kk = half * NK / kPSplit; kk < (half + 1) * NK / kPSplit; ++kk) {
-                if (elect_one()) {
-                  // V (a pair: this CTA's 64 head-dim columns of it) is MN-major.
-                  const uint64_t dv = sdesc_sw128(vbase + kk * Lay::KSTEP * 128, Lay::CHUNK, 1024);
+                for (int kk = half * NK / kPSplit; kk < (half + 1) * NK / kPSplit; ++kk) {
+                  const uint64_t dv = desc_add(dv0, kk * Lay::KSTEP * 128);
                   const uint32_t acc = (j - 1 > los || kk > 0) ? 1u : 0u;
                   if constexpr (PAIR) mma_ts_pair(tO, tS + kk * 8, dv, idesc_o, acc);
                   else if constexpr (F8) mma_ts_f8(tO, tS + kk * 8, dv, idesc_o, acc);
                   else mma_ts(tO, tS + kk * 8, dv, idesc_o, acc);
                 }
-                __syncwarp();
               }
+              __syncwarp();
             }
             if (ok) {
               ph ^= 1u;
@@ -966,20 +968,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t kbase = sb + Lay::KV_OFF + slotK * Lay::SLOT;
             // K's rows (a pair: this CTA's 64 keys) in 128-byte chunks of head dims.
             constexpr int KCHUNK = PAIR ? Lay::SLOT / 2 : Lay::CHUNK;
+            if (elect_one()) {
+              const uint64_t da0 = sdesc_sw128(qbase, 16, 1024);
+              const uint64_t db0 = sdesc_sw128(kbase, 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < D / Lay::KSTEP; ++kk) {
-              const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-              const uint32_t offk = (kk >> 2) * KCHUNK + (kk & 3) * 32;
-              if (elect_one()) {
-                const uint64_t da = sdesc_sw128(qbase + off, 16, 1024);
-                const uint64_t db = sdesc_sw128(kbase + offk, 16, 1024);
+              for (int kk = 0; kk < D / Lay::KSTEP; ++kk) {
+                const uint64_t da = desc_add(da0, (kk >> 2) * Lay::CHUNK + (kk & 3) * 32);
+                const uint64_t db = desc_add(db0, (kk >> 2) * KCHUNK + (kk & 3) * 32);
                 if constexpr (PAIR) mma_ss_pair(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
                 else if constexpr (F8) mma_ss_f8(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
                 else mma_ss(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
               }
-              __syncwarp();
+              commit(Lay::B_SFULL + s);
             }
-            if (elect_one()) commit(Lay::B_SFULL + s);
             __syncwarp();
           }
         }

@@ -249,6 +249,10 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// A descriptor advanced by `bytes` within the same operand (adds to the start
+// address field; shared-memory addresses stay below 2^18, so nothing carries out).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 // Instruction descriptor for kind::f16 with bf16 A/B and an fp32 accumulator.
 // a_mn / b_mn select MN-major (1) instead of K-major (0) operands.
 // Instruction descriptor of kind::f8f6f4 with E4M3 A and B (format code 0) and an
