@@ -69,10 +69,12 @@ struct DkdvLayout {
   static constexpr int Q_OFF = ONES_OFF + XTRA;
   static constexpr int DO_OFF = Q_OFF + NSLOT * SLOT;
   static constexpr int BAR_OFF = DO_OFF + NSLOT * SLOT;
-  // B_S: S^T in TMEM region A; B_DP: dP^T in region B; B_P / B_DS: P^T / dS^T
-  // written back by the eight elementwise warps.
-  static constexpr int B_RES = 0, B_QFULL = 1, B_QEMPTY = 3, B_OFULL = 5, B_OEMPTY = 7, B_S = 9,
-                       B_DP = 10, B_P = 11, B_DS = 12, B_ACC = 13, B_DRAIN = 14, NBARS = 15;
+  // B_S0 / B_S1: query columns 0-63 / 64-127 of S^T in TMEM region A; B_DP: dP^T in
+  // region B; B_P0 / B_P1: P^T of those columns written back by the four warps that
+  // own them; B_DS: dS^T written back by all eight.
+  static constexpr int B_RES = 0, B_QFULL = 1, B_QEMPTY = 3, B_OFULL = 5, B_OEMPTY = 7, B_S0 = 9,
+                       B_S1 = 10, B_DP = 11, B_P0 = 12, B_P1 = 13, B_DS = 14, B_ACC = 15, B_DRAIN = 16,
+                       NBARS = 17;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM = MISC_OFF + 64;
   // TMEM columns: region A (S^T, then packed P^T), region B (dP^T, then packed
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
   }
-  const uint8_t counts[Lay::NBARS] = {1, 2, 2, 1, 1, 2, 2, 1, 1, 1, 1, 8, 8, 1, 1};
+  const uint8_t counts[Lay::NBARS] = {1, 2, 2, 1, 1, 2, 2, 1, 1, 1, 1, 1, 4, 4, 8, 1, 1};
   const uint32_t tmem = bwd_setup<Lay::NBARS>(smem, sb, Lay::BAR_OFF, Lay::MISC_OFF, warp, counts);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::MISC_OFF);
   WaitCtl wc;
@@ -387,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int n = 0; n < nq && ok; ++n) {
       const int i = i_first + n;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_S), s_phase, wc, timeout_code(kSiteS)));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_S0 + hf), s_phase, wc, timeout_code(kSiteS)));
       if (!ok) break;
       s_phase ^= 1u;
       tc_fence_after();
@@ -418,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
       tmem_st_x32(tA, pk);
-      warp_release(bar(Lay::B_P), lane);
+      warp_release(bar(Lay::B_P0 + hf), lane);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DP), dp_phase, wc, timeout_code(kSiteS)));
       if (!ok) break;
       dp_phase ^= 1u;
@@ -520,6 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Each product's K-steps are issued back to back by one elected lane, with
     // descriptors built once and advanced by compile-time offsets.
     constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0, 0);
+    constexpr uint32_t idesc_h = idesc_bf16_f32(kTile, kTile / 2, 0, 0);
     constexpr uint32_t idesc_acc = idesc_bf16_f32(kTile, D, 0, 1);
     const uint32_t tA = tmem + Lay::TM_A, tB = tmem + Lay::TM_B;
     const uint32_t tdV = tmem + Lay::TM_DV, tdK = tmem + Lay::TM_DK;
@@ -548,6 +551,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
+    // S^T for query columns 64h..64h+63 only (N = 64): rows 64h.. of the Q slot and
+    // of its extra-step operand, into TMEM columns 64h..; commit to B_S0 + h.
+    auto issue_st_half = [&](int h, uint32_t slot) {
+      if (elect_one()) {
+        const uint64_t b0 = sdesc_sw128(slot + h * 64 * 128, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+          mma_ss(tA + 64 * h, desc_add(dK0, off), desc_add(b0, off), idesc_h, kk > 0 ? 1u : 0u);
+        }
+        mma_ss(tA + 64 * h, ones, sdesc_kmajor_plain(slot + Lay::TILE + h * 8 * 256, 128, 256), idesc_h, 1u);
+        tc_commit(bar(Lay::B_S0 + h));
+      }
+      __syncwarp();
+    };
+    // dV += the P^T columns of half h (K steps 4h..4h+3) times dO (MN-major).
+    auto issue_dv_half = [&](int h, uint32_t slot, bool first) {
+      if (elect_one()) {
+        const uint64_t b0 = sdesc_sw128(slot, Lay::CHUNK, 1024);
+#pragma unroll
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+          mma_ts(tdV, tA + packed_col(kk), desc_add(b0, kk * 2048), idesc_acc, (!first || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+    };
     // acc += (packed bf16 from TMEM region ta) times the streamed tile (MN-major);
     // commit to `done` (the tile's slot is then free).
     auto issue_acc = [&](uint32_t acc, uint32_t ta, uint32_t slot, bool first, uint32_t done) {
@@ -563,28 +591,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Software pipeline over query tiles: per tile n the tensor pipe runs
     //   dV(n), S^T(n+1), dK(n), dP^T(n+1)
     // so the elementwise work on tile n+1 (exponentials) overlaps dK(n) and
-    // dP^T(n+1), and dS of tile n overlaps dV(n) and S^T(n+1).  Region A is
+    // dP^T(n+1), and dS of tile n overlaps dV(n) and S^T(n+1).  dV and S^T are
+    // issued in two halves of 64 query columns, each half as soon as the four warps
+    // that own those columns release them, so half the exponentials of tile n+1
+    // start while the other half of S^T(n+1) is still being computed.  Region A is
     // rewritten by S^T(n+1) only after dV(n) has read P^T(n) (one issuing thread:
     // in order), region B by dP^T(n+1) only after dK(n) has read dS^T(n).  dO(n)'s
     // slot is released after dV(n), Q(n)'s after dK(n).
     if (ok && nq > 0) {
       ok = wait_full(Lay::B_QFULL, 0);
-      if (ok) issue_score(tA, dK0, q_slot(0), bar(Lay::B_S));
+      if (ok) {
+        issue_st_half(0, q_slot(0));
+        issue_st_half(1, q_slot(0));
+      }
       if (ok) ok = wait_full(Lay::B_OFULL, 0);
       if (ok) issue_score(tB, dV0, o_slot(0), bar(Lay::B_DP));
     }
     for (int n = 0; n < nq && ok; ++n) {
       const int sl2 = n & 1;
-      // dV += P^T dO (A = P^T from TMEM, B = dO MN-major).
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_P), p_phase, wc, timeout_code(kSiteP)));
+      // dV += P^T dO (A = P^T from TMEM, B = dO MN-major), half by half.
+#pragma unroll
+      for (int h = 0; h < 2 && ok; ++h) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_P0 + h), p_phase, wc, timeout_code(kSiteP)));
+        if (!ok) break;
+        tc_fence_after();
+        issue_dv_half(h, o_slot(n), n == 0);
+      }
       if (!ok) break;
       p_phase ^= 1u;
-      tc_fence_after();
-      issue_acc(tdV, tA, o_slot(n), n == 0, bar(Lay::B_OEMPTY + sl2));
+      if (elect_one()) tc_commit(bar(Lay::B_OEMPTY + sl2));
+      __syncwarp();
       if (n + 1 < nq) {
         ok = wait_full(Lay::B_QFULL, n + 1);
         if (!ok) break;
-        issue_score(tA, dK0, q_slot(n + 1), bar(Lay::B_S));
+        issue_st_half(0, q_slot(n + 1));
+        issue_st_half(1, q_slot(n + 1));
       }
       // dK += dS^T Q (A = dS^T from TMEM, B = Q MN-major); scale applied at the end.
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_DS), ds_phase, wc, timeout_code(kSiteDs)));
