@@ -149,6 +149,19 @@ bool make_map_rows64(CUtensorMap* m, const void* ptr, int64_t total, int H, int 
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The bf16 output O as {d, H, total} with box {64, 1, 32} (one softmax warp's 32
+// rows, 64 head dims; 128-byte swizzle): the TMA stores of the forward's epilogue.
+bool make_map_o(CUtensorMap* m, void* ptr, int64_t total, int H, int d) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(total)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
+  const cuuint32_t box[3] = {64, 1, 32};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
@@ -283,8 +296,9 @@ attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total
   const int esz = f8 ? 1 : 2;
   if (!make_map_esz(&a->tm_q, c.q, total, c.H, c.d, esz) || !make_map_esz(&a->tm_k, c.k, total, c.H, c.d, esz) ||
       !make_map_esz(&a->tm_v, c.v, total, c.H, c.d, esz) ||
-      (pl.pair && !make_map_rows64(&a->tm_k2, c.k, total, c.H, c.d)))
-    return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled rejected the Q/K/V views");
+      (pl.pair && !make_map_rows64(&a->tm_k2, c.k, total, c.H, c.d)) ||
+      !make_map_o(&a->tm_o, c.o, total, c.H, c.d))
+    return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled rejected the Q/K/V/O views");
   a->pair = pl.pair;
   const bool varlen = c.cu_seqlens != nullptr;
   a->p.o = static_cast<__nv_bfloat16*>(c.o);
@@ -312,6 +326,10 @@ attn_status_t fill_fwd_launch(const FwdCall& c, const FwdPlan& pl, int64_t total
   // Dense unmasked launches may split their last wave into half items (see the
   // kernel), so up to twice as many CTAs can be useful there.
   a->smem = attn::fwd_smem_bytes(c.d, c.B, static_cast<int>(pl.T), varlen ? 1 : 0, f8 ? 1 : 0, pl.pair);
+  // O leaves through shared-memory staging and TMA stores where the staging
+  // buffers fit beside the rest (not beside the work tables of very many sequences).
+  a->p.stage_off = attn::fwd_stage_offset(c.d, c.B, static_cast<int>(pl.T), varlen ? 1 : 0, f8 ? 1 : 0, pl.pair);
+  if (a->p.stage_off != 0) a->smem = 1024 + a->p.stage_off + attn::kFwdStageBytes;
   if (pl.pair) {
     // Two CTAs per item; as many clusters as fit at once (SMs left over in a GPC
     // of odd SM count cannot hold a cluster).

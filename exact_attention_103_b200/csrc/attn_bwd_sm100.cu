@@ -123,11 +123,6 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_plain(uint32_t saddr, uint32_t 
 // (lbo = 128, sbo = 256).
 __device__ __forceinline__ uint32_t xtra_row_off(int r) { return (r & 7) * 16 + (r >> 3) * 256; }
 
-// Orders this thread's generic-proxy shared-memory writes before later reads by
-// the tensor core (async proxy).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // -x as three bf16 terms whose sum is -x to ~2^-24 relative (x = +inf: -inf, 0, 0),
 // packed as the first four bf16 of an extra-step row: {t0, t1, t2, 0}.

@@ -418,7 +418,7 @@ template <int D, int MASK, int POLY, bool F8, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k2,
-               const FwdParams p) {
+               const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
   using Lay = Layout<D, F8, PAIR>;
   static_assert(!F8 || D == 128, "E4M3 path: one 128-byte row per head");
   static_assert(!PAIR || (D == 128 && !F8), "CTA pairs: bf16, d = 128");
@@ -732,6 +732,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ov[D];
       if constexpr (D == 128) tmem_ld_x128(t_o, ov);
       else tmem_ld_x64(t_o, ov);
+      // Asynchronous write-back: when all 32 rows of this warp lie inside the
+      // sequence, the warp writes them, 64 head dims at a time, into its staging
+      // buffer (the 128-byte-swizzled layout of a {64, 1, 32} box) and one lane
+      // hands each half to a TMA store; the warp goes on without waiting for the
+      // global writes.  Warps whose rows cross the sequence end store directly.
+      const bool staged = p.stage_off != 0 && __all_sync(0xffffffffu, store);
+      uint8_t* stg = smem + p.stage_off + warp * 4096;
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
         uint32_t w[4];
@@ -741,7 +748,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           fmul2_bc(x0, x1, __uint_as_float(ov[8 * c + 2 * i]), __uint_as_float(ov[8 * c + 2 * i + 1]), inv);
           w[i] = pack_bf16x2(x0, x1);
         }
-        if (store) reinterpret_cast<uint4*>(dst)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        if (staged) {
+          if ((c & 7) == 0) {
+            // the previous store from this buffer has finished reading it
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+          }
+          *reinterpret_cast<uint4*>(stg + lane * 128 + (((c & 7) ^ (lane & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+          if ((c & 7) == 7) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tm_o, smem_u32(stg), (c >> 3) * 64, h, seq_start + row0 + wq * 32);
+              bulk_commit_group();
+            }
+          }
+        } else if (store) {
+          reinterpret_cast<uint4*>(dst)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
       }
       if (store) {
         float lse2 = m_ref + __log2f(l);
@@ -755,6 +780,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.lse[li] = lse;
       }
     }
+    // Every TMA store of this warp has completed before the CTA exits.
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
     if (p.stats) {
       atomicAdd(p.stats, static_cast<unsigned long long>(n_rescale));
       atomicAdd(p.stats + 1, static_cast<unsigned long long>(n_rowtiles));
@@ -1041,6 +1069,12 @@ int fwd_smem_bytes(int D, int B, int T, int varlen, int fp8, int pair) {
   return fixed + (varlen ? varlen_table_ints(B, T) * 4 : 0);
 }
 
+int fwd_stage_offset(int D, int B, int T, int varlen, int fp8, int pair) {
+  const int end = fwd_smem_bytes(D, B, T, varlen, fp8, pair) - 1024;  // from the aligned base
+  const int off = (end + 1023) & ~1023;
+  return (1024 + off + kFwdStageBytes <= 232448) ? off : 0;
+}
+
 template <int D, int MASK, int POLY, bool F8 = false, bool PAIR = false>
 static cudaError_t launch_t(const FwdLaunch& a, cudaStream_t st) {
   auto kern = fwd_kernel<D, MASK, POLY, F8, PAIR>;
@@ -1059,10 +1093,10 @@ static cudaError_t launch_t(const FwdLaunch& a, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, a.tm_q, a.tm_k, a.tm_v, a.tm_k2, a.p);
+    e = cudaLaunchKernelEx(&cfg, kern, a.tm_q, a.tm_k, a.tm_v, a.tm_k2, a.tm_o, a.p);
     if (e != cudaSuccess) return e;
   } else {
-    kern<<<a.grid, kThreads, a.smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_k2, a.p);
+    kern<<<a.grid, kThreads, a.smem, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_k2, a.tm_o, a.p);
   }
   return cudaGetLastError();
 }

@@ -35,13 +35,17 @@ struct FwdParams {
   float o_scale;         // E4M3 path: V's per-tensor scale, applied with 1/l
   float p_shift;         // E4M3 path: P~ carries a factor 2^p_shift (an integer) so
                          // it spans E4M3's normal range; l carries it too
+  int stage_off;         // > 0: byte offset (from the 1024-aligned shared-memory base) of
+                         // the O staging buffers (4 KB per softmax warp) that TMA stores
+                         // write back from; 0: O rows are stored directly
 };
 
 struct FwdLaunch {
   // 3-D maps {D, H, total} with 128-byte swizzle; box {64, 1, 128} for bf16 and
   // {128, 1, 128} for E4M3 (one 128-byte row either way); tm_k2: K with box
-  // {64, 1, 64} (the K halves of CTA pairs; unused otherwise)
-  CUtensorMap tm_q, tm_k, tm_v, tm_k2;
+  // {64, 1, 64} (the K halves of CTA pairs; unused otherwise); tm_o: O (bf16) with
+  // box {64, 1, 32} (one softmax warp's 32 rows, 64 head dims)
+  CUtensorMap tm_q, tm_k, tm_v, tm_k2, tm_o;
   FwdParams p;
   int grid;
   int smem;
@@ -50,6 +54,10 @@ struct FwdLaunch {
 
 // T: items of the longest sequence (256 query rows each; CTA pairs: 512).
 int fwd_smem_bytes(int D, int B, int T, int varlen, int fp8, int pair);
+// Offset of the O staging buffers for that launch (0: they do not fit beside the
+// kernel's other shared memory) and their size.
+int fwd_stage_offset(int D, int B, int T, int varlen, int fp8, int pair);
+constexpr int kFwdStageBytes = 8 * 4096;
 // Clusters of two CTAs of the pair kernel that fit on the device at once (0: none).
 int fwd_pair_max_clusters(int smem);
 // poly: exponentials per 8 column pairs on the FMA-pipe polynomial (0, 2 or 8).
