@@ -278,27 +278,40 @@ __device__ __forceinline__ void warp_release(uint32_t bar, int lane) {
 }
 
 // ---------------------------------------------------------------------- D_i
-__global__ void bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
-                               const __nv_bfloat16* __restrict__ dout, BwdParams p, int d) {
+// D_i = <dO_i, O_i> for every (token, head) row: HBM-bound (two bf16 rows read per
+// float written).  A row is read by D/8 lanes with 16-byte loads and reduced by
+// shuffles within those lanes; the grid strides over rows.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                      const __nv_bfloat16* __restrict__ dout, BwdParams p) {
+  constexpr int LPR = D / 8;        // lanes per row
+  constexpr int RPW = 32 / LPR;     // rows per warp and step
   const int lane = threadIdx.x & 31;
+  const int sub = lane % LPR;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t units = static_cast<int64_t>(p.total) * p.H;
-  for (int64_t u = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       u < units; u += warps) {
-    const int64_t tok = u / p.H;
-    const int h = static_cast<int>(u - tok * p.H);
-    const __nv_bfloat16* orow = o + u * d;
-    const __nv_bfloat16* drow = dout + u * d;
+  // The loop bound is uniform across the warp (every lane joins the shuffles).
+  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW;
+       base < units; base += warps * RPW) {
+    const int64_t u = base + lane / LPR;
+    const bool valid = u < units;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    const uint4 a = valid ? __ldg(reinterpret_cast<const uint4*>(o + u * D) + sub) : zero;
+    const uint4 g = valid ? __ldg(reinterpret_cast<const uint4*>(dout + u * D) + sub) : zero;
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
     float acc = 0.f;
-    for (int c = lane * 2; c < d; c += 64) {
-      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(orow + c);
-      const __nv_bfloat162 g = *reinterpret_cast<const __nv_bfloat162*>(drow + c);
-      acc = fmaf(__bfloat162float(a.x), __bfloat162float(g.x), acc);
-      acc = fmaf(__bfloat162float(a.y), __bfloat162float(g.y), acc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 af = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[i]));
+      const float2 gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[i]));
+      acc = fmaf(af.x, gf.x, acc);
+      acc = fmaf(af.y, gf.y, acc);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (valid && sub == 0) {
+      const int64_t tok = u / p.H;
+      const int h = static_cast<int>(u - tok * p.H);
       int64_t idx;
       if (p.cu_seqlens == nullptr) {
         const int b = static_cast<int>(tok / p.N);
@@ -922,11 +935,16 @@ cudaError_t launch_main(const BwdLaunch& a, cudaStream_t st) {
 cudaError_t launch_bwd(const BwdLaunch& a, const void* o, const void* dout, int D, int mask,
                        cudaStream_t st) {
   const int64_t units = static_cast<int64_t>(a.p.total) * a.p.H;
-  int blocks = static_cast<int>((units + 7) / 8);
-  if (blocks > 148 * 16) blocks = 148 * 16;
+  const int rows_per_block = 256 / (D / 8);  // 256 threads, D/8 lanes per row
+  int64_t blocks = (units + rows_per_block - 1) / rows_per_block;
+  if (blocks > 148 * 8) blocks = 148 * 8;  // 8 blocks of 256 threads per SM, grid-stride beyond
   if (blocks < 1) blocks = 1;
-  bwd_pre_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
-                                          static_cast<const __nv_bfloat16*>(dout), a.p, D);
+  if (D == 128)
+    bwd_pre_kernel<128><<<static_cast<int>(blocks), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
+                                                                  static_cast<const __nv_bfloat16*>(dout), a.p);
+  else
+    bwd_pre_kernel<64><<<static_cast<int>(blocks), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
+                                                                 static_cast<const __nv_bfloat16*>(dout), a.p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (D == 128) {
