@@ -69,6 +69,10 @@ constexpr float kLn2 = 0.693147180559945309f;
 #define ATTN_P_SPLIT 2
 #endif
 constexpr int kPSplit = ATTN_P_SPLIT;
+#ifndef ATTN_EARLY_PAIRS
+#define ATTN_EARLY_PAIRS 8
+#endif
+constexpr int kEarlyPairs = ATTN_EARLY_PAIRS;
 static_assert(kPSplit == 1 || kPSplit == 2 || kPSplit == 4, "P~ split");
 
 // Error codes recorded in the device error word: 4 (= ATTN_ERR_TIMEOUT) in the
@@ -645,6 +649,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         float nm = (MASK == kMaskWindow && m_ref == -INFINITY) ? 0.f : -m_ref;
         if constexpr (F8) nm += p.p_shift;  // P~ * 2^p_shift <= 256 stays in E4M3's range
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (!F8 && kPSplit == 2 && kEarlyPairs > 0) {
+          // bf16, two parts: the first pairs of the second part are computed before
+          // waiting for the first part's TMEM store, so that wait returns at once.
+          auto pair_bf16 = [&](int c) -> uint32_t {  // column pair c (keys 2c, 2c+1)
+            const uint32_t x0 = c < 32 ? sa[2 * c] : sz[2 * c - 64];
+            const uint32_t x1 = c < 32 ? sa[2 * c + 1] : sz[2 * c - 63];
+            float a, e;
+            ffma2_bc(a, e, __uint_as_float(x0), __uint_as_float(x1), sl, nm);
+            if ((c & 7) >= 8 - POLY) {
+              exp2_poly_x2(a, e);
+            } else {
+              a = fast_exp2(a);
+              e = fast_exp2(e);
+            }
+            if (c & 1) fadd2_acc(ls[2], ls[3], a, e);
+            else fadd2_acc(ls[0], ls[1], a, e);
+            return pack_bf16x2(a, e);
+          };
+          auto release = [&](int part) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if (PAIR && !leader) mbar_arrive_remote(lbar(Lay::B_PFULL + kPSplit * s + part));
+              else mbar_arrive(bar(Lay::B_PFULL + kPSplit * s + part));
+            }
+          };
+          uint32_t pk0[32], pk1[32];
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) pk0[cc] = pair_bf16(cc);
+          tmem_st_x32(t_s, pk0);
+          if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t ov[32];
+              tmem_ld_x32(t_o + 32 * c, ov);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tmem_st_x32(t_o + 32 * c, ov);
+            }
+          }
+#pragma unroll
+          for (int cc = 0; cc < kEarlyPairs; ++cc) pk1[cc] = pair_bf16(32 + cc);
+          release(0);
+#pragma unroll
+          for (int cc = kEarlyPairs; cc < 32; ++cc) pk1[cc] = pair_bf16(32 + cc);
+          tmem_st_x32(t_s + 32, pk1);
+          release(1);
+          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          continue;
+        }
 #pragma unroll
         for (int half = 0; half < kPSplit; ++half) {
           constexpr int PAIRS = 64 / kPSplit;  // column pairs per part
