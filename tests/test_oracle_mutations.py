@@ -1,10 +1,14 @@
 """The pins are strong enough to catch plausible mistakes: each case plants one
 mistake in a private copy of the oracle's C source (never in the oracle itself),
 builds it, and checks that a pin from test_oracle_pins.py's families fails on it
-while the real oracle passes the same check."""
+while the real oracle passes the same check.  Each case runs in a fresh Python
+process, so no mutant library shares a process (or a dlopen namespace) with the
+real oracle or with another mutant."""
 import importlib.util
 import math
 import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -107,8 +111,24 @@ MUTATIONS = [
 ]
 
 
-@pytest.mark.parametrize("name,old,new,check", MUTATIONS, ids=[m[0] for m in MUTATIONS])
-def test_pin_catches_planted_mistake(tmp_path, name, old, new, check):
-    assert check(oracle), f"the real oracle fails the {name} check"
+def _run_case(index, tmp_dir):
+    """Child-process body: print whether the real oracle and the mutant pass the check."""
+    import pathlib
+    name, old, new, check = MUTATIONS[index]
+    real = check(oracle)
     with np.errstate(all="ignore"):
-        assert not check(_mutant(tmp_path, old, new)), f"{name} went unnoticed"
+        mutant = check(_mutant(pathlib.Path(tmp_dir), old, new))
+    print(f"RESULT real={int(real)} mutant={int(mutant)}")
+
+
+@pytest.mark.parametrize("index", range(len(MUTATIONS)), ids=[m[0] for m in MUTATIONS])
+def test_pin_catches_planted_mistake(tmp_path, index):
+    name = MUTATIONS[index][0]
+    code = ("import sys; sys.path[:0] = [sys.argv[1], sys.argv[2]]; "
+            "import test_oracle_mutations as t; t._run_case(int(sys.argv[3]), sys.argv[4])")
+    run = subprocess.run([sys.executable, "-c", code, ROOT, os.path.join(ROOT, "tests"),
+                          str(index), str(tmp_path)], capture_output=True, text=True, timeout=300)
+    out = [ln for ln in run.stdout.splitlines() if ln.startswith("RESULT ")]
+    assert run.returncode == 0 and out, f"{name}: child failed\n{run.stdout}\n{run.stderr}"
+    assert out[-1].split()[1] == "real=1", f"the real oracle fails the {name} check"
+    assert out[-1].split()[2] == "mutant=0", f"{name} went unnoticed"
