@@ -6,12 +6,14 @@
 // two sub-tiles while the other one's softmax runs ("FlashAttention V4 deep-dive"
 // (pnsm.cn), section 3.1, two Q tiles in ping-pong).
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads; warps 0-7 run with 192 registers, warps 8-11 with 120,
+// moved by setmaxnreg after the set-up):
 //   warps 0-3   softmax + epilogue of sub-tile 0 (one query row per thread)
 //   warps 4-7   softmax + epilogue of sub-tile 1
 //   warp  8     TMA producer: Q pair, then K_j / V_j tiles into an smem ring
 //   warp  9     TMEM owner and tcgen05.mma issuer (whole warp; one elected lane
 //               issues each instruction)
+//   warps 10-11 no role: they complete warpgroup 2, whose registers go to 0-7
 //
 // Per sub-tile s and key tile j ("FlashAttention 1-4 详解", FlashAttention 1 /
 // Online Softmax 数学推导; FlashAttention 2 / 减少非矩阵乘运算占比):
@@ -22,12 +24,16 @@
 //        FlashAttention 4 / 三项核心技术 (2)): O_s, l scaled by 2^(m_ref - m)
 //   P~  = 2^(scale*S*log2e - m_ref)    MUFU ex2, or for POLY of every 8 column pairs
 //       the FMA-pipe polynomial ("FlashAttention V4 deep-dive", section 3.2);
-//       l += sum P~ (fp32, before rounding)
+//       l += sum P~ (fp32, before rounding) -- the LSE's sum; the sum O is divided
+//       by takes the same fp32 P~ on a full tile and, on a tile the mask cuts,
+//       the bf16 P~ that the PV product uses (read back from TMEM; bf16 causal,
+//       unmasked and packed kernels)
 //   P~ -> bf16 (E4M3 on the 8-bit path), written back over S_s in TMEM in two
 //       halves of 64 keys, each released to the MMA warp as soon as it is stored
 //   O_s += P~ V_j                      tcgen05.mma, A = P~ from TMEM, B = V from smem,
 //                                      issued per half of P~
-// after the last key tile: O = O_s / l -> bf16 -> global; LSE = ln2*(m_ref + log2 l).
+// after the last key tile: O = O_s / (that second sum) -> bf16 -> global;
+// LSE = ln2*(m_ref + log2 l).
 // The mask hook (MaskFn below) decides which key tiles an item visits and which
 // keys of a tile are hidden: causal items skip key tiles above the diagonal
 // ("FlashAttention 1-4 详解", 其他优化 / FlashAttention 2 的工程优化) and mask the
@@ -58,7 +64,7 @@ namespace attn {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kBM = 128;  // query rows per sub-tile
 constexpr int kBN = 128;  // keys per key tile
 constexpr float kLn2 = 0.693147180559945309f;
@@ -557,6 +563,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     return idx;
   };
 
+  // Registers move from warpgroup 2 (producer, MMA issuer, two idle warps) to the
+  // two softmax warpgroups.  The launch gives every thread 168 (three warps share
+  // each SM sub-partition); 4 x 32 x (168 - 120) = 6144 are released and
+  // 8 x 32 x (192 - 168) = 6144 taken, so the increase always finds its registers.
+  if (warp >= 8) asm volatile("setmaxnreg.dec.sync.aligned.u32 120;\n" ::: "memory");
+  else asm volatile("setmaxnreg.inc.sync.aligned.u32 192;\n" ::: "memory");
+
   if (warp < 8) {
     // ------------------------------------------------------------ softmax
     // Sub-tile s = warp / 4; warp w owns TMEM lanes 32(w%4)..+31: one query row per
@@ -579,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (jhi <= jlo) continue;
       const int row0 = it.row_base + s * SUB + static_cast<int>(rank) * kBM;  // this CTA's rows
       const int q_row = row0 + r;
-      float m_ref = -INFINITY, l = 0.f;
+      float m_ref = -INFINITY, l = 0.f, lr = 0.f;  // lr: the row sum O is divided by
       bool ok = true;
       for (int j = jlo; j < jhi; ++j) {
         ok = mbar_wait(bar(Lay::B_SFULL + s), s_phase, wc, timeout_code(kSiteSFull));
@@ -638,6 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             alpha = fast_exp2(m_ref - m_tile);
             m_ref = m_tile;
             l *= alpha;
+            lr *= alpha;
             ++n_rescale;
           }
         }
@@ -649,6 +663,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         float nm = (MASK == kMaskWindow && m_ref == -INFINITY) ? 0.f : -m_ref;
         if constexpr (F8) nm += p.p_shift;  // P~ * 2^p_shift <= 256 stays in E4M3's range
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        // On a tile the mask cuts for this sub-tile, the sum O is divided by is
+        // taken over the bf16 P~ the PV product uses, read back from TMEM after
+        // the stores (every score and P~ register is dead by then).  Not in the
+        // sliding-window kernels: there the read-back costs the softmax loop its
+        // registers, and their rows keep the fp32 sum.
+        constexpr bool RSUM = !F8 && MASK != kMaskWindow;
+        auto rounded_sum = [&]() -> float {
+          tmem_st_wait();
+          uint32_t pr[64];
+          tmem_ld_x64(t_s, pr);
+          float q0 = 0.f, q1 = 0.f;
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            fadd2_acc(q0, q1, __uint_as_float(pr[i] << 16), __uint_as_float(pr[i] & 0xffff0000u));
+          return q0 + q1;
+        };
         if constexpr (!F8 && kPSplit == 2 && kEarlyPairs > 0) {
           // bf16, two parts: the first pairs of the second part are computed before
           // waiting for the first part's TMEM store, so that wait returns at once.
@@ -667,13 +697,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             else fadd2_acc(ls[0], ls[1], a, e);
             return pack_bf16x2(a, e);
           };
-          auto release = [&](int part) {
+          auto release = [&](int half) {
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-              if (PAIR && !leader) mbar_arrive_remote(lbar(Lay::B_PFULL + kPSplit * s + part));
-              else mbar_arrive(bar(Lay::B_PFULL + kPSplit * s + part));
+              if (PAIR && !leader) mbar_arrive_remote(lbar(Lay::B_PFULL + kPSplit * s + half));
+              else mbar_arrive(bar(Lay::B_PFULL + kPSplit * s + half));
             }
           };
           uint32_t pk0[32], pk1[32];
@@ -696,10 +726,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int cc = kEarlyPairs; cc < 32; ++cc) pk1[cc] = pair_bf16(32 + cc);
           tmem_st_x32(t_s + 32, pk1);
+          const float lq = (RSUM && part) ? rounded_sum() : 0.f;
           release(1);
-          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          const float lt = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          l += lt;
+          lr += (RSUM && part) ? lq : lt;
           continue;
         }
+        float lq_gen = 0.f;
 #pragma unroll
         for (int half = 0; half < kPSplit; ++half) {
           constexpr int PAIRS = 64 / kPSplit;  // column pairs per part
@@ -759,6 +793,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
+          if constexpr (RSUM) {
+            if (half == kPSplit - 1 && part) lq_gen = rounded_sum();
+          }
           tmem_st_wait();
           // One arrival per warp: every lane's TMEM stores are complete (wait::st)
           // and fenced before the warp converges; lane 0 then releases them.
@@ -769,7 +806,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             else mbar_arrive(bar(Lay::B_PFULL + kPSplit * s + half));
           }
         }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        const float lt = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        l += lt;
+        lr += (RSUM && part) ? lq_gen : lt;
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
@@ -778,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       o_phase ^= 1u;
       tc_fence_after();
-      float inv = 1.f / l;
+      float inv = 1.f / lr;
       if constexpr (F8) inv *= p.o_scale;  // V's per-tensor scale
       const bool store = q_row < L;
       __nv_bfloat16* dst =
@@ -958,7 +997,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(bar(Lay::B_KVFULL + n % NS), (n / NS) & 1u, kDrainLimitNs);
       if (n_items > 0) drain_wait(bar(Lay::B_QFULL), (n_items - 1) & 1u, kDrainLimitNs);
     }
-  } else if (leader) {
+  } else if (warp == 9 && leader) {
     // ---------------------------------------------------------------- MMA
     // (a pair's follower has no MMA role: the leader issues the pair's products)
     // The whole warp walks the loop and waits; one elected lane issues each MMA

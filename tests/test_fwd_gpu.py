@@ -250,8 +250,9 @@ def test_fwd_full_workload_whole_output(name, poly):
 def test_fwd_varlen_workload_every_item():
     """The packed causal workload (16 sequences, 125 841 tokens): every output written
     (NaN-prefilled buffers), one random row of EVERY (sequence, head, 128-row
-    sub-tile) plus each sequence's first and last rows compared with the oracle,
-    and a second launch bitwise equal to the first."""
+    sub-tile), each sequence's first 16 rows (they average the fewest keys, so |O|
+    and the rounding error are largest there) and its last row compared with the
+    oracle under the raw max-abs bar, and a second launch bitwise equal to the first."""
     w = ai.VARLEN
     (q, k, v), o, lse = _run_workload(w)
     rng = np.random.default_rng(7)
@@ -259,7 +260,7 @@ def test_fwd_varlen_workload_every_item():
     rows, heads = [], []
     for b, L in enumerate(w.seq_lengths()):
         for h in range(w.H):
-            picks = {0, L - 1}
+            picks = set(range(min(16, L))) | {L - 1}
             for t0 in range(0, L, 128):
                 picks.add(int(rng.integers(t0, min(t0 + 128, L))))
             rows += [cu[b] + i for i in sorted(picks)]
