@@ -567,10 +567,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // two softmax warpgroups.  The launch gives every thread 168 (three warps share
   // each SM sub-partition); 4 x 32 x (168 - 120) = 6144 are released and
   // 8 x 32 x (192 - 168) = 6144 taken, so the increase always finds its registers.
-  if (warp >= 8) asm volatile("setmaxnreg.dec.sync.aligned.u32 120;\n" ::: "memory");
-  else asm volatile("setmaxnreg.inc.sync.aligned.u32 192;\n" ::: "memory");
-
+  // Each warpgroup changes its budget at one instruction at the head of its
+  // branch, so the code after it is compiled for the new budget.
   if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 192;\n" ::: "memory");
     // ------------------------------------------------------------ softmax
     // Sub-tile s = warp / 4; warp w owns TMEM lanes 32(w%4)..+31: one query row per
     // thread, all 128 key columns of each tile.
@@ -881,251 +881,254 @@ __global__ void __launch_bounds__(kThreads, 1)
       atomicAdd(p.stats, static_cast<unsigned long long>(n_rescale));
       atomicAdd(p.stats + 1, static_cast<unsigned long long>(n_rowtiles));
     }
-  } else if (warp == 8) {
-    // ----------------------------------------------------------- producer
-    // Whole warp walks the loop and waits; one elected lane issues the copies.
-    if (elect_one()) {
-      tma_prefetch_map(&tm_q);
-      tma_prefetch_map(PAIR ? &tm_k2 : &tm_k);
-      tma_prefetch_map(&tm_v);
-    }
-    __syncwarp();
-    const uint64_t pol_kv = l2_policy_evict_last();
-    const uint64_t pol_q = l2_policy_evict_first();
-    uint32_t n_ld = 0, qe_phase = 0;
-    int n_items = 0;
-    bool ok = true;
-    for (int k = 0; ok; ++k) {
-      // Claim the next list position once its queue entry is free, and publish it
-      // (to both CTAs of a pair; the follower's producer takes it like the other roles).
-      const int e = k & 1;
-      int idx = -1;
-      if (PAIR && !leader) {
-        idx = take_item(k);
-      } else {
-        if (k >= 2) {
-          ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_ITEME + e), ((k >> 1) - 1) & 1, wc,
-                                                       timeout_code(kSiteItemEmpty)));
-          if (!ok) break;
-        }
-        if (lane == 0) {
-          const unsigned c = atomicAdd(p.work, 1u);
-          if (c < static_cast<unsigned>(sch.count)) idx = static_cast<int>(c);
-          queue[e] = idx;
-          mbar_arrive(bar(Lay::B_ITEMF + e));
-          if constexpr (PAIR) {
-            const uint32_t qaddr = sb + Lay::MISC_OFF + 4 * (8 + e);
-            st_shared_remote_u32(mapa_shared(qaddr, 1), static_cast<uint32_t>(idx));
-            mbar_arrive_remote(mapa_shared(bar(Lay::B_ITEMF + e), 1));  // release: orders the store
-          }
-        }
-        idx = __shfl_sync(0xffffffffu, idx, 0);
-      }
-      if (idx < 0) break;
-      const Item it = sch.template decode<SPLIT>(idx);
-      const int h = it.h, seq_start = it.seq_start;
-      int jlo, nkv;
-      item_range<MASK, SUB>(it, mk, jlo, nkv);
-      if (k > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QEMPTY), qe_phase, wc, timeout_code(kSiteQEmpty)));
-        if (!ok) break;
-        qe_phase ^= 1u;
-      }
-      // Failure-path test: the first query tile's copy is never issued, so its
-      // consumers' waits run out.
-      const bool withhold = p.test_fault == 1 && k == 0;
-      if (!withhold && elect_one()) {
-        // Each CTA loads its own query rows; the leader counts the pair's bytes.
-        if (leader) mbar_arrive_expect_tx(bar(Lay::B_QFULL), (PAIR ? 4 : 2) * Lay::TILE);
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          const int qr = seq_start + it.row_base + s * SUB + static_cast<int>(rank) * kBM;
-#pragma unroll
-          for (int c = 0; c < Lay::NCHUNK; ++c) {
-            const uint32_t dst = sb + Lay::Q_OFF + s * Lay::TILE + c * Lay::CHUNK;
-            if constexpr (PAIR) tma_load_3d_pair(dst, &tm_q, lbar(Lay::B_QFULL), c * 64, h, qr, pol_q);
-            else tma_load_3d(dst, &tm_q, bar(Lay::B_QFULL), c * (128 / Lay::ESZ), h, qr, pol_q);
-          }
-        }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 120;\n" ::: "memory");
+    if (warp == 8) {
+      // ----------------------------------------------------------- producer
+      // Whole warp walks the loop and waits; one elected lane issues the copies.
+      if (elect_one()) {
+        tma_prefetch_map(&tm_q);
+        tma_prefetch_map(PAIR ? &tm_k2 : &tm_k);
+        tma_prefetch_map(&tm_v);
       }
       __syncwarp();
-      if (!withhold) ++n_items;
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int key0 = seq_start + (jlo + j) * kBN;
-#pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          const uint32_t slot = n_ld % NS;
-          if (n_ld >= static_cast<uint32_t>(NS)) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KVEMPTY + slot), ((n_ld / NS) - 1) & 1u,
-                                                   wc, timeout_code(kSiteKvEmpty)));
+      const uint64_t pol_kv = l2_policy_evict_last();
+      const uint64_t pol_q = l2_policy_evict_first();
+      uint32_t n_ld = 0, qe_phase = 0;
+      int n_items = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        // Claim the next list position once its queue entry is free, and publish it
+        // (to both CTAs of a pair; the follower's producer takes it like the other roles).
+        const int e = k & 1;
+        int idx = -1;
+        if (PAIR && !leader) {
+          idx = take_item(k);
+        } else {
+          if (k >= 2) {
+            ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_ITEME + e), ((k >> 1) - 1) & 1, wc,
+                                                         timeout_code(kSiteItemEmpty)));
             if (!ok) break;
           }
-          if (elect_one()) {
-            const uint32_t dst = sb + Lay::KV_OFF + slot * Lay::SLOT;
+          if (lane == 0) {
+            const unsigned c = atomicAdd(p.work, 1u);
+            if (c < static_cast<unsigned>(sch.count)) idx = static_cast<int>(c);
+            queue[e] = idx;
+            mbar_arrive(bar(Lay::B_ITEMF + e));
             if constexpr (PAIR) {
-              // K: keys 64*rank..+63 (two 64-row boxes, one per 64 head-dim columns);
-              // V: all 128 keys, head-dim columns 64*rank..+63 (one box).
-              if (leader) mbar_arrive_expect_tx(bar(Lay::B_KVFULL + slot), 2 * Lay::SLOT);
-              if (which == 0) {
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-                  tma_load_3d_pair(dst + c * (Lay::SLOT / 2), &tm_k2, lbar(Lay::B_KVFULL + slot), c * 64, h,
-                                   key0 + static_cast<int>(rank) * 64, pol_kv);
-              } else {
-                tma_load_3d_pair(dst, &tm_v, lbar(Lay::B_KVFULL + slot), static_cast<int>(rank) * 64, h,
-                                 key0, pol_kv);
-              }
-            } else {
-              mbar_arrive_expect_tx(bar(Lay::B_KVFULL + slot), Lay::TILE);
-#pragma unroll
-              for (int c = 0; c < Lay::NCHUNK; ++c)
-                tma_load_3d(dst + c * Lay::CHUNK, which ? &tm_v : &tm_k, bar(Lay::B_KVFULL + slot),
-                            c * (128 / Lay::ESZ), h, key0, pol_kv);
+              const uint32_t qaddr = sb + Lay::MISC_OFF + 4 * (8 + e);
+              st_shared_remote_u32(mapa_shared(qaddr, 1), static_cast<uint32_t>(idx));
+              mbar_arrive_remote(mapa_shared(bar(Lay::B_ITEMF + e), 1));  // release: orders the store
             }
           }
-          __syncwarp();
-          ++n_ld;
+          idx = __shfl_sync(0xffffffffu, idx, 0);
+        }
+        if (idx < 0) break;
+        const Item it = sch.template decode<SPLIT>(idx);
+        const int h = it.h, seq_start = it.seq_start;
+        int jlo, nkv;
+        item_range<MASK, SUB>(it, mk, jlo, nkv);
+        if (k > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_QEMPTY), qe_phase, wc, timeout_code(kSiteQEmpty)));
+          if (!ok) break;
+          qe_phase ^= 1u;
+        }
+        // Failure-path test: the first query tile's copy is never issued, so its
+        // consumers' waits run out.
+        const bool withhold = p.test_fault == 1 && k == 0;
+        if (!withhold && elect_one()) {
+          // Each CTA loads its own query rows; the leader counts the pair's bytes.
+          if (leader) mbar_arrive_expect_tx(bar(Lay::B_QFULL), (PAIR ? 4 : 2) * Lay::TILE);
+#pragma unroll
+          for (int s = 0; s < 2; ++s) {
+            const int qr = seq_start + it.row_base + s * SUB + static_cast<int>(rank) * kBM;
+#pragma unroll
+            for (int c = 0; c < Lay::NCHUNK; ++c) {
+              const uint32_t dst = sb + Lay::Q_OFF + s * Lay::TILE + c * Lay::CHUNK;
+              if constexpr (PAIR) tma_load_3d_pair(dst, &tm_q, lbar(Lay::B_QFULL), c * 64, h, qr, pol_q);
+              else tma_load_3d(dst, &tm_q, bar(Lay::B_QFULL), c * (128 / Lay::ESZ), h, qr, pol_q);
+            }
+          }
+        }
+        __syncwarp();
+        if (!withhold) ++n_items;
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int key0 = seq_start + (jlo + j) * kBN;
+#pragma unroll
+          for (int which = 0; which < 2; ++which) {
+            const uint32_t slot = n_ld % NS;
+            if (n_ld >= static_cast<uint32_t>(NS)) {
+              ok = __all_sync(0xffffffffu, mbar_wait(bar(Lay::B_KVEMPTY + slot), ((n_ld / NS) - 1) & 1u,
+                                                     wc, timeout_code(kSiteKvEmpty)));
+              if (!ok) break;
+            }
+            if (elect_one()) {
+              const uint32_t dst = sb + Lay::KV_OFF + slot * Lay::SLOT;
+              if constexpr (PAIR) {
+                // K: keys 64*rank..+63 (two 64-row boxes, one per 64 head-dim columns);
+                // V: all 128 keys, head-dim columns 64*rank..+63 (one box).
+                if (leader) mbar_arrive_expect_tx(bar(Lay::B_KVFULL + slot), 2 * Lay::SLOT);
+                if (which == 0) {
+#pragma unroll
+                  for (int c = 0; c < 2; ++c)
+                    tma_load_3d_pair(dst + c * (Lay::SLOT / 2), &tm_k2, lbar(Lay::B_KVFULL + slot), c * 64, h,
+                                     key0 + static_cast<int>(rank) * 64, pol_kv);
+                } else {
+                  tma_load_3d_pair(dst, &tm_v, lbar(Lay::B_KVFULL + slot), static_cast<int>(rank) * 64, h,
+                                   key0, pol_kv);
+                }
+              } else {
+                mbar_arrive_expect_tx(bar(Lay::B_KVFULL + slot), Lay::TILE);
+#pragma unroll
+                for (int c = 0; c < Lay::NCHUNK; ++c)
+                  tma_load_3d(dst + c * Lay::CHUNK, which ? &tm_v : &tm_k, bar(Lay::B_KVFULL + slot),
+                              c * (128 / Lay::ESZ), h, key0, pol_kv);
+              }
+            }
+            __syncwarp();
+            ++n_ld;
+          }
         }
       }
-    }
-    // Drain: every issued copy must have landed before the CTA may exit (a pair's
-    // copies all complete on the leader's barriers; the leader drains them, and
-    // the pair waits for each other before exiting).
-    if (leader) {
-      const uint32_t first = n_ld > static_cast<uint32_t>(NS) ? n_ld - NS : 0u;
-      for (uint32_t n = first; n < n_ld; ++n)
-        drain_wait(bar(Lay::B_KVFULL + n % NS), (n / NS) & 1u, kDrainLimitNs);
-      if (n_items > 0) drain_wait(bar(Lay::B_QFULL), (n_items - 1) & 1u, kDrainLimitNs);
-    }
-  } else if (warp == 9 && leader) {
-    // ---------------------------------------------------------------- MMA
-    // (a pair's follower has no MMA role: the leader issues the pair's products)
-    // The whole warp walks the loop and waits; one elected lane issues each MMA
-    // and commit.  Issue order per key tile j (ping-pong of the two sub-tiles):
-    //   PV(0, j-1), S(0, j), PV(1, j-1), S(1, j)
-    // each only where tile j (j-1) lies in that sub-tile's key range.
-    // S(s, j) overwrites P(s, j-1) in TMEM, which PV(s, j-1) read just before; the
-    // tensor pipe executes one thread's MMAs in issue order.
-    constexpr int M = PAIR ? 2 * kBM : kBM;  // rows of one product (a pair: 128 in each CTA)
-    constexpr uint32_t idesc_s = F8 ? idesc_e4m3_f32(M, kBN, 0, 0) : idesc_bf16_f32(M, kBN, 0, 0);
-    constexpr uint32_t idesc_o = F8 ? idesc_e4m3_f32(M, D, 0, 1) : idesc_bf16_f32(M, D, 0, 1);
-    // Commit to this CTA's barrier, or to the barrier at the same offset in both
-    // CTAs of a pair.
-    auto commit = [&](int i) {
-      if constexpr (PAIR) tc_commit_pair(bar(i), 0x3);
-      else tc_commit(bar(i));
-    };
-    const uint32_t tS0 = tmem + Lay::TM_S0, tS1 = tmem + Lay::TM_S1;
-    const uint32_t tO0 = tmem + Lay::TM_O0, tO1 = tmem + Lay::TM_O1;
-    uint32_t n_ld = 0, q_phase = 0, p_phase0 = 0, p_phase1 = 0;
-    bool ok = true;
-    for (int k = 0; ok; ++k) {
-      const int idx = take_item(k);
-      if (idx < 0) break;
-      const Item it = sch.template decode<SPLIT>(idx);
-      int jlo, nkv, lo0, hi0, lo1, hi1;
-      item_range<MASK, SUB>(it, mk, jlo, nkv);
-      kv_range<MASK, SUB>(it, 0, mk, lo0, hi0);
-      kv_range<MASK, SUB>(it, 1, mk, lo1, hi1);
-      ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_QFULL), q_phase, wc, timeout_code(kSiteQFull)));
-      if (!ok) break;
-      q_phase ^= 1u;
-      tc_fence_after();
-      for (int jj = 0; jj <= nkv && ok; ++jj) {
-        const int j = jlo + jj;              // key tile
-        const uint32_t nK = n_ld + 2u * jj;  // load sequence number of K_j
-        const uint32_t nV = nK - 1u;        // ... and of V_{j-1}
-        const uint32_t slotK = nK % NS, slotV = nV % NS;
-        if (jj < nkv)
-          ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_KVFULL + slotK), (nK / NS) & 1u, wc,
-                                                       timeout_code(kSiteKvFull)));
-        if (ok && jj > 0)
-          ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_KVFULL + slotV), (nV / NS) & 1u, wc,
-                                                       timeout_code(kSiteKvFull)));
+      // Drain: every issued copy must have landed before the CTA may exit (a pair's
+      // copies all complete on the leader's barriers; the leader drains them, and
+      // the pair waits for each other before exiting).
+      if (leader) {
+        const uint32_t first = n_ld > static_cast<uint32_t>(NS) ? n_ld - NS : 0u;
+        for (uint32_t n = first; n < n_ld; ++n)
+          drain_wait(bar(Lay::B_KVFULL + n % NS), (n / NS) & 1u, kDrainLimitNs);
+        if (n_items > 0) drain_wait(bar(Lay::B_QFULL), (n_items - 1) & 1u, kDrainLimitNs);
+      }
+    } else if (warp == 9 && leader) {
+      // ---------------------------------------------------------------- MMA
+      // (a pair's follower has no MMA role: the leader issues the pair's products)
+      // The whole warp walks the loop and waits; one elected lane issues each MMA
+      // and commit.  Issue order per key tile j (ping-pong of the two sub-tiles):
+      //   PV(0, j-1), S(0, j), PV(1, j-1), S(1, j)
+      // each only where tile j (j-1) lies in that sub-tile's key range.
+      // S(s, j) overwrites P(s, j-1) in TMEM, which PV(s, j-1) read just before; the
+      // tensor pipe executes one thread's MMAs in issue order.
+      constexpr int M = PAIR ? 2 * kBM : kBM;  // rows of one product (a pair: 128 in each CTA)
+      constexpr uint32_t idesc_s = F8 ? idesc_e4m3_f32(M, kBN, 0, 0) : idesc_bf16_f32(M, kBN, 0, 0);
+      constexpr uint32_t idesc_o = F8 ? idesc_e4m3_f32(M, D, 0, 1) : idesc_bf16_f32(M, D, 0, 1);
+      // Commit to this CTA's barrier, or to the barrier at the same offset in both
+      // CTAs of a pair.
+      auto commit = [&](int i) {
+        if constexpr (PAIR) tc_commit_pair(bar(i), 0x3);
+        else tc_commit(bar(i));
+      };
+      const uint32_t tS0 = tmem + Lay::TM_S0, tS1 = tmem + Lay::TM_S1;
+      const uint32_t tO0 = tmem + Lay::TM_O0, tO1 = tmem + Lay::TM_O1;
+      uint32_t n_ld = 0, q_phase = 0, p_phase0 = 0, p_phase1 = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = take_item(k);
+        if (idx < 0) break;
+        const Item it = sch.template decode<SPLIT>(idx);
+        int jlo, nkv, lo0, hi0, lo1, hi1;
+        item_range<MASK, SUB>(it, mk, jlo, nkv);
+        kv_range<MASK, SUB>(it, 0, mk, lo0, hi0);
+        kv_range<MASK, SUB>(it, 1, mk, lo1, hi1);
+        ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_QFULL), q_phase, wc, timeout_code(kSiteQFull)));
         if (!ok) break;
+        q_phase ^= 1u;
         tc_fence_after();
+        for (int jj = 0; jj <= nkv && ok; ++jj) {
+          const int j = jlo + jj;              // key tile
+          const uint32_t nK = n_ld + 2u * jj;  // load sequence number of K_j
+          const uint32_t nV = nK - 1u;        // ... and of V_{j-1}
+          const uint32_t slotK = nK % NS, slotV = nV % NS;
+          if (jj < nkv)
+            ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_KVFULL + slotK), (nK / NS) & 1u, wc,
+                                                         timeout_code(kSiteKvFull)));
+          if (ok && jj > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_KVFULL + slotV), (nV / NS) & 1u, wc,
+                                                         timeout_code(kSiteKvFull)));
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          const uint32_t tS = s ? tS1 : tS0, tO = s ? tO1 : tO0;
-          const int los = s ? lo1 : lo0, his = s ? hi1 : hi0;
-          if (ok && jj > 0 && j - 1 >= los && j - 1 < his) {
-            uint32_t& ph = s ? p_phase1 : p_phase0;
-            const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::SLOT;
-            constexpr int NK = kBN / Lay::KSTEP;  // PV K steps per key tile
-            // Each part of P~ is multiplied as soon as the softmax warps release it.
-            // One K step: KSTEP keys = 32 bytes of a P~ row (8 TMEM columns) and
-            // KSTEP rows of V (128 bytes each).
-            static_assert(NK % kPSplit == 0, "K steps per part");
+          for (int s = 0; s < 2; ++s) {
+            const uint32_t tS = s ? tS1 : tS0, tO = s ? tO1 : tO0;
+            const int los = s ? lo1 : lo0, his = s ? hi1 : hi0;
+            if (ok && jj > 0 && j - 1 >= los && j - 1 < his) {
+              uint32_t& ph = s ? p_phase1 : p_phase0;
+              const uint32_t vbase = sb + Lay::KV_OFF + slotV * Lay::SLOT;
+              constexpr int NK = kBN / Lay::KSTEP;  // PV K steps per key tile
+              // Each part of P~ is multiplied as soon as the softmax warps release it.
+              // One K step: KSTEP keys = 32 bytes of a P~ row (8 TMEM columns) and
+              // KSTEP rows of V (128 bytes each).
+              static_assert(NK % kPSplit == 0, "K steps per part");
 #pragma unroll
-            for (int half = 0; half < kPSplit && ok; ++half) {
-              ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_PFULL + kPSplit * s + half), ph, wc,
-                                                           timeout_code(kSitePFull)));
-              if (!ok) break;
-              tc_fence_after();
-              // The part's K steps are issued back to back by one elected lane.
-              if (elect_one()) {
-                // V (a pair: this CTA's 64 head-dim columns of it) is MN-major.
-                const uint64_t dv0 = sdesc_sw128(vbase, Lay::CHUNK, 1024);
+              for (int half = 0; half < kPSplit && ok; ++half) {
+                ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(bar(Lay::B_PFULL + kPSplit * s + half), ph, wc,
+                                                             timeout_code(kSitePFull)));
+                if (!ok) break;
+                tc_fence_after();
+                // The part's K steps are issued back to back by one elected lane.
+                if (elect_one()) {
+                  // V (a pair: this CTA's 64 head-dim columns of it) is MN-major.
+                  const uint64_t dv0 = sdesc_sw128(vbase, Lay::CHUNK, 1024);
 #pragma unroll
-                for (int kk = half * NK / kPSplit; kk < (half + 1) * NK / kPSplit; ++kk) {
-                  const uint64_t dv = desc_add(dv0, kk * Lay::KSTEP * 128);
-                  const uint32_t acc = (j - 1 > los || kk > 0) ? 1u : 0u;
-                  if constexpr (PAIR) mma_ts_pair(tO, tS + kk * 8, dv, idesc_o, acc);
-                  else if constexpr (F8) mma_ts_f8(tO, tS + kk * 8, dv, idesc_o, acc);
-                  else mma_ts(tO, tS + kk * 8, dv, idesc_o, acc);
+                  for (int kk = half * NK / kPSplit; kk < (half + 1) * NK / kPSplit; ++kk) {
+                    const uint64_t dv = desc_add(dv0, kk * Lay::KSTEP * 128);
+                    const uint32_t acc = (j - 1 > los || kk > 0) ? 1u : 0u;
+                    if constexpr (PAIR) mma_ts_pair(tO, tS + kk * 8, dv, idesc_o, acc);
+                    else if constexpr (F8) mma_ts_f8(tO, tS + kk * 8, dv, idesc_o, acc);
+                    else mma_ts(tO, tS + kk * 8, dv, idesc_o, acc);
+                  }
                 }
+                __syncwarp();
+              }
+              if (ok) {
+                ph ^= 1u;
+                if (j == his) {
+                  if (elect_one()) commit(Lay::B_OFULL + s);
+                  __syncwarp();
+                }
+              }
+            }
+            if (ok && j >= los && j < his) {
+              const uint32_t qbase = sb + Lay::Q_OFF + s * Lay::TILE;
+              const uint32_t kbase = sb + Lay::KV_OFF + slotK * Lay::SLOT;
+              // K's rows (a pair: this CTA's 64 keys) in 128-byte chunks of head dims.
+              constexpr int KCHUNK = PAIR ? Lay::SLOT / 2 : Lay::CHUNK;
+              if (elect_one()) {
+                const uint64_t da0 = sdesc_sw128(qbase, 16, 1024);
+                const uint64_t db0 = sdesc_sw128(kbase, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / Lay::KSTEP; ++kk) {
+                  const uint64_t da = desc_add(da0, (kk >> 2) * Lay::CHUNK + (kk & 3) * 32);
+                  const uint64_t db = desc_add(db0, (kk >> 2) * KCHUNK + (kk & 3) * 32);
+                  if constexpr (PAIR) mma_ss_pair(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
+                  else if constexpr (F8) mma_ss_f8(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
+                  else mma_ss(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                commit(Lay::B_SFULL + s);
               }
               __syncwarp();
             }
-            if (ok) {
-              ph ^= 1u;
-              if (j == his) {
-                if (elect_one()) commit(Lay::B_OFULL + s);
-                __syncwarp();
-              }
-            }
           }
-          if (ok && j >= los && j < his) {
-            const uint32_t qbase = sb + Lay::Q_OFF + s * Lay::TILE;
-            const uint32_t kbase = sb + Lay::KV_OFF + slotK * Lay::SLOT;
-            // K's rows (a pair: this CTA's 64 keys) in 128-byte chunks of head dims.
-            constexpr int KCHUNK = PAIR ? Lay::SLOT / 2 : Lay::CHUNK;
-            if (elect_one()) {
-              const uint64_t da0 = sdesc_sw128(qbase, 16, 1024);
-              const uint64_t db0 = sdesc_sw128(kbase, 16, 1024);
-#pragma unroll
-              for (int kk = 0; kk < D / Lay::KSTEP; ++kk) {
-                const uint64_t da = desc_add(da0, (kk >> 2) * Lay::CHUNK + (kk & 3) * 32);
-                const uint64_t db = desc_add(db0, (kk >> 2) * KCHUNK + (kk & 3) * 32);
-                if constexpr (PAIR) mma_ss_pair(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
-                else if constexpr (F8) mma_ss_f8(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
-                else mma_ss(tS, da, db, idesc_s, kk > 0 ? 1u : 0u);
-              }
-              commit(Lay::B_SFULL + s);
-            }
-            __syncwarp();
+          if (!ok) break;
+          if (elect_one()) {
+            if (jj < nkv) commit(Lay::B_KVEMPTY + slotK);
+            if (jj > 0) commit(Lay::B_KVEMPTY + slotV);
+            // The query tiles are free after the item's last S product (an item
+            // without key tiles -- an empty half item -- frees them at once).
+            if (jj == (nkv > 0 ? nkv - 1 : 0)) commit(Lay::B_QEMPTY);
           }
+          __syncwarp();
         }
-        if (!ok) break;
-        if (elect_one()) {
-          if (jj < nkv) commit(Lay::B_KVEMPTY + slotK);
-          if (jj > 0) commit(Lay::B_KVEMPTY + slotV);
-          // The query tiles are free after the item's last S product (an item
-          // without key tiles -- an empty half item -- frees them at once).
-          if (jj == (nkv > 0 ? nkv - 1 : 0)) commit(Lay::B_QEMPTY);
-        }
-        __syncwarp();
+        n_ld += 2u * nkv;
       }
-      n_ld += 2u * nkv;
+      // Drain: every MMA issued by this warp completes before TMEM is freed.
+      if (elect_one()) {
+        if constexpr (PAIR) tc_commit_pair(bar(Lay::B_DRAIN), 0x1);
+        else tc_commit(bar(Lay::B_DRAIN));
+      }
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, kDrainLimitNs)) && lane == 0 && p.err)
+        atomicCAS(p.err, 0, timeout_code(kSiteDrain));
     }
-    // Drain: every MMA issued by this warp completes before TMEM is freed.
-    if (elect_one()) {
-      if constexpr (PAIR) tc_commit_pair(bar(Lay::B_DRAIN), 0x1);
-      else tc_commit(bar(Lay::B_DRAIN));
-    }
-    __syncwarp();
-    if (!__all_sync(0xffffffffu, drain_wait(bar(Lay::B_DRAIN), 0u, kDrainLimitNs)) && lane == 0 && p.err)
-      atomicCAS(p.err, 0, timeout_code(kSiteDrain));
   }
 
   tc_fence_before();
