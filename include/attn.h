@@ -79,6 +79,11 @@ typedef enum {
  * Online softmax: "FlashAttention 1-4 详解", FlashAttention 1 / Online Softmax
  * 数学推导, with deferred normalisation (FlashAttention 2 / 减少非矩阵乘运算占比)
  * and the conditional rescale of "FlashAttention V4 deep-dive", section 3.2.
+ * The probabilities enter the P V product as bf16.  O is divided by the sum of
+ * those bf16 values over key tiles the mask cuts (the causal diagonal, a
+ * sequence's last tile) and of the unrounded fp32 values over full tiles, so
+ * rows whose keys all lie in cut tiles get exactly the weights applied to V.
+ * Sliding-window calls use the fp32 sum throughout.  LSE always uses the fp32 sum.
  * The result does not depend on how the work is scheduled: each output row is
  * produced by one CTA with a fixed key order, so repeated calls are bitwise equal.
  */
