@@ -337,6 +337,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p) {
   using Lay = DkdvLayout<D>;
+  // The dQ kernel that follows reads nothing this kernel writes: let it be
+  // scheduled onto SMs as they free up in this grid's last wave.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   BwdItem it;
   constexpr bool CAUSAL = MASK == 1;
   if (!decode_block(p, true, CAUSAL, it)) return;  // uniform for the CTA
@@ -674,7 +677,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   using Lay = DqLayout<D>;
   BwdItem it;
   constexpr bool CAUSAL = MASK == 1;
-  if (!decode_block(p, false, CAUSAL, it)) return;  // uniform for the CTA
+  if (!decode_block(p, false, CAUSAL, it)) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    return;
+  }  // uniform for the CTA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -912,6 +918,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 9) tmem_dealloc(tmem, 512);
+  // Launched to overlap the dK/dV kernel's tail: finish only after that grid has
+  // (its results are then visible to whatever the stream runs next).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 template <int D, int MASK>
@@ -926,8 +935,17 @@ cudaError_t launch_main(const BwdLaunch& a, cudaStream_t st) {
   k1<<<a.grid, kThreads, smem1, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k2<<<a.grid, kThreads, smem2, st>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = a.grid;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem2;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k2, a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.p);
 }
 
 }  // namespace
