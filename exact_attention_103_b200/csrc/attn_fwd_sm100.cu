@@ -26,8 +26,8 @@
 //       the FMA-pipe polynomial ("FlashAttention V4 deep-dive", section 3.2);
 //       l += sum P~ (fp32, before rounding) -- the LSE's sum; the sum O is divided
 //       by takes the same fp32 P~ on a full tile and, on a tile the mask cuts,
-//       the bf16 P~ that the PV product uses (read back from TMEM; bf16 causal,
-//       unmasked and packed kernels)
+//       the bf16 P~ that the PV product uses (read back from TMEM; bf16 causal
+//       kernels and d = 128 unmasked ones)
 //   P~ -> bf16 (E4M3 on the 8-bit path), written back over S_s in TMEM in two
 //       halves of 64 keys, each released to the MMA warp as soon as it is stored
 //   O_s += P~ V_j                      tcgen05.mma, A = P~ from TMEM, B = V from smem,
@@ -666,9 +666,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // On a tile the mask cuts for this sub-tile, the sum O is divided by is
         // taken over the bf16 P~ the PV product uses, read back from TMEM after
         // the stores (every score and P~ register is dead by then).  Not in the
-        // sliding-window kernels: there the read-back costs the softmax loop its
-        // registers, and their rows keep the fp32 sum.
-        constexpr bool RSUM = !F8 && MASK != kMaskWindow;
+        // sliding-window kernels nor the unmasked d = 64 ones: there the read-back
+        // costs the softmax loop its registers, and their rows keep the fp32 sum.
+        constexpr bool RSUM = !F8 && MASK != kMaskWindow && !(D == 64 && MASK == kMaskNone);
         auto rounded_sum = [&]() -> float {
           tmem_st_wait();
           uint32_t pr[64];

@@ -83,7 +83,8 @@ typedef enum {
  * those bf16 values over key tiles the mask cuts (the causal diagonal, a
  * sequence's last tile) and of the unrounded fp32 values over full tiles, so
  * rows whose keys all lie in cut tiles get exactly the weights applied to V.
- * Sliding-window calls use the fp32 sum throughout.  LSE always uses the fp32 sum.
+ * Sliding-window calls and unmasked d = 64 calls use the fp32 sum throughout.  LSE
+ * always uses the fp32 sum.
  * The result does not depend on how the work is scheduled: each output row is
  * produced by one CTA with a fixed key order, so repeated calls are bitwise equal.
  */
