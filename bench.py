@@ -38,12 +38,6 @@ METRIC_E4M3 = "attention fwd TFLOP/s (e4m3 inputs, d=128, 1 B200) and % of dense
 
 
 FLUSH_BYTES = 256 << 20
-# A device-side wait placed after the L2 flush and before each timed step's start
-# event: the host has queued the step's launches by the time the event fires, so
-# the device-timed region holds device work only (the host path is timed in e2e).
-QUEUE_WAIT_CYCLES = 200_000
-TIMING = ("CUDA events on the launching stream; before each step's start event, an L2 flush and a "
-          "device wait of 200k cycles (about 0.1 ms) while the host queues the step's launches")
 MUFU_EX2_PER_CLK_PER_SM = 16  # 4 SFU lanes per SM sub-partition, 4 sub-partitions
 
 
@@ -362,7 +356,6 @@ def run_ours(args, rank, world, local):
     with ClockSampler(local) as clocks:
         for i in range(args.steps):
             flush.fill_(float(i))
-            torch.cuda._sleep(QUEUE_WAIT_CYCLES)
             starts[i].record()
             step()
             ends[i].record()
@@ -445,7 +438,6 @@ def run_ours(args, rank, world, local):
                 "e2e": e2e,
                 "gpu_launches": args.steps,
                 "clocks": clk,
-                "timing": TIMING,
                 "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
 
@@ -508,7 +500,6 @@ def run_bwd(args, rank, world, local):
     with ClockSampler(local) as clocks:
         for i in range(args.steps):
             flush.fill_(float(i))
-            torch.cuda._sleep(QUEUE_WAIT_CYCLES)
             starts[i].record()
             ea.bwd(q, k, v, o, lse, do, causal=True, scale=scale)
             ends[i].record()
@@ -530,7 +521,7 @@ def run_bwd(args, rank, world, local):
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                              "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                              "traffic": None},
-                "gpu_launches": 3 * args.steps, "clocks": clocks.summary(), "timing": TIMING}
+                "gpu_launches": 3 * args.steps, "clocks": clocks.summary()}
         print(json.dumps(line), flush=True)
 
 
